@@ -1,0 +1,406 @@
+"""Benchmark of the fused ZeRO-2 step (reduce-scatter + Adam) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Workload: a GPT-2 1.5B-shaped parameter list (48 layers, d=1600, ffn=6400,
+vocab 50257, ctx 1024; 580 tensors, 1,557,611,200 elements) packed into
+constant-size buffers of at most 500M elements (4 buckets), N = 8 simulated
+data-parallel replicas whose fp16 gradients (N(0, 1e-3) x 65536) are resident
+in HBM, fp32 master ~ N(0, 0.02), AdamW (lr 1e-3, betas 0.9/0.999, eps 1e-8,
+wd 0.01), dynamic loss scale 65536.  Synthetic, seeded data.
+
+A step = the fused kernel over the 4 buckets (every rank's partition), the
+overflow flag read back to the host, the bank commit and the loss-scale
+update.  `value` is Gparams/s (padded elements updated per second, all
+ranks); the roofline object rates the fused kernel's algorithmic HBM bytes,
+(2N + 26) per element, against the measured B200 copy bandwidth.
+
+Under torchrun with N > 1, every GPU runs its own instance of the workload
+(no exchange between GPUs: the replicas are simulated inside each GPU), the
+step time is the max over ranks, and `value` sums all ranks' elements.
+
+--impl reference times the CPU oracle (C, OpenMP) on the host cores, each
+step a bounded slice of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "fused ZeRO step: Gparams/s and achieved HBM GB/s vs B200 peak (1 GPU)"
+UNIT = "Gparams/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def bytes_per_elem(world: int) -> int:
+    """Algorithmic HBM bytes per partition element of the fused step."""
+    return 2 * world + 26
+
+
+# ----------------------------------------------------------------- helpers
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.dev), "-lms", "100"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        under_load = [x for x in sm if x >= 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(under_load), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    p = os.path.join(ROOT, "zero_sharded_optimizer_reduce_b200", "csrc", "step.cu")
+    h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(elems_per_launch: float):
+    """DRAM bytes per launch of the fused kernel from the committed ncu summary,
+    if it was taken on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "fused_step_traffic.json")
+    try:
+        d = json.load(open(p))
+    except Exception:
+        return None
+    if d.get("step_cu_sha256_16") != source_digest():
+        return None
+    return float(d["dram_bytes_per_elem"]) * elems_per_launch
+
+
+# --------------------------------------------------------------- CPU side
+
+def cpu_baseline(w: workloads.Workload, sample_elems: int, min_seconds: float = 10.0, max_seconds: float = 30.0):
+    """The oracle on this host's cores on a contiguous slice of bucket 0."""
+    import oracle
+    N = w.world
+    G = [workloads.grads(sample_elems, workloads.seed_for(w.seed, 1, k), w.grad_std, w.loss_scale)
+         for k in range(N)]
+    st = oracle.initial_state(workloads.master(sample_elems, 7 * w.seed))
+    done, t0, t = 0, time.perf_counter(), 0
+    while True:
+        t += 1
+        oracle.flat_step(G, st, w.adam, t, w.loss_scale, float(N))
+        done += sample_elems
+        el = time.perf_counter() - t0
+        if el >= min_seconds or el >= max_seconds:
+            break
+    return {"value": done / el / 1e9, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{t} oracle steps (reduce-scatter, overflow test, AdamW) over a {sample_elems:,}-element "
+                      f"slice of bucket 0 with N={N} replicas, {el:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    w = workloads.gpt2_1p5b()
+    N = w.world
+    sample = args.ref_sample
+    G = [workloads.grads(sample, workloads.seed_for(w.seed, 1, k), w.grad_std, w.loss_scale) for k in range(N)]
+    st = oracle.initial_state(workloads.master(sample, 7 * w.seed))
+    for t in range(1, args.warmup + 1):
+        oracle.flat_step(G, st, w.adam, t, w.loss_scale, float(N))
+    t0 = time.perf_counter()
+    for t in range(args.warmup + 1, args.warmup + args.steps + 1):
+        oracle.flat_step(G, st, w.adam, t, w.loss_scale, float(N))
+    el = time.perf_counter() - t0
+    value = sample * args.steps / el / 1e9
+    sample_desc = f"{sample:,}-element slice of the {w.name} workload per step (N={N})"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": {"workload": w.name, "world": N, "elems_per_step": sample,
+                                            "note": "CPU oracle on a bounded slice"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+                             "sample": sample_desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------- GPU side
+
+def fill_workload(opt, w, seed_base: int):
+    """Seeded device-side draws: gradients, master weights, parameters."""
+    import torch
+    gen = torch.Generator(device="cuda")
+    L = opt.layout
+    for b in range(L.n_buckets):
+        n = L.bucket_padded[b]
+        for k in range(w.world):
+            gen.manual_seed(workloads.seed_for(seed_base, 1, k) + 7919 * b)
+            buf = opt.grads[b][k]
+            chunk = 1 << 27
+            for o in range(0, n, chunk):
+                e = min(n, o + chunk)
+                x = torch.randn(e - o, generator=gen, device="cuda", dtype=torch.float32)
+                buf[o:e].copy_(x.mul_(w.grad_std * w.loss_scale))
+            buf[L.bucket_numel[b]:].zero_()
+        gen.manual_seed(7 * seed_base + b)
+        for o in range(0, n, 1 << 27):
+            e = min(n, o + (1 << 27))
+            x = torch.randn(e - o, generator=gen, device="cuda", dtype=torch.float32).mul_(w.master_std)
+            opt.master[b][0][o:e].copy_(x)
+        opt.master[b][0][L.bucket_numel[b]:].zero_()
+        opt.params_bank[b][0].copy_(opt.master[b][0])
+        for bank in (opt.m, opt.v):
+            bank[b][0].zero_()
+        opt.master[b][1].copy_(opt.master[b][0])
+        opt.params_bank[b][1].copy_(opt.params_bank[b][0])
+    torch.cuda.synchronize()
+
+
+def select_workload(args) -> workloads.Workload:
+    if args.flat:
+        return workloads.Workload(f"flat_{args.flat}_n{args.world}_{args.grad_dtype}", (args.flat,), args.world,
+                                  65536.0, 1, workloads.AdamConfig(weight_decay=0.01), seed=5)
+    return workloads.gpt2_1p5b()
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    import zero_sharded_optimizer_reduce_b200 as Z
+
+    world_gpus = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world_gpus > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world_gpus > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    w = select_workload(args)
+    gdt = torch.bfloat16 if args.grad_dtype == "bf16" else torch.float16
+    opt = Z.ZeroAdam(w.numels, w.world, w.bucket_elems, lr=w.adam.lr, betas=(w.adam.beta1, w.adam.beta2),
+                     eps=w.adam.eps, weight_decay=w.adam.weight_decay, loss_scale=w.loss_scale,
+                     grad_dtype=gdt, param_dtype=gdt)
+    L = opt.layout
+    psi_p = sum(L.bucket_padded)
+    fill_workload(opt, w, w.seed + 100 * rank)
+    stream = torch.cuda.current_stream()
+
+    # ---- device-timed steps
+    ev = {}
+
+    def on_launch(b, phase):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)
+        ev.setdefault(b, []).append(e)
+
+    for _ in range(args.warmup):
+        opt.step()
+    barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    ev.clear()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.profiler.start()      # ncu --profile-from-start off captures only the timed steps
+    t_start.record(stream)
+    applied = 0
+    for _ in range(args.steps):
+        applied += bool(opt.step(on_launch=on_launch))
+    t_end.record(stream)
+    barrier()
+    torch.cuda.profiler.stop()
+    clock = clocks.stop()
+    ms = t_start.elapsed_time(t_end)
+    # per-launch durations of the fused kernel
+    launch_ms, launch_elems = [], []
+    for b, es in ev.items():
+        for i in range(0, len(es), 2):
+            launch_ms.append(es[i].elapsed_time(es[i + 1]))
+            launch_elems.append(L.bucket_padded[b])
+    if world_gpus > 1:
+        tt = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    ms_per_step = ms / args.steps
+    value = world_gpus * psi_p / (ms_per_step * 1e-3) / 1e9
+    bpe = bytes_per_elem(w.world)
+    peak, peak_kind = peaks()
+    kern_bytes = sum(launch_elems) * bpe
+    kern_s = sum(launch_ms) * 1e-3
+    achieved = kern_bytes / kern_s / 1e9
+    avg_elems = sum(launch_elems) / len(launch_elems)
+    traffic = profiled_traffic(avg_elems)
+
+    # ---- end to end through the public API: host gradients in, flag out
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(opt, args, stream, barrier, world_gpus)
+
+    # ---- CPU baseline (oracle) on rank 0, single-GPU runs only
+    cpu = None
+    if rank == 0 and world_gpus == 1 and not args.no_cpu:
+        cpu = cpu_baseline(w, args.cpu_sample)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world_gpus, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic (seeded N(0,1e-3)x65536 fp16 gradients, N(0,0.02) fp32 master)",
+                "config": {"workload": w.name, "psi": sum(w.numels), "psi_padded": psi_p, "world": w.world,
+                           "buckets": L.n_buckets, "bucket_elems": w.bucket_elems, "grad_dtype": args.grad_dtype,
+                           "param_dtype": args.grad_dtype, "optimizer": "AdamW wd=0.01", "stage": 2,
+                           "parallelism": f"{world_gpus} GPU(s) x {w.world} simulated replicas",
+                           "l2": (f"inputs larger than L2: {psi_p * bpe / 1e9:.1f} GB of HBM traffic per step"
+                                  if psi_p * bpe > 4 * 126e6 else "L2-influenced (footprint < 4x L2)")},
+                "hbm_gbs": value * 1e9 * bpe / world_gpus / 1e9,
+                "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
+                             "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                             "kernel": "fused_step_kernel", "bytes_per_elem": bpe,
+                             "elems_per_launch": avg_elems, "launches_timed": len(launch_ms)},
+                "gpu_launches": args.steps * L.n_buckets,
+                "applied_steps": applied,
+                "clocks": clock,
+                "e2e": e2e,
+                "cpu_baseline": cpu}
+        print(json.dumps(line), flush=True)
+    if world_gpus > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(opt, args, stream, barrier, world_gpus):
+    """Same step through ZeroAdam.step_from_host: every step copies the N
+    replicas' gradients from pinned host memory and reads the flag back."""
+    import torch
+    try:
+        import psutil
+        need = sum(g.numel() * g.element_size() for per in opt.grads for g in per)
+        if psutil.virtual_memory().available < 1.5 * need * max(1, world_gpus):
+            return {"value": None, "unit": UNIT, "skipped": "not enough host memory for pinned gradients"}
+    except Exception:
+        pass
+    host = [[torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in per] for per in opt.grads]
+    for b, per in enumerate(opt.grads):
+        for k, g in enumerate(per):
+            host[b][k].copy_(g)
+    h2d = sum(h.numel() * h.element_size() for per in host for h in per)
+    steps = max(1, min(args.steps, args.e2e_steps))
+    opt.step_from_host(host)
+    barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        opt.step_from_host(host)
+    t1.record(stream)
+    barrier()
+    ms = t0.elapsed_time(t1)
+    if world_gpus > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    psi_p = sum(opt.layout.bucket_padded)
+    del host
+    return {"value": world_gpus * psi_p * steps / (ms * 1e-3) / 1e9, "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4, "steps": steps,
+            "ms_per_step": ms / steps}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-sample", type=int, default=1 << 23)
+    ap.add_argument("--ref-sample", type=int, default=1 << 23)
+    ap.add_argument("--flat", type=int, default=0, help="flat workload of this many elements instead of GPT-2")
+    ap.add_argument("--world", type=int, default=8, help="simulated replicas of the flat workload")
+    ap.add_argument("--grad-dtype", choices=["f16", "bf16"], default="f16")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,279 @@
+/*
+ * zero.h - C ABI of the ZeRO-DP partitioned mixed-precision Adam step (B200).
+ *
+ * The method: ZeRO, "Memory Optimizations Toward Training Trillion Parameter
+ * Models" (arXiv 1910.02054), as described by the azimuth.plus explainer of
+ * that title ("ZeRO explainer" below) and the codewithpapers method record
+ * "ZeRO".  Data-parallel replicas keep only 1/N of the model states; the
+ * gradients of the N replicas are reduce-scattered so that every rank holds
+ * the reduced gradients of its own partition, every rank updates its
+ * partition of the fp32 Adam states, and the updated low-precision parameters
+ * are all-gathered.
+ *
+ * Conventions shared by every call:
+ *  - Device pointers are CUDA global-memory addresses on the current device.
+ *    Host pointers are ordinary process memory.  Each argument says which.
+ *  - The caller owns all memory.  No call allocates device memory; only
+ *    zero_partition_layout allocates host arrays, released by
+ *    zero_layout_free.
+ *  - Device work is enqueued on `stream` (NULL = the legacy default stream)
+ *    and is asynchronous: nothing synchronizes inside a call.  Results written
+ *    to device memory (flags, norms) are valid once the stream reaches them.
+ *  - Every call returns ZERO_OK (0) or a negative ZERO_ERR_* code, validates
+ *    all arguments before launching anything, and launches nothing on error.
+ *    zero_last_error() returns a message for the calling thread's last error.
+ *  - Element counts and offsets are in elements of the named dtype.
+ */
+#ifndef ZERO_STEP_H
+#define ZERO_STEP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t); declared opaque so that this header needs no
+ * CUDA include. */
+typedef struct CUstream_st* zero_stream_t;
+
+typedef enum {
+    ZERO_F16 = 0,   /* IEEE binary16 */
+    ZERO_BF16 = 1,  /* bfloat16 */
+    ZERO_F32 = 2    /* IEEE binary32 (flatten only) */
+} zero_dtype_t;
+
+enum {
+    ZERO_OK = 0,
+    ZERO_ERR_ARG = -1,            /* null pointer, bad count, bad world size */
+    ZERO_ERR_ALIGN = -2,          /* pointer not aligned to its element size */
+    ZERO_ERR_DTYPE = -3,          /* dtype not supported by this call */
+    ZERO_ERR_RANGE = -4,          /* partition / bucket / range out of bounds */
+    ZERO_ERR_CUDA = -5,           /* a CUDA launch or query failed */
+    ZERO_ERR_NOMEM = -6           /* host allocation failed (layout only) */
+};
+
+/* Largest number of replicas (ranks) one call accepts. */
+#define ZERO_MAX_WORLD 128
+
+/* `partition` value that processes every rank's partition in one launch. */
+#define ZERO_ALL_PARTITIONS (-1)
+
+/* ------------------------------------------------------------------------ */
+/* Partition layout                                                          */
+/* ------------------------------------------------------------------------ */
+
+/* Layout of a parameter list in constant-size fused buffers ("buckets").
+ * All arrays are library-owned host memory. */
+typedef struct {
+    int32_t world;              /* N */
+    int32_t align_elems;        /* padding unit factor (>= 1) */
+    int64_t n_tensors;
+    int64_t n_buckets;
+    int64_t* bucket_numel;      /* [n_buckets] real elements */
+    int64_t* bucket_padded;     /* [n_buckets] multiple of world*align_elems */
+    int64_t* bucket_offset;     /* [n_buckets] start in the flat concatenation of padded buckets */
+    int64_t* bucket_first;      /* [n_buckets] first tensor index */
+    int64_t* bucket_count;      /* [n_buckets] number of tensors */
+    int64_t* tensor_numel;      /* [n_tensors] copy of the input element counts */
+    int64_t* tensor_bucket;     /* [n_tensors] bucket of each tensor */
+    int64_t* tensor_offset;     /* [n_tensors] start of each tensor inside its bucket */
+} zero_layout_t;
+
+/*
+ * zero_partition_layout - pack tensors into constant-size buffers and split
+ * each buffer into N equal partitions.
+ *
+ * Source: ZeRO explainer, "Constant-size buffers" (many small tensors fused
+ * into one buffer of a fixed size that does not grow with the model) and
+ * "Stage 1 - Optimizer State Partitioning (P_os)" (each of N GPUs holds 1/N
+ * of the states).  The pages fix no packing rule; this one is: tensors in
+ * list order, appended to the open bucket while the bucket stays within
+ * `bucket_elems`; a tensor that does not fit closes the bucket; a tensor
+ * larger than the capacity gets a bucket of its own; tensors are never split.
+ * `bucket_elems == 0` means one bucket.  Each bucket is padded with zeros up
+ * to a multiple of world*align_elems; rank r's partition of bucket b is
+ * elements [r*P_b, (r+1)*P_b) with P_b = bucket_padded[b] / world.
+ *
+ * numels      host, [n_tensors] element counts (>= 0)
+ * n_tensors   >= 0
+ * world       N, 1..ZERO_MAX_WORLD
+ * bucket_elems capacity in elements, >= 0
+ * align_elems >= 1 (1 = pad to a multiple of N only)
+ * out         host; filled on success, untouched on error
+ * Errors: ZERO_ERR_ARG, ZERO_ERR_NOMEM.  Host only, no CUDA call.
+ */
+int zero_partition_layout(const int64_t* numels, int64_t n_tensors, int32_t world,
+                          int64_t bucket_elems, int32_t align_elems, zero_layout_t* out);
+
+/* Release the arrays of a layout filled by zero_partition_layout (safe on a
+ * zeroed struct; the struct itself is the caller's). */
+void zero_layout_free(zero_layout_t* layout);
+
+/*
+ * zero_flatten_bucket - copy one bucket's tensors into its fused buffer.
+ *
+ * Source: ZeRO explainer, "Constant-size buffers" and "Memory
+ * defragmentation" (state lives in pre-allocated contiguous blocks).  Tensor
+ * i of bucket b is copied to bucket_buf[tensor_offset[i] ...]; the padding
+ * [bucket_numel[b], bucket_padded[b]) is set to zero.
+ *
+ * layout      host, from zero_partition_layout
+ * bucket      0 .. n_buckets-1
+ * tensor_ptrs host array of n_tensors DEVICE pointers indexed by tensor id;
+ *             only the bucket's entries are read; each holds numels[i]
+ *             contiguous elements of `dtype`
+ * dtype       ZERO_F16, ZERO_BF16 or ZERO_F32
+ * bucket_buf  device, bucket_padded[b] elements, must not overlap a source
+ * Errors: ZERO_ERR_ARG, ZERO_ERR_RANGE, ZERO_ERR_DTYPE, ZERO_ERR_ALIGN,
+ * ZERO_ERR_CUDA.
+ */
+int zero_flatten_bucket(const zero_layout_t* layout, int64_t bucket,
+                        const void* const* tensor_ptrs, zero_dtype_t dtype,
+                        void* bucket_buf, zero_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* The fused step                                                            */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    float lr;
+    float beta1;
+    float beta2;
+    float eps;
+    float weight_decay;   /* decoupled (AdamW): weights scale by 1 - lr*wd */
+    int64_t step;         /* t of THIS update, 1-based; counts applied updates only */
+    float grad_divisor;   /* replicas' sum is divided by this; 0 = world (the mean) */
+} zero_adam_hparams_t;
+
+/* Bytes of device workspace that zero_reduce_scatter_adam_step needs when it
+ * is asked for the gradient square-norm. */
+size_t zero_step_workspace_bytes(void);
+
+/*
+ * zero_reduce_scatter_adam_step - one fused pass of the ZeRO-2 step over one
+ * bucket: reduce-scatter + unscale + overflow test + Adam + parameter
+ * write-back.
+ *
+ * Sources: ZeRO explainer, "Stage 2 - Gradient Partitioning (P_os+g)" (each
+ * rank receives by reduce-scatter only the reduced gradients of its own
+ * partition and updates that partition), "Stage 1 - Optimizer State
+ * Partitioning (P_os)" (each rank updates its parameters with its 1/N of the
+ * fp32 optimizer states, then an all-gather distributes the updated
+ * parameters), model-states paragraph (fp16 parameters and gradients, fp32
+ * master weights, momentum and variance).
+ *
+ * The N replicas' gradient buffers are resident on this GPU.  For each
+ * processed element i (see `partition`):
+ *   s   = fp32(G_0[i]) + fp32(G_1[i]) + ... + fp32(G_{N-1}[i])   (left to right)
+ *   g   = s * fp32(1 / (divisor * loss_scale))
+ *   overflow if s is inf or NaN (any element of the call)
+ *   m'  = fma(b1, m, (1-b1)*g);  v' = fma(b2, v, ((1-b2)*g)*g)
+ *   u   = (m' * 1/(1-b1^t)) / fma(sqrt(v'), 1/sqrt(1-b2^t), eps)
+ *   p'  = fma(-lr, u, p * (1 - lr*wd));   param = round_to_nearest_even(p')
+ * Scalar constants are computed in double and rounded once to float; the
+ * division and square root are IEEE correctly rounded.  The results do not
+ * depend on the launch configuration.
+ *
+ * grad_bufs    host array of `world` DEVICE pointers, each padded_numel
+ *              elements of grad_dtype (replica k's bucket, unscaled by nothing)
+ * world        N, 1..ZERO_MAX_WORLD
+ * padded_numel elements of a replica's bucket, a multiple of world (>= 0)
+ * partition    ZERO_ALL_PARTITIONS: every rank's partition in one launch; the
+ *              state arrays and param_out then hold padded_numel elements in
+ *              flat order (the concatenation of the partitions in rank order).
+ *              r in 0..world-1: rank r only; state arrays and param_out hold
+ *              P = padded_numel/world elements, element j reads gradient
+ *              element r*P + j.
+ * grad_dtype   ZERO_F16 or ZERO_BF16
+ * master_in, m_in, v_in       device fp32, the current state (read)
+ * master_out, m_out, v_out    device fp32, the updated state (written).  May
+ *              equal the *_in pointers (in-place update); otherwise they must
+ *              not overlap them.  Writing to a second bank and committing it
+ *              only when *overflow_flag stays 0 keeps a skipped step's state
+ *              bit-identical.
+ * param_out    device, updated parameters in param_dtype (ZERO_F16/ZERO_BF16):
+ *              the all-gather payload, in the same indexing as the states
+ * hp           host, hyper-parameters; hp->step >= 1
+ * loss_scale   > 0 and finite: the gradients carry this factor
+ * overflow_flag device int32; set to 1 if any reduced gradient of this call
+ *              is inf or NaN, never written otherwise.  Clear it before the
+ *              first call of a step; calls over several buckets then OR into
+ *              one flag for the whole step.
+ * grad_sqnorm  device double or NULL; when not NULL, sum over the call's
+ *              elements of g*g is ADDED to it (clear it at the start of a
+ *              step).  Deterministic: per-block fp32 partial sums folded in a
+ *              fixed order in double.
+ * workspace    device, zero_step_workspace_bytes() bytes, zero-filled once
+ *              before its first use; required when grad_sqnorm is not NULL
+ *              (NULL allowed otherwise).  Each call leaves it zero-filled
+ *              again.  Calls that share a workspace must not run concurrently.
+ * Errors: ZERO_ERR_ARG, ZERO_ERR_RANGE, ZERO_ERR_DTYPE, ZERO_ERR_ALIGN
+ * (fp32 pointers need 4-byte, 16-bit pointers 2-byte alignment; 16-byte
+ * alignment of all arrays at the same element gives the vector path),
+ * ZERO_ERR_CUDA.
+ */
+int zero_reduce_scatter_adam_step(
+    const void* const* grad_bufs, int32_t world, int64_t padded_numel, int32_t partition,
+    zero_dtype_t grad_dtype,
+    const float* master_in, const float* m_in, const float* v_in,
+    float* master_out, float* m_out, float* v_out,
+    void* param_out, zero_dtype_t param_dtype,
+    const zero_adam_hparams_t* hp, float loss_scale,
+    int32_t* overflow_flag, double* grad_sqnorm, void* workspace,
+    zero_stream_t stream);
+
+/*
+ * zero_allgather_params - rebuild full parameters from N rank shards.
+ *
+ * Source: ZeRO explainer, "Stage 3 - Parameter Partitioning (P_os+g+p)" (each
+ * layer's parameters are reconstructed by all-gather from the ranks that own
+ * its slices, used, then discarded) and Stage 1/2 (all-gather of the updated
+ * parameters).  dst[r*part_numel + j] = shards[r][shard_offset + j] for
+ * r < world, j < part_numel: a bit-exact copy.  With shards that concatenate
+ * each unit's slices in unit order, shard_offset selects one unit.
+ *
+ * shards       host array of `world` DEVICE pointers
+ * world        1..ZERO_MAX_WORLD
+ * shard_offset first element of the slice in every shard (>= 0)
+ * part_numel   elements per rank (>= 0)
+ * dtype        ZERO_F16, ZERO_BF16 or ZERO_F32
+ * dst          device, world*part_numel elements, must not overlap a shard
+ * Errors: ZERO_ERR_ARG, ZERO_ERR_DTYPE, ZERO_ERR_ALIGN, ZERO_ERR_CUDA.
+ */
+int zero_allgather_params(const void* const* shards, int32_t world, int64_t shard_offset,
+                          int64_t part_numel, zero_dtype_t dtype, void* dst,
+                          zero_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Host helpers                                                              */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * zero_loss_scale_update - dynamic loss scale after a step (host only).
+ *
+ * Not on the pages (they fix only the fp16 storage of gradients); the usual
+ * rule: on overflow the update was skipped, the scale halves (not below
+ * min_scale) and the good-step count restarts; otherwise the count grows and
+ * the scale doubles after growth_interval consecutive good steps.
+ * scale, good_steps  host, updated in place
+ * Errors: ZERO_ERR_ARG (null pointer, growth_interval < 1, bad scale).
+ */
+int zero_loss_scale_update(float* scale, int32_t* good_steps, int32_t overflow,
+                           int32_t growth_interval, float min_scale);
+
+/* Static description of an error code. */
+const char* zero_strerror(int code);
+
+/* Message of the calling thread's most recent error ("" if none). */
+const char* zero_last_error(void);
+
+/* Version string of the library build. */
+const char* zero_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZERO_STEP_H */

@@ -1,0 +1,174 @@
+"""The C ABI without a GPU: exported symbols, host-only calls, validation.
+
+- every function declared in include/zero.h is exported by libzero.so;
+- zero_partition_layout equals the oracle's layout bit for bit;
+- zero_loss_scale_update follows the oracle's rule;
+- every device call rejects bad arguments with its error code before it
+  touches CUDA (so these run on a machine without a GPU).
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from zero_sharded_optimizer_reduce_b200 import build as zbuild
+
+zbuild.build()
+import zero_sharded_optimizer_reduce_b200 as Z  # noqa: E402
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "zero.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(zero_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared_functions()
+    assert len(names) >= 10
+    lib = ctypes.CDLL(Z.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_library_reports_version_and_errors():
+    assert "sm_100a" in Z.version()
+    assert Z.lib.zero_strerror(0) == b"ok"
+    assert Z.lib.zero_strerror(-2) == b"misaligned pointer"
+
+
+@pytest.mark.parametrize("world", [1, 3, 4, 8])
+@pytest.mark.parametrize("cap", [0, 7, 50])
+@pytest.mark.parametrize("align", [1, 8])
+def test_layout_equals_oracle(world, cap, align):
+    rng = np.random.Generator(np.random.PCG64(world * 31 + cap + align))
+    for _ in range(6):
+        numels = rng.integers(0, 40, rng.integers(0, 15)).tolist()
+        a = Z.zero_partition_layout(numels, world, cap, align)
+        b = oracle.partition_layout(numels, world, cap, align)
+        assert list(a.bucket_numel) == b.bucket_numel
+        assert list(a.bucket_padded) == b.bucket_padded
+        assert list(a.bucket_offset) == b.bucket_offset
+        assert list(a.tensor_bucket) == b.tensor_bucket
+        assert list(a.tensor_offset) == b.tensor_offset
+        assert [list(range(f, f + c)) for f, c in zip(a.bucket_first, a.bucket_count)] == b.bucket_tensors
+
+
+def test_layout_gpt2_and_6p7b():
+    numels = workloads.gpt2_1p5b_tensor_numels()
+    a = Z.zero_partition_layout(numels, 8, 500_000_000)
+    assert list(a.bucket_padded) == oracle.partition_layout(numels, 8, 500_000_000).bucket_padded
+    units = workloads.gpt_6p7b_unit_numels()
+    a = Z.zero_partition_layout(units, 8, 1)
+    assert a.n_buckets == 33 and a.part(0) == 25_172_480
+
+
+def test_layout_errors():
+    for args in [([3], 0, 0, 1), ([3], 129, 0, 1), ([3], 2, -1, 1), ([3], 2, 0, 0), ([-3], 2, 0, 1)]:
+        with pytest.raises(Z.ZeroError) as e:
+            Z.zero_partition_layout(*args)
+        assert e.value.code == -1
+    out = Z._Layout()
+    assert Z.lib.zero_partition_layout(None, 1, 2, 0, 1, ctypes.byref(out)) == -1
+    assert Z.lib.zero_partition_layout(None, 0, 2, 0, 1, None) == -1
+    # an empty list is a valid, empty layout
+    assert Z.zero_partition_layout([], 4).n_buckets == 0
+
+
+def test_loss_scale_matches_oracle():
+    rng = np.random.Generator(np.random.PCG64(3))
+    s, g = 65536.0, 0
+    so, go = s, g
+    for _ in range(200):
+        ovf = bool(rng.random() < 0.2)
+        s, g = Z.zero_loss_scale_update(s, g, ovf, growth_interval=5, min_scale=1.0)
+        so, go = oracle.loss_scale_update(so, go, ovf, growth_interval=5, min_scale=1.0)
+        assert (s, g) == (so, go)
+    with pytest.raises(Z.ZeroError):
+        Z.zero_loss_scale_update(1.0, 0, False, growth_interval=0)
+    with pytest.raises(Z.ZeroError):
+        Z.zero_loss_scale_update(-1.0, 0, False)
+
+
+# ------------------------------------------------------------- validation
+
+def _step_call(**kw):
+    """Raw call with fake (never dereferenced) pointers; returns the code."""
+    L = Z.lib
+    world = kw.get("world", 2)
+    grads = kw.get("grads", [0x10000 * (k + 1) for k in range(world)])
+    g = None if grads is None else (ctypes.c_void_p * max(1, len(grads)))(*grads)
+    hp = kw.get("hp", Z.hparams())
+    base = 0x7000_0000
+    f = lambda i: kw.get(f"p{i}", base + 0x100_0000 * i)
+    return L.zero_reduce_scatter_adam_step(
+        g, world, kw.get("n", 64), kw.get("part", -1), kw.get("gd", 0),
+        f(1), f(2), f(3), f(4), f(5), f(6), f(7), kw.get("pd", 0),
+        None if hp is None else ctypes.byref(hp), kw.get("scale", 1024.0),
+        kw.get("flag", base + 0x100_0000 * 9), kw.get("norm", None), kw.get("ws", None), None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(grads=None), -1),
+    (dict(hp=None), -1),
+    (dict(flag=0), -1),
+    (dict(world=0, grads=[]), -1),
+    (dict(world=129, grads=[0x10000] * 129), -1),
+    (dict(n=63), -1),
+    (dict(n=-2), -1),
+    (dict(part=2), -4),
+    (dict(part=-2), -4),
+    (dict(gd=2), -3),
+    (dict(pd=7), -3),
+    (dict(hp=Z.hparams(step=0)), -1),
+    (dict(hp=Z.hparams(beta1=1.0)), -1),
+    (dict(hp=Z.hparams(beta2=-0.1)), -1),
+    (dict(hp=Z.hparams(lr=float("nan"))), -1),
+    (dict(scale=0.0), -1),
+    (dict(scale=float("inf")), -1),
+    (dict(norm=0x7F00_0000), -1),                 # norm without workspace
+    (dict(flag=0x7000_0002), -2),                  # misaligned flag
+    (dict(p1=0), -1),                              # NULL master_in
+    (dict(p7=0), -1),                              # NULL param_out
+    (dict(p1=0x7000_0002), -2),                    # master_in not 4-byte aligned
+    (dict(p7=0x7700_0001), -2),                    # param_out not 2-byte aligned
+    (dict(grads=[0x10000, 0]), -1),                # NULL replica
+    (dict(grads=[0x10000, 0x10001]), -2),          # misaligned replica
+    (dict(p4=0x7200_0000 + 8), -1),                # master_out overlaps m_in
+    (dict(p5=0x7400_0000 + 64), -1),              # m_out overlaps master_out
+    (dict(p7=0x10000 + 16), -1),                   # param_out overlaps a gradient buffer
+])
+def test_step_rejects_bad_arguments(kw, code):
+    assert _step_call(**kw) == code
+    assert Z.lib.zero_last_error() != b""
+
+
+def test_step_with_nothing_to_do_is_ok():
+    assert _step_call(n=0) == 0
+
+
+def test_allgather_and_flatten_reject_bad_arguments():
+    L = Z.lib
+    sh = (ctypes.c_void_p * 2)(0x10000, 0x20000)
+    assert L.zero_allgather_params(None, 2, 0, 8, 0, 0x30000, None) == -1
+    assert L.zero_allgather_params(sh, 0, 0, 8, 0, 0x30000, None) == -1
+    assert L.zero_allgather_params(sh, 2, -1, 8, 0, 0x30000, None) == -1
+    assert L.zero_allgather_params(sh, 2, 0, 8, 9, 0x30000, None) == -3
+    assert L.zero_allgather_params(sh, 2, 0, 8, 2, 0x30002, None) == -2
+    assert L.zero_allgather_params(sh, 2, 0, 8, 0, 0x10008, None) == -1   # dst overlaps shard 0
+    bad = (ctypes.c_void_p * 2)(0x10001, 0x20000)
+    assert L.zero_allgather_params(bad, 2, 0, 8, 0, 0x30000, None) == -2
+    assert L.zero_allgather_params(sh, 2, 0, 0, 0, 0x30000, None) == 0     # nothing to copy
+    lay = Z.zero_partition_layout([5, 7], 2)._c()
+    tp = (ctypes.c_void_p * 2)(0x10000, 0x20000)
+    assert L.zero_flatten_bucket(None, 0, tp, 0, 0x30000, None) == -1
+    assert L.zero_flatten_bucket(ctypes.byref(lay), 1, tp, 0, 0x30000, None) == -4
+    assert L.zero_flatten_bucket(ctypes.byref(lay), 0, tp, 5, 0x30000, None) == -3
+    assert L.zero_flatten_bucket(ctypes.byref(lay), 0, tp, 2, 0x30002, None) == -2
+    assert L.zero_flatten_bucket(ctypes.byref(lay), 0, tp, 0, 0x10004, None) == -1

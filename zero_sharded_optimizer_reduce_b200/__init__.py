@@ -1,0 +1,226 @@
+"""Python binding of libzero, the C ABI of the ZeRO-DP partitioned Adam step.
+
+Argument marshalling only: every computation runs in the CUDA kernels of
+libzero.so.  The functions carry the names of the C calls in include/zero.h
+and take torch tensors (device memory, `data_ptr()`) or plain Python values;
+streams default to torch's current stream.
+
+The library is loaded from this package directory.  If it is missing, import
+fails with an error that says how to build it: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libzero.so")
+
+ZERO_F16, ZERO_BF16, ZERO_F32 = 0, 1, 2
+ZERO_ALL_PARTITIONS = -1
+ZERO_MAX_WORLD = 128
+ERRORS = {0: "ZERO_OK", -1: "ZERO_ERR_ARG", -2: "ZERO_ERR_ALIGN", -3: "ZERO_ERR_DTYPE",
+          -4: "ZERO_ERR_RANGE", -5: "ZERO_ERR_CUDA", -6: "ZERO_ERR_NOMEM"}
+
+
+class ZeroError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{ERRORS.get(code, code)}: {msg}")
+        self.code = code
+
+
+class _Layout(ctypes.Structure):
+    _fields_ = [("world", ctypes.c_int32), ("align_elems", ctypes.c_int32),
+                ("n_tensors", ctypes.c_int64), ("n_buckets", ctypes.c_int64),
+                ("bucket_numel", ctypes.POINTER(ctypes.c_int64)),
+                ("bucket_padded", ctypes.POINTER(ctypes.c_int64)),
+                ("bucket_offset", ctypes.POINTER(ctypes.c_int64)),
+                ("bucket_first", ctypes.POINTER(ctypes.c_int64)),
+                ("bucket_count", ctypes.POINTER(ctypes.c_int64)),
+                ("tensor_numel", ctypes.POINTER(ctypes.c_int64)),
+                ("tensor_bucket", ctypes.POINTER(ctypes.c_int64)),
+                ("tensor_offset", ctypes.POINTER(ctypes.c_int64))]
+
+
+class AdamHParams(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float),
+                ("step", ctypes.c_int64), ("grad_divisor", ctypes.c_float)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m zero_sharded_optimizer_reduce_b200.build` (nvcc, sm_100a)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+    L.zero_partition_layout.argtypes = [ctypes.POINTER(ctypes.c_int64), i64, i32, i64, i32,
+                                        ctypes.POINTER(_Layout)]
+    L.zero_partition_layout.restype = ctypes.c_int
+    L.zero_layout_free.argtypes = [ctypes.POINTER(_Layout)]
+    L.zero_layout_free.restype = None
+    L.zero_flatten_bucket.argtypes = [ctypes.POINTER(_Layout), i64, ctypes.POINTER(vp), ctypes.c_int, vp, vp]
+    L.zero_flatten_bucket.restype = ctypes.c_int
+    L.zero_step_workspace_bytes.argtypes = []
+    L.zero_step_workspace_bytes.restype = ctypes.c_size_t
+    L.zero_reduce_scatter_adam_step.argtypes = [
+        ctypes.POINTER(vp), i32, i64, i32, ctypes.c_int,
+        vp, vp, vp, vp, vp, vp, vp, ctypes.c_int,
+        ctypes.POINTER(AdamHParams), f32, vp, vp, vp, vp]
+    L.zero_reduce_scatter_adam_step.restype = ctypes.c_int
+    L.zero_allgather_params.argtypes = [ctypes.POINTER(vp), i32, i64, i64, ctypes.c_int, vp, vp]
+    L.zero_allgather_params.restype = ctypes.c_int
+    L.zero_loss_scale_update.argtypes = [ctypes.POINTER(f32), ctypes.POINTER(i32), i32, i32, f32]
+    L.zero_loss_scale_update.restype = ctypes.c_int
+    L.zero_strerror.argtypes = [ctypes.c_int]
+    L.zero_strerror.restype = ctypes.c_char_p
+    L.zero_last_error.argtypes = []
+    L.zero_last_error.restype = ctypes.c_char_p
+    L.zero_version.argtypes = []
+    L.zero_version.restype = ctypes.c_char_p
+    return L
+
+
+lib = _load()
+
+
+def _check(rc: int) -> None:
+    if rc != 0:
+        raise ZeroError(rc, lib.zero_last_error().decode())
+
+
+def _dtype_code(t) -> int:
+    import torch
+    m = {torch.float16: ZERO_F16, torch.bfloat16: ZERO_BF16, torch.float32: ZERO_F32}
+    if t.dtype not in m:
+        raise ZeroError(-3, f"unsupported dtype {t.dtype}")
+    return m[t.dtype]
+
+
+def _stream(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else int(t.data_ptr())
+
+
+def _ptrs(ts) -> ctypes.Array:
+    return (ctypes.c_void_p * len(ts))(*[_ptr(t) for t in ts])
+
+
+# ---------------------------------------------------------------------------
+# Layout
+# ---------------------------------------------------------------------------
+
+@dataclasses.dataclass(frozen=True)
+class Layout:
+    """Host copy of a zero_layout_t (the C arrays are freed after copying)."""
+    world: int
+    align_elems: int
+    bucket_numel: tuple
+    bucket_padded: tuple
+    bucket_offset: tuple
+    bucket_first: tuple
+    bucket_count: tuple
+    tensor_numel: tuple
+    tensor_bucket: tuple
+    tensor_offset: tuple
+
+    @property
+    def n_buckets(self) -> int:
+        return len(self.bucket_numel)
+
+    def part(self, b: int) -> int:
+        return self.bucket_padded[b] // self.world
+
+    def _c(self) -> _Layout:
+        def arr(x):
+            return (ctypes.c_int64 * max(1, len(x)))(*x)
+        c = _Layout()
+        c.world, c.align_elems = self.world, self.align_elems
+        c.n_tensors, c.n_buckets = len(self.tensor_numel), len(self.bucket_numel)
+        keep = []
+        for name in ("bucket_numel", "bucket_padded", "bucket_offset", "bucket_first", "bucket_count",
+                     "tensor_numel", "tensor_bucket", "tensor_offset"):
+            a = arr(getattr(self, name))
+            keep.append(a)
+            setattr(c, name, ctypes.cast(a, ctypes.POINTER(ctypes.c_int64)))
+        c._keep = keep
+        return c
+
+
+def zero_partition_layout(numels, world: int, bucket_elems: int = 0, align_elems: int = 1) -> Layout:
+    n = len(numels)
+    arr = (ctypes.c_int64 * max(1, n))(*numels)
+    out = _Layout()
+    _check(lib.zero_partition_layout(arr, n, world, bucket_elems, align_elems, ctypes.byref(out)))
+    try:
+        nb, nt = out.n_buckets, out.n_tensors
+        get = lambda p, k: tuple(p[i] for i in range(k))
+        return Layout(out.world, out.align_elems,
+                      get(out.bucket_numel, nb), get(out.bucket_padded, nb), get(out.bucket_offset, nb),
+                      get(out.bucket_first, nb), get(out.bucket_count, nb),
+                      get(out.tensor_numel, nt), get(out.tensor_bucket, nt), get(out.tensor_offset, nt))
+    finally:
+        lib.zero_layout_free(ctypes.byref(out))
+
+
+# ---------------------------------------------------------------------------
+# Device calls
+# ---------------------------------------------------------------------------
+
+def zero_flatten_bucket(layout: Layout, bucket: int, tensors, bucket_buf, stream=None) -> None:
+    """Copy bucket `bucket`'s tensors (list indexed by tensor id) into bucket_buf."""
+    ptrs = (ctypes.c_void_p * max(1, len(tensors)))(*[_ptr(t) for t in tensors])
+    c = layout._c()
+    _check(lib.zero_flatten_bucket(ctypes.byref(c), bucket, ptrs, _dtype_code(bucket_buf),
+                                   _ptr(bucket_buf), _stream(stream)))
+
+
+def zero_step_workspace_bytes() -> int:
+    return int(lib.zero_step_workspace_bytes())
+
+
+def hparams(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, step=1,
+            grad_divisor=0.0) -> AdamHParams:
+    return AdamHParams(lr, beta1, beta2, eps, weight_decay, step, grad_divisor)
+
+
+def zero_reduce_scatter_adam_step(grad_bufs, padded_numel: int, partition: int,
+                                  master_in, m_in, v_in, master_out, m_out, v_out, param_out,
+                                  hp: AdamHParams, loss_scale: float, overflow_flag,
+                                  grad_sqnorm=None, workspace=None, stream=None) -> None:
+    """One fused reduce-scatter + Adam pass over one bucket (see include/zero.h)."""
+    world = len(grad_bufs)
+    _check(lib.zero_reduce_scatter_adam_step(
+        _ptrs(grad_bufs), world, padded_numel, partition, _dtype_code(grad_bufs[0]),
+        _ptr(master_in), _ptr(m_in), _ptr(v_in), _ptr(master_out), _ptr(m_out), _ptr(v_out),
+        _ptr(param_out), _dtype_code(param_out), ctypes.byref(hp), float(loss_scale),
+        _ptr(overflow_flag), _ptr(grad_sqnorm), _ptr(workspace), _stream(stream)))
+
+
+def zero_allgather_params(shards, shard_offset: int, part_numel: int, dst, stream=None) -> None:
+    """dst[r*part + j] = shards[r][shard_offset + j] (bit-exact copy)."""
+    _check(lib.zero_allgather_params(_ptrs(shards), len(shards), shard_offset, part_numel,
+                                     _dtype_code(dst), _ptr(dst), _stream(stream)))
+
+
+def zero_loss_scale_update(scale: float, good_steps: int, overflow: bool,
+                           growth_interval: int = 1000, min_scale: float = 1.0):
+    s = ctypes.c_float(scale)
+    g = ctypes.c_int32(good_steps)
+    _check(lib.zero_loss_scale_update(ctypes.byref(s), ctypes.byref(g), int(bool(overflow)),
+                                      growth_interval, min_scale))
+    return s.value, g.value
+
+
+def version() -> str:
+    return lib.zero_version().decode()
+
+
+from .optimizer import ZeroAdam  # noqa: E402  (uses the bindings above)

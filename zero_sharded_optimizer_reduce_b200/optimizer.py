@@ -1,0 +1,148 @@
+"""ZeroAdam: a ZeRO-2 partitioned mixed-precision Adam step on one GPU.
+
+N data-parallel replicas are simulated by N resident gradient buffers per
+bucket.  A step runs the fused reduce-scatter + Adam kernel over every bucket,
+reads the overflow flag, and commits or skips:
+
+  - the fp32 master / momentum / variance states and the low-precision
+    parameters live in two banks; a step reads bank `cur` and writes bank
+    `cur ^ 1`, and the bank flips only when no reduced gradient of the whole
+    step was inf or NaN, so a skipped step leaves every state bit-identical;
+  - the loss scale follows zero_loss_scale_update (halve on overflow, double
+    after `growth_interval` good steps) and the Adam step count t advances
+    only on applied updates.
+
+The second bank doubles the 12 Psi/N bytes of optimizer state that ZeRO
+keeps per rank (ZeRO explainer, "Stage 1 - Optimizer State Partitioning");
+it buys a single pass over HBM per step with an exact skip.
+
+This class only allocates buffers and sequences library calls; all
+arithmetic is in libzero's kernels.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (ZERO_ALL_PARTITIONS, hparams, zero_flatten_bucket, zero_loss_scale_update,
+               zero_partition_layout, zero_reduce_scatter_adam_step, zero_step_workspace_bytes)
+
+
+class ZeroAdam:
+    def __init__(self, numels, world: int, bucket_elems: int = 0, align_elems: int = 1, *,
+                 lr: float = 1e-3, betas=(0.9, 0.999), eps: float = 1e-8, weight_decay: float = 0.0,
+                 grad_dtype=torch.float16, param_dtype=torch.float16, loss_scale: float = 65536.0,
+                 growth_interval: int = 1000, min_scale: float = 1.0, grad_divisor: float = 0.0,
+                 track_grad_norm: bool = False, device="cuda"):
+        self.layout = zero_partition_layout(list(numels), world, bucket_elems, align_elems)
+        self.world = world
+        self.device = torch.device(device)
+        self.lr, self.betas, self.eps, self.weight_decay = lr, betas, eps, weight_decay
+        self.grad_divisor = grad_divisor
+        self.scale, self.good_steps = float(loss_scale), 0
+        self.growth_interval, self.min_scale = growth_interval, min_scale
+        self.t = 0
+        self.cur = 0
+        L, dev = self.layout, self.device
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.master = [[torch.zeros(L.bucket_padded[b], **f32) for _ in range(2)] for b in range(L.n_buckets)]
+        self.m = [[torch.zeros(L.bucket_padded[b], **f32) for _ in range(2)] for b in range(L.n_buckets)]
+        self.v = [[torch.zeros(L.bucket_padded[b], **f32) for _ in range(2)] for b in range(L.n_buckets)]
+        self.params_bank = [[torch.zeros(L.bucket_padded[b], dtype=param_dtype, device=dev) for _ in range(2)]
+                            for b in range(L.n_buckets)]
+        self.grads = [[torch.zeros(L.bucket_padded[b], dtype=grad_dtype, device=dev) for _ in range(world)]
+                      for b in range(L.n_buckets)]
+        self.flag = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.flag_host = torch.zeros(1, dtype=torch.int32, pin_memory=True)
+        self.track_grad_norm = track_grad_norm
+        self.sqnorm = torch.zeros(1, dtype=torch.float64, device=dev) if track_grad_norm else None
+        self.workspace = (torch.zeros(zero_step_workspace_bytes(), dtype=torch.uint8, device=dev)
+                          if track_grad_norm else None)
+        self.last_overflow = 0
+
+    # ------------------------------------------------------------ state access
+    def load(self, params, master=None, stream=None) -> None:
+        """Fill both banks from per-tensor parameters (and fp32 masters).
+
+        `params`: list of low-precision tensors (one per tensor of the layout);
+        `master`: list of fp32 tensors, default the parameters widened to fp32.
+        m and v start at zero; t restarts at 0.
+        """
+        if master is None:
+            master = [p.float() for p in params]
+        for b in range(self.layout.n_buckets):
+            zero_flatten_bucket(self.layout, b, master, self.master[b][0], stream)
+            zero_flatten_bucket(self.layout, b, params, self.params_bank[b][0], stream)
+            for bank in (self.master, self.params_bank):
+                bank[b][1].copy_(bank[b][0])
+            for bank in (self.m, self.v):
+                bank[b][0].zero_()
+                bank[b][1].zero_()
+        self.cur = 0
+        self.t = 0
+
+    def state(self, b: int):
+        """Committed (master, m, v, params) of bucket b."""
+        c = self.cur
+        return self.master[b][c], self.m[b][c], self.v[b][c], self.params_bank[b][c]
+
+    def grad_buffers(self, b: int):
+        """The N replicas' gradient buffers of bucket b (write gradients here)."""
+        return self.grads[b]
+
+    # -------------------------------------------------------------------- step
+    def launch(self, stream=None, on_launch=None) -> None:
+        """Enqueue the fused kernel over every bucket (no host synchronization).
+
+        `on_launch(bucket, phase)` is called with phase "before" / "after"
+        around each kernel launch (used to record timing events).
+        """
+        if stream is not None:
+            with torch.cuda.stream(stream):
+                return self.launch(None, on_launch)
+        self.flag.zero_()
+        if self.sqnorm is not None:
+            self.sqnorm.zero_()
+        hp = hparams(self.lr, self.betas[0], self.betas[1], self.eps, self.weight_decay,
+                     self.t + 1, self.grad_divisor)
+        c, n = self.cur, self.cur ^ 1
+        for b in range(self.layout.n_buckets):
+            if on_launch is not None:
+                on_launch(b, "before")
+            zero_reduce_scatter_adam_step(
+                self.grads[b], self.layout.bucket_padded[b], ZERO_ALL_PARTITIONS,
+                self.master[b][c], self.m[b][c], self.v[b][c],
+                self.master[b][n], self.m[b][n], self.v[b][n], self.params_bank[b][n],
+                hp, self.scale, self.flag, self.sqnorm, self.workspace)
+            if on_launch is not None:
+                on_launch(b, "after")
+
+    def commit(self, stream=None) -> bool:
+        """Read the overflow flag (device -> host), flip banks or skip, update the scale."""
+        s = torch.cuda.current_stream() if stream is None else stream
+        self.flag_host.copy_(self.flag, non_blocking=True)
+        s.synchronize()
+        ovf = int(self.flag_host.item())
+        if not ovf:
+            self.cur ^= 1
+            self.t += 1
+        self.scale, self.good_steps = zero_loss_scale_update(self.scale, self.good_steps, bool(ovf),
+                                                             self.growth_interval, self.min_scale)
+        self.last_overflow = ovf
+        return not ovf
+
+    def step(self, stream=None, on_launch=None) -> bool:
+        """One whole step over all buckets; returns True if the update was applied."""
+        self.launch(stream, on_launch)
+        return self.commit(stream)
+
+    def step_from_host(self, host_grads, stream=None) -> bool:
+        """Copy host gradients (host_grads[b][k], pinned) in, then step."""
+        with torch.cuda.stream(stream if stream is not None else torch.cuda.current_stream()):
+            for b in range(self.layout.n_buckets):
+                for k in range(self.world):
+                    self.grads[b][k].copy_(host_grads[b][k], non_blocking=True)
+            return self.step()
+
+    def grad_sqnorm(self) -> float:
+        """Sum of squared unscaled gradients of the last step (if tracked)."""
+        return float(self.sqnorm.item()) if self.sqnorm is not None else float("nan")
