@@ -117,7 +117,7 @@ class ClockSampler:
 
 def source_digest() -> str:
     h = hashlib.sha256()
-    p = os.path.join(ROOT, "zero_sharded_optimizer_reduce_b200", "csrc", "step.cu")
+    p = os.path.join(ROOT, "zero_sharded_optimizer_reduce_b200", "csrc", "fused_step.cuh")
     h.update(open(p, "rb").read())
     return h.hexdigest()[:16]
 
@@ -130,7 +130,7 @@ def profiled_traffic(elems_per_launch: float):
         d = json.load(open(p))
     except Exception:
         return None
-    if d.get("step_cu_sha256_16") != source_digest():
+    if d.get("kernel_source_sha256_16") != source_digest():
         return None
     return float(d["dram_bytes_per_elem"]) * elems_per_launch
 

@@ -1,0 +1,281 @@
+"""Parity at the workloads' full sizes, in the launch configuration the
+benchmark times (every rank's partition in one launch per bucket).
+
+- GPT-2 1.5B parameter list, 4 buckets of <= 500M elements, N = 8, AdamW,
+  5 steps: sampled windows (seeded windows, every partition and bucket
+  boundary, first and last elements) against the oracle run on the same
+  windows; the overflow flag is 0 at every step, as it must be for finite
+  fp16 gradients (8 x 65504 cannot overflow fp32).
+- Dynamic loss-scale workload: flat 100M elements, N = 16, 6 steps, +inf /
+  NaN injected at 17 positions at steps 2 and 4: full arrays against the
+  oracle, flag bit-exact, skipped steps leave every state bit-identical,
+  scale 65536 -> 32768 -> 16384.
+- Stage 3 layer-wise path on the 6.7B GPT shape, N = 8, fp16 and bf16: per
+  unit an all-gather of the unit's parameters from 8 rank-major shards into a
+  reused layer buffer, then one fused call per rank writing its updated
+  parameters into its own shard; windows against the oracle, whole gathered
+  units bit-exact.
+- Flat bandwidth-sweep points: windows.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import zero_sharded_optimizer_reduce_b200 as Z
+from _gpu import assert_f32_close, assert_u16_close, host_f32, host_u16
+
+pytestmark = pytest.mark.gpu
+
+TD = {oracle.F16: torch.float16, oracle.BF16: torch.bfloat16}
+
+
+def _free_gb():
+    free, _ = torch.cuda.mem_get_info()
+    return free / 1e9
+
+
+def _device_grads(buf, seed, std, scale):
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(seed)
+    n = buf.numel()
+    chunk = 1 << 27
+    for o in range(0, n, chunk):
+        e = min(n, o + chunk)
+        buf[o:e].copy_(torch.randn(e - o, generator=gen, device="cuda").mul_(std * scale))
+
+
+def _device_master(buf, seed, std=0.02):
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(seed)
+    n = buf.numel()
+    for o in range(0, n, 1 << 27):
+        e = min(n, o + (1 << 27))
+        buf[o:e].copy_(torch.randn(e - o, generator=gen, device="cuda").mul_(std))
+
+
+def _windows(padded, world, n_random=64, width=65_536, seed=0):
+    """Sorted, disjoint [lo, hi) windows: random, partition boundaries, ends."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    P = padded // world
+    spans = [(0, 4096), (padded - 4096, padded)]
+    for r in range(1, world):
+        spans.append((r * P - 4, r * P + 4))
+    for lo in rng.integers(0, max(1, padded - width), n_random):
+        spans.append((int(lo), int(lo) + width))
+    spans = sorted((max(0, a), min(padded, b)) for a, b in spans)
+    merged = []
+    for a, b in spans:
+        if merged and a <= merged[-1][1]:
+            merged[-1] = (merged[-1][0], max(merged[-1][1], b))
+        else:
+            merged.append((a, b))
+    return merged
+
+
+def _take(t, wins):
+    return [t[a:b] for a, b in wins]
+
+
+def _u16(t):
+    return host_u16(t)
+
+
+@pytest.mark.skipif(not torch.cuda.is_available() or _free_gb() < 80, reason="needs ~70 GB of HBM")
+def test_gpt2_1p5b_windows_five_steps():
+    w = workloads.gpt2_1p5b()
+    opt = Z.ZeroAdam(w.numels, w.world, w.bucket_elems, lr=w.adam.lr, betas=(w.adam.beta1, w.adam.beta2),
+                     eps=w.adam.eps, weight_decay=w.adam.weight_decay, loss_scale=w.loss_scale)
+    L = opt.layout
+    wins, refs = [], []
+    for b in range(L.n_buckets):
+        _device_master(opt.master[b][0], 700 + b)
+        opt.master[b][0][L.bucket_numel[b]:].zero_()
+        opt.params_bank[b][0].copy_(opt.master[b][0])
+        opt.master[b][1].copy_(opt.master[b][0])
+        opt.params_bank[b][1].copy_(opt.params_bank[b][0])
+        wb = _windows(L.bucket_padded[b], w.world, n_random=16, seed=b)
+        wins.append(wb)
+        # the oracle's state on the windows, from the device's initial values
+        refs.append([oracle.FlatState(host_f32(opt.master[b][0][lo:hi]).copy(),
+                                      np.zeros(hi - lo, np.float32), np.zeros(hi - lo, np.float32),
+                                      _u16(opt.params_bank[b][0][lo:hi]).copy()) for lo, hi in wb])
+    for step in range(1, w.steps + 1):
+        win_grads = []
+        for b in range(L.n_buckets):
+            for k in range(w.world):
+                _device_grads(opt.grads[b][k], workloads.seed_for(w.seed, step, k) + 31 * b, w.grad_std, w.loss_scale)
+                opt.grads[b][k][L.bucket_numel[b]:].zero_()
+            win_grads.append([[_u16(opt.grads[b][k][lo:hi]) for k in range(w.world)] for lo, hi in wins[b]])
+        assert opt.step(), f"unexpected overflow at step {step}"
+        assert int(opt.flag.item()) == 0
+        for b in range(L.n_buckets):
+            for (lo, hi), G, st in zip(wins[b], win_grads[b], refs[b]):
+                ovf, _ = oracle.flat_step(G, st, w.adam, step, w.loss_scale, float(w.world))
+                assert ovf == 0
+    for b in range(L.n_buckets):
+        master, m, v, p = opt.state(b)
+        for (lo, hi), st in zip(wins[b], refs[b]):
+            assert assert_f32_close(host_f32(master[lo:hi]), st.master, "master") == 0
+            assert assert_f32_close(host_f32(m[lo:hi]), st.m, "m") == 0
+            assert assert_f32_close(host_f32(v[lo:hi]), st.v, "v") == 0
+            assert assert_u16_close(_u16(p[lo:hi]), st.params, "params") == 0
+    assert opt.t == w.steps and opt.scale == w.loss_scale
+
+
+@pytest.mark.skipif(not torch.cuda.is_available() or _free_gb() < 12, reason="needs ~8 GB of HBM")
+def test_overflow_workload_full_arrays():
+    w = workloads.overflow_flat()
+    (psi,) = w.numels
+    N = w.world
+    opt = Z.ZeroAdam([psi], N, lr=w.adam.lr, betas=(w.adam.beta1, w.adam.beta2), eps=w.adam.eps,
+                     weight_decay=w.adam.weight_decay, loss_scale=w.loss_scale, track_grad_norm=True)
+    padded = opt.layout.bucket_padded[0]
+    assert padded == psi
+    _device_master(opt.master[0][0], 900)
+    opt.params_bank[0][0].copy_(opt.master[0][0])
+    opt.master[0][1].copy_(opt.master[0][0])
+    opt.params_bank[0][1].copy_(opt.params_bank[0][0])
+    ref = oracle.FlatState(host_f32(opt.master[0][0]).copy(), np.zeros(psi, np.float32),
+                           np.zeros(psi, np.float32), _u16(opt.params_bank[0][0]).copy())
+    scaler = oracle.Scaler(w.loss_scale)
+    scales = []
+    for step in range(1, w.steps + 1):
+        G = []
+        for k in range(N):
+            _device_grads(opt.grads[0][k], workloads.seed_for(w.seed, step, k), w.grad_std, opt.scale)
+            G.append(_u16(opt.grads[0][k]))
+        injected = step in (2, 4)
+        if injected:
+            rep, pos, is_inf = workloads.injection_sites(psi, step, N)
+            workloads.inject(G[rep], pos, is_inf)
+            opt.grads[0][rep].copy_(torch.from_numpy(G[rep].view(np.int16)).cuda().view(torch.float16))
+        before = [x.clone() for x in opt.state(0)]
+        applied = opt.step()
+        s = oracle.reduce(G)
+        ovf = oracle.any_nonfinite(s)
+        assert ovf == int(injected) and applied == (not ovf) and int(opt.flag.item()) == ovf
+        if not ovf:
+            c = oracle.adam_constants(w.adam, scaler.t + 1, float(N), scaler.scale)
+            sq = oracle.grad_sqnorm(s, c[4])
+            oracle.adam_update(s, c, ref.master, ref.m, ref.v, ref.params)
+            scaler.t += 1
+            assert abs(opt.grad_sqnorm() - sq) <= 1e-5 * sq
+        else:
+            for x, y in zip(before, opt.state(0)):
+                assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
+        scaler.scale, scaler.good_steps = oracle.loss_scale_update(scaler.scale, scaler.good_steps, bool(ovf))
+        assert opt.scale == scaler.scale and opt.t == scaler.t
+        scales.append(opt.scale)
+        master, m, v, p = opt.state(0)
+        assert assert_f32_close(host_f32(master), ref.master, "master") == 0
+        assert assert_f32_close(host_f32(m), ref.m, "m") == 0
+        assert assert_f32_close(host_f32(v), ref.v, "v") == 0
+        assert assert_u16_close(_u16(p), ref.params, "params") == 0
+    assert scales == [65536.0, 32768.0, 32768.0, 16384.0, 16384.0, 16384.0]
+    assert opt.t == 4
+
+
+@pytest.mark.parametrize("dtype", [oracle.F16, oracle.BF16])
+def test_stage3_layerwise_6p7b(dtype):
+    """Stage 3 on the 6.7B GPT shape: per unit, gather then fused update per rank.
+
+    Runs every unit when the GPU has room for the whole fp32 state (~80 GB);
+    otherwise the first, a middle and the last unit.
+    """
+    w = workloads.gpt_6p7b_layerwise()
+    units = list(w.numels)
+    N = w.world
+    lay = Z.zero_partition_layout(units, N, 1)
+    parts = [lay.part(u) for u in range(len(units))]
+    shard_off = np.concatenate([[0], np.cumsum(parts)]).astype(np.int64)
+    need_gb = sum(lay.bucket_padded) * 14 / 1e9 + 6
+    run_units = list(range(len(units))) if _free_gb() > need_gb + 10 else [0, 16, len(units) - 1]
+    tdt = TD[dtype]
+    shards = [torch.empty(int(shard_off[-1]), dtype=tdt, device="cuda") for _ in range(N)]
+    max_pad = max(lay.bucket_padded)
+    layer_buf = torch.empty(max_pad, dtype=tdt, device="cuda")
+    grads = [torch.empty(max_pad, dtype=tdt, device="cuda") for _ in range(N)]
+    st = {nm: torch.empty(max_pad, dtype=torch.float32, device="cuda") for nm in ("p", "m", "v")}
+    spare = {nm: torch.empty(max_pad, dtype=torch.float32, device="cuda") for nm in ("p", "m", "v")}
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    adam = w.adam
+    hp = Z.hparams(adam.lr, adam.beta1, adam.beta2, adam.eps, adam.weight_decay, 1)
+    for u in run_units:
+        pad, P = lay.bucket_padded[u], parts[u]
+        # unit u's fp32 state (flat, rank-major) and its parameter slices in the shards
+        _device_master(st["p"][:pad], 1200 + u)
+        st["p"][lay.bucket_numel[u]:pad].zero_()
+        st["m"][:pad].zero_()
+        st["v"][:pad].zero_()
+        for r in range(N):
+            shards[r][shard_off[u]:shard_off[u] + P].copy_(st["p"][r * P:(r + 1) * P])
+        # forward/backward reconstruct: all-gather the unit into the layer buffer
+        Z.zero_allgather_params(shards, int(shard_off[u]), P, layer_buf[:pad])
+        torch.cuda.synchronize()
+        if u in (0, len(units) - 1):
+            ref_full = oracle.allgather([_u16(s[shard_off[u]:shard_off[u] + P]) for s in shards], 0, P)
+            assert np.array_equal(_u16(layer_buf[:pad]), ref_full)
+        p0 = host_f32(st["p"][:pad]).copy()
+        for k in range(N):
+            _device_grads(grads[k][:pad], workloads.seed_for(w.seed, 1, k) + 17 * u, w.grad_std, w.loss_scale)
+            grads[k][lay.bucket_numel[u]:pad].zero_()
+        flag.zero_()
+        # one fused call per rank: reduce-scatter slice r, update, write rank r's shard
+        for r in range(N):
+            sl = slice(r * P, (r + 1) * P)
+            Z.zero_reduce_scatter_adam_step([g[:pad] for g in grads], pad, r,
+                                            st["p"][sl], st["m"][sl], st["v"][sl],
+                                            spare["p"][sl], spare["m"][sl], spare["v"][sl],
+                                            shards[r][shard_off[u]:shard_off[u] + P], hp, w.loss_scale, flag)
+        torch.cuda.synchronize()
+        assert int(flag.item()) == 0
+        wins = _windows(pad, N, n_random=8, seed=u)
+        for lo, hi in wins:
+            G = [_u16(g[lo:hi]) for g in grads]
+            ref = oracle.initial_state(p0[lo:hi].copy(), dtype)
+            ovf, _ = oracle.flat_step(G, ref, adam, 1, w.loss_scale, float(N), dtype, dtype)
+            assert ovf == 0
+            assert assert_f32_close(host_f32(spare["p"][lo:hi]), ref.master, "master") == 0
+            assert assert_f32_close(host_f32(spare["m"][lo:hi]), ref.m, "m") == 0
+            assert assert_f32_close(host_f32(spare["v"][lo:hi]), ref.v, "v") == 0
+            # parameters live in the shards: element i of the unit is shard i // P, slot i % P
+            pieces = []
+            for r in range(lo // P, (hi - 1) // P + 1):
+                a = max(lo, r * P) - r * P
+                b = min(hi, (r + 1) * P) - r * P
+                pieces.append(_u16(shards[r][shard_off[u] + a:shard_off[u] + b]))
+            got = np.concatenate(pieces)
+            assert assert_u16_close(got, ref.params, "params") == 0
+
+
+@pytest.mark.parametrize("psi,world,dtype", [(1 << 20, 64, oracle.F16), (16 << 20, 16, oracle.BF16),
+                                             (256 << 20, 8, oracle.F16), (256 << 20, 2, oracle.BF16)])
+def test_sweep_points_windows(psi, world, dtype):
+    tdt = TD[dtype]
+    grads = [torch.empty(psi, dtype=tdt, device="cuda") for _ in range(world)]
+    for k in range(world):
+        _device_grads(grads[k], 5000 + k, 1e-3, 65536.0)
+    st_in = {nm: torch.empty(psi, dtype=torch.float32, device="cuda") for nm in ("p", "m", "v")}
+    _device_master(st_in["p"], 77)
+    st_in["m"].zero_()
+    st_in["v"].zero_()
+    st_out = {nm: torch.empty_like(st_in["p"]) for nm in ("p", "m", "v")}
+    params = torch.empty(psi, dtype=tdt, device="cuda")
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    adam = workloads.AdamConfig(weight_decay=0.01)
+    Z.zero_reduce_scatter_adam_step(grads, psi, Z.ZERO_ALL_PARTITIONS, st_in["p"], st_in["m"], st_in["v"],
+                                    st_out["p"], st_out["m"], st_out["v"], params,
+                                    Z.hparams(adam.lr, adam.beta1, adam.beta2, adam.eps, adam.weight_decay, 1),
+                                    65536.0, flag)
+    torch.cuda.synchronize()
+    assert int(flag.item()) == 0
+    for lo, hi in _windows(psi, world, n_random=8, seed=psi + world):
+        G = [_u16(g[lo:hi]) for g in grads]
+        ref = oracle.initial_state(host_f32(st_in["p"][lo:hi]).copy(), dtype)
+        oracle.flat_step(G, ref, adam, 1, 65536.0, float(world), dtype, dtype)
+        assert assert_f32_close(host_f32(st_out["p"][lo:hi]), ref.master, "master") == 0
+        assert assert_f32_close(host_f32(st_out["m"][lo:hi]), ref.m, "m") == 0
+        assert assert_f32_close(host_f32(st_out["v"][lo:hi]), ref.v, "v") == 0
+        assert assert_u16_close(_u16(params[lo:hi]), ref.params, "params") == 0

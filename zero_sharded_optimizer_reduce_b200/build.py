@@ -19,7 +19,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libzero.so")
 
 SOURCES = ["step.cu", "copy.cu", "host.cpp"]
-HEADERS = [os.path.join(CSRC, "common.h"), os.path.join(INCLUDE, "zero.h")]
+HEADERS = [os.path.join(CSRC, "common.h"), os.path.join(CSRC, "fused_step.cuh"), os.path.join(INCLUDE, "zero.h")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
