@@ -11,7 +11,18 @@ if HERE not in sys.path:
     sys.path.insert(0, HERE)
 
 
+def _build_libzero():
+    """Compile libzero.so if missing or stale (nvcc cross-compiles; no GPU needed)."""
+    import importlib.util
+    path = os.path.join(ROOT, "zero_sharded_optimizer_reduce_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("zero_step_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+
+
 def pytest_configure(config):
+    _build_libzero()
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running CPU test")
 

@@ -15,10 +15,7 @@ import pytest
 
 import oracle
 import workloads
-from zero_sharded_optimizer_reduce_b200 import build as zbuild
-
-zbuild.build()
-import zero_sharded_optimizer_reduce_b200 as Z  # noqa: E402
+import zero_sharded_optimizer_reduce_b200 as Z
 
 HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "zero.h")
 

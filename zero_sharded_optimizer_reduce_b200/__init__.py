@@ -52,7 +52,7 @@ class AdamHParams(ctypes.Structure):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
-                          "`python -m zero_sharded_optimizer_reduce_b200.build` (nvcc, sm_100a)")
+                          "`python zero_sharded_optimizer_reduce_b200/build.py` (nvcc, sm_100a)")
     L = ctypes.CDLL(LIB_PATH)
     vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
     L.zero_partition_layout.argtypes = [ctypes.POINTER(ctypes.c_int64), i64, i32, i64, i32,

@@ -1,6 +1,9 @@
 """Build libzero.so (the C ABI of include/zero.h) for sm_100a with nvcc.
 
-    python -m zero_sharded_optimizer_reduce_b200.build [--verbose-ptxas]
+    python zero_sharded_optimizer_reduce_b200/build.py [--verbose-ptxas]
+
+Run it as a script (or load it by path): importing the package loads the
+library, so the package cannot build itself on import.
 
 The library is built in-tree, next to this file.  nvcc cross-compiles, so no
 GPU is needed to build.
