@@ -225,6 +225,47 @@ int zero_reduce_scatter_adam_step(
     zero_stream_t stream);
 
 /*
+ * zero_reduce_scatter_adam_step_noalloc - zero_reduce_scatter_adam_step for
+ * callers that cannot allocate device memory.
+ *
+ * The paper has no counterpart: this is a calling convention of this
+ * library, not a step of the method.  Some callers cannot provide the
+ * device workspace that the gradient norm needs: code under an allocator
+ * that owns all device memory and forbids direct cudaMalloc, a host thread
+ * that must not take cudaMalloc's implicit device synchronization, or a C
+ * caller with no device allocator.  This entry point takes the same
+ * arguments minus `workspace` and keeps that scratch in a fixed array in the
+ * library's device image instead (16,640 bytes per GPU that loads the
+ * library, held until exit); it calls no cudaMalloc, cudaFree or other
+ * allocating routine.  Inputs and outputs are still the caller's.
+ *
+ * Results equal those of zero_reduce_scatter_adam_step.  Limits:
+ *  - the scratch holds 4096 per-block partial sums; the kernel's grid is
+ *    SM count x resident blocks, so every input size fits, and a call whose
+ *    grid would exceed 4096 blocks returns ZERO_ERR_RANGE;
+ *  - all calls on a device share the scratch: calls that overlap on the GPU
+ *    (other streams, other host threads) race on it; each call clears the
+ *    ticket word it needs before its kernel, stream-ordered;
+ *  - the first call on a device that passes grad_sqnorm looks up the
+ *    scratch's device address (cudaGetSymbolAddress, once per device, with
+ *    that device current): make that first call before any stream capture.
+ * Errors: those of zero_reduce_scatter_adam_step, plus ZERO_ERR_RANGE above.
+ */
+int zero_reduce_scatter_adam_step_noalloc(
+    const void* const* grad_bufs, int32_t world, int64_t padded_numel, int32_t partition,
+    zero_dtype_t grad_dtype,
+    const float* master_in, const float* m_in, const float* v_in,
+    float* master_out, float* m_out, float* v_out,
+    void* param_out, zero_dtype_t param_dtype,
+    const zero_adam_hparams_t* hp, float loss_scale,
+    int32_t* overflow_flag, double* grad_sqnorm,
+    zero_stream_t stream);
+
+/* Bytes of the fixed scratch array used by
+ * zero_reduce_scatter_adam_step_noalloc (per GPU that loads the library). */
+size_t zero_step_static_scratch_bytes(void);
+
+/*
  * zero_allgather_params - rebuild full parameters from N rank shards.
  *
  * Source: ZeRO explainer, "Stage 3 - Parameter Partitioning (P_os+g+p)" (each

@@ -69,6 +69,13 @@ def _load():
         vp, vp, vp, vp, vp, vp, vp, ctypes.c_int,
         ctypes.POINTER(AdamHParams), f32, vp, vp, vp, vp]
     L.zero_reduce_scatter_adam_step.restype = ctypes.c_int
+    L.zero_reduce_scatter_adam_step_noalloc.argtypes = [
+        ctypes.POINTER(vp), i32, i64, i32, ctypes.c_int,
+        vp, vp, vp, vp, vp, vp, vp, ctypes.c_int,
+        ctypes.POINTER(AdamHParams), f32, vp, vp, vp]
+    L.zero_reduce_scatter_adam_step_noalloc.restype = ctypes.c_int
+    L.zero_step_static_scratch_bytes.argtypes = []
+    L.zero_step_static_scratch_bytes.restype = ctypes.c_size_t
     L.zero_allgather_params.argtypes = [ctypes.POINTER(vp), i32, i64, i64, ctypes.c_int, vp, vp]
     L.zero_allgather_params.restype = ctypes.c_int
     L.zero_loss_scale_update.argtypes = [ctypes.POINTER(f32), ctypes.POINTER(i32), i32, i32, f32]
@@ -202,6 +209,21 @@ def zero_reduce_scatter_adam_step(grad_bufs, padded_numel: int, partition: int,
         _ptr(master_in), _ptr(m_in), _ptr(v_in), _ptr(master_out), _ptr(m_out), _ptr(v_out),
         _ptr(param_out), _dtype_code(param_out), ctypes.byref(hp), float(loss_scale),
         _ptr(overflow_flag), _ptr(grad_sqnorm), _ptr(workspace), _stream(stream)))
+
+
+def zero_reduce_scatter_adam_step_noalloc(grad_bufs, padded_numel: int, partition: int,
+                                          master_in, m_in, v_in, master_out, m_out, v_out, param_out,
+                                          hp: AdamHParams, loss_scale: float, overflow_flag,
+                                          grad_sqnorm=None, stream=None) -> None:
+    """The fused step without a workspace argument, for callers that cannot
+    allocate device memory: the norm's scratch lives in a fixed array inside
+    libzero (see include/zero.h for its limits)."""
+    world = len(grad_bufs)
+    _check(lib.zero_reduce_scatter_adam_step_noalloc(
+        _ptrs(grad_bufs), world, padded_numel, partition, _dtype_code(grad_bufs[0]),
+        _ptr(master_in), _ptr(m_in), _ptr(v_in), _ptr(master_out), _ptr(m_out), _ptr(v_out),
+        _ptr(param_out), _dtype_code(param_out), ctypes.byref(hp), float(loss_scale),
+        _ptr(overflow_flag), _ptr(grad_sqnorm), _stream(stream)))
 
 
 def zero_allgather_params(shards, shard_offset: int, part_numel: int, dst, stream=None) -> None:
