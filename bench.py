@@ -327,7 +327,8 @@ def run_gpu(args):
                 "hbm_gbs": value * 1e9 * bpe / world_gpus / 1e9,
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
                              "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
-                             "kernel": "fused_step_kernel", "bytes_per_elem": bpe,
+                             "kernel": "fused_step (shared-memory pipeline kernel for aligned calls of >= 2 tiles per SM)",
+                             "bytes_per_elem": bpe,
                              "elems_per_launch": avg_elems, "launches_timed": len(launch_ms)},
                 "gpu_launches": args.steps * L.n_buckets,
                 "applied_steps": applied,
@@ -338,6 +339,62 @@ def run_gpu(args):
     if world_gpus > 1:
         dist.barrier()
         dist.destroy_process_group()
+    return 0
+
+
+def run_sweep(args):
+    """Flat bandwidth sweep: psi in {1M, 16M, 256M, 1B, 2B} x N in {1..64}
+    (N x 2 x psi <= 96 GB), fp16 and bf16; one JSON line per point.  Each
+    step is timed on its own with CUDA events; when a point's footprint is
+    below 4x L2 an L2-sized buffer is written between steps (untimed)."""
+    import torch
+    import zero_sharded_optimizer_reduce_b200 as Z
+    torch.cuda.set_device(0)
+    peak, peak_kind = peaks()
+    free_gb = torch.cuda.mem_get_info()[0] / 1e9
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    dtypes = [args.grad_dtype] if args.sweep_dtype_only else ["f16", "bf16"]
+    for dt in dtypes:
+        gdt = torch.bfloat16 if dt == "bf16" else torch.float16
+        for psi, N in workloads.sweep_points():
+            need = psi * (2 * N + 28) / 1e9 + 1
+            if need > 0.92 * free_gb:
+                print(json.dumps({"sweep": True, "psi": psi, "world": N, "grad_dtype": dt,
+                                  "skipped": f"needs {need:.0f} GB"}), flush=True)
+                continue
+            w = workloads.Workload(f"flat_{psi}_n{N}_{dt}", (psi,), N, 65536.0, 1,
+                                   workloads.AdamConfig(weight_decay=0.01), seed=5)
+            opt = Z.ZeroAdam(w.numels, N, 0, lr=w.adam.lr, weight_decay=0.01, loss_scale=65536.0,
+                             grad_dtype=gdt, param_dtype=gdt)
+            fill_workload(opt, w, w.seed)
+            bpe = bytes_per_elem(N)
+            small = psi * bpe < 4 * 126e6
+            for _ in range(3):
+                opt.step()
+            times = []
+            for _ in range(args.steps):
+                if small:
+                    flush.fill_(1)
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                ms_launch = []
+
+                def on_launch(b, phase, _l=ms_launch):
+                    e = torch.cuda.Event(enable_timing=True)
+                    e.record()
+                    _l.append(e)
+                opt.step(on_launch=on_launch)
+                torch.cuda.synchronize()
+                times.append(ms_launch[0].elapsed_time(ms_launch[1]))
+            ms = statistics.median(times)
+            gbs = psi * bpe / (ms * 1e-3) / 1e9
+            print(json.dumps({"sweep": True, "psi": psi, "world": N, "grad_dtype": dt,
+                              "kernel_ms_median": ms, "gparams_s": psi / (ms * 1e-3) / 1e9, "gbs": gbs,
+                              "frac_measured": gbs / peak, "frac_nominal_8tbs": gbs / 8000.0,
+                              "l2": "L2-influenced (footprint < 4x L2, flushed between steps)" if small
+                              else "footprint > 4x L2"}), flush=True)
+            del opt
+            torch.cuda.empty_cache()
     return 0
 
 
@@ -394,11 +451,15 @@ def main(argv=None):
     ap.add_argument("--flat", type=int, default=0, help="flat workload of this many elements instead of GPT-2")
     ap.add_argument("--world", type=int, default=8, help="simulated replicas of the flat workload")
     ap.add_argument("--grad-dtype", choices=["f16", "bf16"], default="f16")
+    ap.add_argument("--sweep", action="store_true", help="flat bandwidth sweep, one JSON line per point")
+    ap.add_argument("--sweep-dtype-only", action="store_true", help="sweep only --grad-dtype")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
     return run_gpu(args)
 
 

@@ -197,10 +197,14 @@ size_t zero_step_workspace_bytes(void);
  *              the all-gather payload, in the same indexing as the states
  * hp           host, hyper-parameters; hp->step >= 1
  * loss_scale   > 0 and finite: the gradients carry this factor
- * overflow_flag device int32; set to 1 if any reduced gradient of this call
- *              is inf or NaN, never written otherwise.  Clear it before the
- *              first call of a step; calls over several buckets then OR into
- *              one flag for the whole step.
+ * overflow_flag device int32, OR-ed into, never cleared by the call:
+ *              bit 0 (value 1) when any reduced gradient of this call is inf
+ *              or NaN; bit 1 (value 2) when the kernel gave up waiting on its
+ *              own shared-memory copy pipeline (2 s without progress: a device
+ *              fault, not a property of the data) and its outputs are
+ *              incomplete.  Commit a step only when the flag is 0.  Clear it
+ *              before the first call of a step; calls over several buckets
+ *              then OR into one flag for the whole step.
  * grad_sqnorm  device double or NULL; when not NULL, sum over the call's
  *              elements of g*g is ADDED to it (clear it at the start of a
  *              step).  Deterministic: per-block fp32 partial sums folded in a
@@ -241,8 +245,9 @@ int zero_reduce_scatter_adam_step(
  *
  * Results equal those of zero_reduce_scatter_adam_step.  Limits:
  *  - the scratch holds 4096 per-block partial sums; the kernel's grid is
- *    SM count x resident blocks, so every input size fits, and a call whose
- *    grid would exceed 4096 blocks returns ZERO_ERR_RANGE;
+ *    SM count x resident blocks (at most 296 on a B200), so every input
+ *    size fits, and a call whose grid would exceed 4096 blocks returns
+ *    ZERO_ERR_RANGE;
  *  - all calls on a device share the scratch: calls that overlap on the GPU
  *    (other streams, other host threads) race on it; each call clears the
  *    ticket word it needs before its kernel, stream-ordered;

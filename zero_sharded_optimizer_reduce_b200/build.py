@@ -22,7 +22,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libzero.so")
 
 SOURCES = ["step.cu", "step_static.cu", "copy.cu", "host.cpp"]
-HEADERS = [os.path.join(CSRC, "common.h"), os.path.join(CSRC, "fused_step.cuh"), os.path.join(INCLUDE, "zero.h")]
+HEADERS = [os.path.join(CSRC, n) for n in ("common.h", "fused_step.cuh", "step_launch.h")] + [os.path.join(INCLUDE, "zero.h")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

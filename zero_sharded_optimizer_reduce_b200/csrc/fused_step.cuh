@@ -37,6 +37,7 @@ struct StepParams {
     int64_t count;  // elements processed
     int64_t head;   // elements [0, head) take the scalar path
     int64_t nvec;   // vectors of kVec elements starting at `head`
+    int32_t tile;   // 0: register-streaming kernel; else elements per pipeline tile
     const float* master_in;
     const float* m_in;
     const float* v_in;
@@ -72,6 +73,10 @@ __device__ __forceinline__ float4 ld_state16(const float* p) {
 __device__ __forceinline__ void st_state16(float* p, float a, float b, float c, float d) {
     asm volatile("st.global.v4.f32 [%0], {%1,%2,%3,%4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
                  : "memory");
+}
+
+__device__ __forceinline__ void st_u16x4(void* p, uint2 v) {
+    asm volatile("st.global.v2.u32 [%0], {%1,%2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
 }
 
 __device__ __forceinline__ void st_u16x8(void* p, uint4 v) {
@@ -159,6 +164,69 @@ __device__ __forceinline__ double warp_sum_d(double x) {
     return x;
 }
 
+// Elements outside the vector (or tile) region: [0, head) and
+// [head + nvec*kVec, count), one element per thread and iteration.
+template <typename GT, typename PT>
+__device__ __forceinline__ void scalar_elements(const StepParams& p, const Consts& c, int64_t tid, int64_t nthreads,
+                                                bool& bad, float& sq) {
+    const int world = p.world;
+    const int64_t vec_end = p.head + p.nvec * kVec;
+    const int64_t nscalar = p.head + (p.count - vec_end);
+    for (int64_t q = tid; q < nscalar; q += nthreads) {
+        const int64_t e = q < p.head ? q : vec_end + (q - p.head);
+        float s = Fmt<GT>::one(static_cast<const uint16_t*>(p.grads[0])[e]);
+        for (int k = 1; k < world; ++k)
+            s = __fadd_rn(s, Fmt<GT>::one(static_cast<const uint16_t*>(p.grads[k])[e]));
+        float pw = p.master_in[e], mw = p.m_in[e], vw = p.v_in[e];
+        bad |= !isfinite(s);
+        const float g = adam(s, pw, mw, vw, c);
+        sq = __fmaf_rn(g, g, sq);
+        p.master_out[e] = pw;
+        p.m_out[e] = mw;
+        p.v_out[e] = vw;
+        static_cast<uint16_t*>(p.param_out)[e] = Fmt<PT>::round1(pw);
+    }
+}
+
+// Overflow vote and the optional deterministic norm fold.  Every thread of
+// the block must call it (it synchronizes the block).
+template <int NT>
+__device__ __forceinline__ void finish_block(const StepParams& p, bool bad, float sq) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // one atomic per warp that saw a non-finite sum
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.overflow, 1);
+    if (p.sqnorm == nullptr) return;
+    __shared__ float wsum[NT / 32];
+    __shared__ bool last;
+    sq = warp_sum(sq);
+    if (lane == 0) wsum[warp] = sq;
+    __syncthreads();
+    if (warp == 0) {
+        float x = lane < NT / 32 ? wsum[lane] : 0.0f;
+        x = warp_sum(x);
+        if (lane == 0) {
+            p.partials[blockIdx.x] = x;
+            __threadfence();
+            const unsigned int t = atomicAdd(p.ticket, 1u);
+            last = (t == gridDim.x - 1);
+        }
+    }
+    __syncthreads();
+    if (last && warp == 0) {
+        __threadfence();
+        double acc = 0.0;
+        for (unsigned int b = lane; b < gridDim.x; b += 32) acc += static_cast<double>(__ldcg(p.partials + b));
+        acc = warp_sum_d(acc);
+        if (lane == 0) {
+            *p.sqnorm += acc;
+            *p.ticket = 0u;  // leave the workspace ready for the next call
+        }
+    }
+}
+
+// Register-streaming kernel: each thread loads its kVec elements of every
+// stream straight into registers.  Used for buffers whose 16-byte phases
+// differ, for small calls and for very large N.
 template <typename GT, typename PT>
 __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_constant__ StepParams p) {
     const int64_t tid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
@@ -220,246 +288,219 @@ __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_const
         st_u16x8(static_cast<uint16_t*>(p.param_out) + e0, q);
     }
 
-    // ---- scalar path: the head before and the tail after the vector region
-    const int64_t vec_end = p.head + p.nvec * kVec;
-    const int64_t nscalar = p.head + (p.count - vec_end);
-    for (int64_t q = tid; q < nscalar; q += nthreads) {
-        const int64_t e = q < p.head ? q : vec_end + (q - p.head);
-        float s = Fmt<GT>::one(static_cast<const uint16_t*>(p.grads[0])[e]);
-        for (int k = 1; k < world; ++k)
-            s = __fadd_rn(s, Fmt<GT>::one(static_cast<const uint16_t*>(p.grads[k])[e]));
-        float pw = p.master_in[e], mw = p.m_in[e], vw = p.v_in[e];
-        bad |= !isfinite(s);
-        const float g = adam(s, pw, mw, vw, c);
-        sq = __fmaf_rn(g, g, sq);
-        p.master_out[e] = pw;
-        p.m_out[e] = mw;
-        p.v_out[e] = vw;
-        static_cast<uint16_t*>(p.param_out)[e] = Fmt<PT>::round1(pw);
+    scalar_elements<GT, PT>(p, c, tid, nthreads, bad, sq);
+    finish_block<kThreads>(p, bad, sq);
+}
+
+// ------------------------------------------------------- bulk-copy pipeline
+
+__device__ __forceinline__ uint32_t smem_addr(const void* ptr) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(ptr));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for the phase of `bar` with the given parity, for at most
+// kWaitLimitNs of wall time.  Returns false when the limit ran out.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
     }
+}
 
-    // ---- overflow flag: one atomic per warp that saw a non-finite sum
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.overflow, 1);
+// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
+// No multicast: the destination is the issuing CTA's own shared memory.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
 
-    // ---- optional squared norm, deterministic fold by the last block
-    if (p.sqnorm != nullptr) {
-        __shared__ float wsum[kThreads / 32];
-        __shared__ bool last;
-        sq = warp_sum(sq);
-        if (lane == 0) wsum[warp] = sq;
-        __syncthreads();
-        if (warp == 0) {
-            float x = lane < kThreads / 32 ? wsum[lane] : 0.0f;
-            x = warp_sum(x);
-            if (lane == 0) {
-                p.partials[blockIdx.x] = x;
-                __threadfence();
-                const unsigned int t = atomicAdd(p.ticket, 1u);
-                last = (t == gridDim.x - 1);
+constexpr int kPipeStages = 2;
+constexpr int kPipeConsumerWarps = 16;
+constexpr int kPipeThreads = (kPipeConsumerWarps + 1) * 32;   // + one producer warp
+
+// Device bit set in *overflow when a pipeline wait ran out of time: the
+// call's outputs are incomplete and must not be committed.
+constexpr int32_t kFlagDeviceTimeout = 2;
+
+// Pipeline kernel: one CTA per SM.  A producer warp streams tiles of `tile`
+// elements of every input (N gradient slices, master, m, v) into a ring of
+// kPipeStages shared-memory stages with 1-D bulk copies that complete on an
+// mbarrier; kPipeConsumerWarps warps reduce, update and store each tile
+// straight to global memory (coalesced 16-byte stores) and release the
+// stage.  Stage layout: N x tile gradients, then tile x fp32 master, m, v.
+template <typename GT, typename PT>
+__global__ void __launch_bounds__(kPipeThreads, 1) fused_step_pipe_kernel(const __grid_constant__ StepParams p) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ __align__(8) uint64_t full[kPipeStages];
+    __shared__ __align__(8) uint64_t empty[kPipeStages];
+    __shared__ int abort_flag;
+    const int world = p.world;
+    const int T = p.tile;
+    const uint32_t gbytes = 2u * static_cast<uint32_t>(T);
+    const uint32_t sbytes = 4u * static_cast<uint32_t>(T);
+    const uint32_t stage = static_cast<uint32_t>(world) * gbytes + 3u * sbytes;
+    const int64_t ntiles = p.nvec * kVec / T;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPipeStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kPipeConsumerWarps);
+        }
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    const Consts c = p.c;
+    bool bad = false;
+    float sq = 0.0f;
+
+    if (warp == kPipeConsumerWarps) {
+        // ---- producer warp: lane 0 arms the stage, all lanes issue copies
+        int64_t i = 0;
+        for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+            const int s = static_cast<int>(i % kPipeStages);
+            const uint32_t ph = static_cast<uint32_t>((i / kPipeStages) & 1);
+            bool ok = true;
+            if (i >= kPipeStages && lane == 0) ok = mbar_wait_bounded(&empty[s], ph ^ 1u);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) {
+                if (lane == 0) {
+                    atomicOr(p.overflow, kFlagDeviceTimeout);
+                    abort_flag = 1;
+                }
+                break;
+            }
+            if (__shfl_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&abort_flag), 0)) break;
+            unsigned char* st = smem + static_cast<size_t>(s) * stage;
+            if (lane == 0) mbar_arrive_expect_tx(&full[s], stage);
+            __syncwarp();
+            const int64_t e0 = p.head + tile * T;
+            for (int q = lane; q < world + 3; q += 32) {
+                if (q < 3) {
+                    const float* src = q == 0 ? p.master_in : (q == 1 ? p.m_in : p.v_in);
+                    bulk_load(st + static_cast<size_t>(world) * gbytes + q * sbytes, src + e0, sbytes, &full[s]);
+                } else {
+                    const int k = q - 3;
+                    bulk_load(st + static_cast<size_t>(k) * gbytes, static_cast<const uint16_t*>(p.grads[k]) + e0,
+                              gbytes, &full[s]);
+                }
             }
         }
-        __syncthreads();
-        if (last && warp == 0) {
-            __threadfence();
-            double acc = 0.0;
-            for (unsigned int b = lane; b < gridDim.x; b += 32) acc += static_cast<double>(__ldcg(p.partials + b));
-            acc = warp_sum_d(acc);
-            if (lane == 0) {
-                *p.sqnorm += acc;
-                *p.ticket = 0u;  // leave the workspace ready for the next call
-            }
+        // drain: this CTA's copies must land before it exits (bounded)
+        if (lane == 0) {
+            const int64_t issued = i;
+            for (int64_t j = issued > kPipeStages ? issued - kPipeStages : 0; j < issued; ++j)
+                if (!mbar_wait_bounded(&full[j % kPipeStages], static_cast<uint32_t>((j / kPipeStages) & 1)))
+                    atomicOr(p.overflow, kFlagDeviceTimeout);
         }
+        __syncwarp();
+    } else {
+        // ---- consumer warps: thread t takes 4 elements per chunk
+        constexpr int C = kPipeConsumerWarps * 32;
+        const int t = threadIdx.x;
+        int64_t i = 0;
+        for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+            const int s = static_cast<int>(i % kPipeStages);
+            const uint32_t ph = static_cast<uint32_t>((i / kPipeStages) & 1);
+            bool ok = true;
+            if (lane == 0) ok = !*reinterpret_cast<volatile int*>(&abort_flag) && mbar_wait_bounded(&full[s], ph);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) {
+                if (lane == 0) {
+                    atomicOr(p.overflow, kFlagDeviceTimeout);
+                    abort_flag = 1;
+                }
+                break;
+            }
+            const unsigned char* st = smem + static_cast<size_t>(s) * stage;
+            const float* sm_p = reinterpret_cast<const float*>(st + static_cast<size_t>(world) * gbytes);
+            const float* sm_m = sm_p + T;
+            const float* sm_v = sm_m + T;
+            const int64_t base = p.head + tile * T;
+            for (int ch = t; ch < T / 4; ch += C) {
+                const int j = 4 * ch;
+                float sacc[4];
+                const uint2 r0 = *reinterpret_cast<const uint2*>(st + 2 * j);
+                sacc[0] = Fmt<GT>::lo(r0.x);
+                sacc[1] = Fmt<GT>::hi(r0.x);
+                sacc[2] = Fmt<GT>::lo(r0.y);
+                sacc[3] = Fmt<GT>::hi(r0.y);
+#pragma unroll 4
+                for (int k = 1; k < world; ++k) {
+                    const uint2 r = *reinterpret_cast<const uint2*>(st + static_cast<size_t>(k) * gbytes + 2 * j);
+                    sacc[0] = __fadd_rn(sacc[0], Fmt<GT>::lo(r.x));
+                    sacc[1] = __fadd_rn(sacc[1], Fmt<GT>::hi(r.x));
+                    sacc[2] = __fadd_rn(sacc[2], Fmt<GT>::lo(r.y));
+                    sacc[3] = __fadd_rn(sacc[3], Fmt<GT>::hi(r.y));
+                }
+                float4 pw = *reinterpret_cast<const float4*>(sm_p + j);
+                float4 mw = *reinterpret_cast<const float4*>(sm_m + j);
+                float4 vw = *reinterpret_cast<const float4*>(sm_v + j);
+                bad |= !isfinite(sacc[0]) | !isfinite(sacc[1]) | !isfinite(sacc[2]) | !isfinite(sacc[3]);
+                float g;
+                g = adam(sacc[0], pw.x, mw.x, vw.x, c);
+                sq = __fmaf_rn(g, g, sq);
+                g = adam(sacc[1], pw.y, mw.y, vw.y, c);
+                sq = __fmaf_rn(g, g, sq);
+                g = adam(sacc[2], pw.z, mw.z, vw.z, c);
+                sq = __fmaf_rn(g, g, sq);
+                g = adam(sacc[3], pw.w, mw.w, vw.w, c);
+                sq = __fmaf_rn(g, g, sq);
+                st_state16(p.master_out + base + j, pw.x, pw.y, pw.z, pw.w);
+                st_state16(p.m_out + base + j, mw.x, mw.y, mw.z, mw.w);
+                st_state16(p.v_out + base + j, vw.x, vw.y, vw.z, vw.w);
+                uint2 pk;
+                pk.x = Fmt<PT>::pack(pw.x, pw.y);
+                pk.y = Fmt<PT>::pack(pw.z, pw.w);
+                st_u16x4(static_cast<uint16_t*>(p.param_out) + base + j, pk);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+        }
+        // the scalar head and tail, spread over every consumer thread of the grid
+        scalar_elements<GT, PT>(p, c, static_cast<int64_t>(blockIdx.x) * C + t, static_cast<int64_t>(gridDim.x) * C,
+                                bad, sq);
     }
+    finish_block<kPipeThreads>(p, bad, sq);
 }
 
 // ------------------------------------------------------------------ host side
-
-using KernelFn = void (*)(StepParams);
-
-inline KernelFn pick_kernel(zero_dtype_t g, zero_dtype_t pd) {
-    if (g == ZERO_F16 && pd == ZERO_F16) return fused_step_kernel<__half, __half>;
-    if (g == ZERO_F16 && pd == ZERO_BF16) return fused_step_kernel<__half, __nv_bfloat16>;
-    if (g == ZERO_BF16 && pd == ZERO_F16) return fused_step_kernel<__nv_bfloat16, __half>;
-    return fused_step_kernel<__nv_bfloat16, __nv_bfloat16>;
-}
-
-struct DeviceInfo {
-    int sms = 0;
-    int blocks_per_sm[4] = {0, 0, 0, 0};
-};
-
-std::mutex g_dev_mu;
-DeviceInfo g_dev[64];
-
-inline int grid_limit(zero_dtype_t g, zero_dtype_t pd, int* out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
-        return fail(ZERO_ERR_CUDA, "cudaGetDevice failed");
-    const int which = static_cast<int>(g) * 2 + static_cast<int>(pd);
-    std::lock_guard<std::mutex> lk(g_dev_mu);
-    DeviceInfo& d = g_dev[dev];
-    if (d.sms == 0) {
-        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return fail(ZERO_ERR_CUDA, "cannot query the SM count");
-    }
-    if (d.blocks_per_sm[which] == 0) {
-        int n = 0;
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, pick_kernel(g, pd), kThreads, 0);
-        if (e != cudaSuccess || n < 1) return fail(ZERO_ERR_CUDA, "occupancy query failed: %s", cudaGetErrorString(e));
-        d.blocks_per_sm[which] = n;
-    }
-    int lim = d.sms * d.blocks_per_sm[which];
-    *out = lim < kMaxBlocks ? lim : kMaxBlocks;
-    return ZERO_OK;
-}
-
-// Smallest h in [0, kVec) at which every array sits on a 16-byte boundary,
-// or -1 if their phases never coincide.
-inline int64_t common_phase(const StepParams& p) {
-    for (int64_t h = 0; h < kVec; ++h) {
-        bool good = true;
-        for (int k = 0; k < p.world && good; ++k)
-            good = ((reinterpret_cast<uintptr_t>(p.grads[k]) + 2 * h) % 16) == 0;
-        const void* f32s[] = {p.master_in, p.m_in, p.v_in, p.master_out, p.m_out, p.v_out};
-        for (const void* a : f32s) good = good && ((reinterpret_cast<uintptr_t>(a) + 4 * h) % 16) == 0;
-        good = good && ((reinterpret_cast<uintptr_t>(p.param_out) + 2 * h) % 16) == 0;
-        if (good) return h;
-    }
-    return -1;
-}
-
-
-// Validate the arguments of a fused-step call and build its kernel
-// parameters and grid size.  `workspace` is the scratch used for the
-// gradient norm (ticket + per-block partials).  On success *blocks_out is the
-// number of blocks to launch (0: nothing to do).
-inline int prepare_step(const char* fn, const void* const* grad_bufs, int32_t world, int64_t padded_numel,
-                        int32_t partition, zero_dtype_t grad_dtype, const float* master_in, const float* m_in,
-                        const float* v_in, float* master_out, float* m_out, float* v_out, void* param_out,
-                        zero_dtype_t param_dtype, const zero_adam_hparams_t* hp, float loss_scale,
-                        int32_t* overflow_flag, double* grad_sqnorm, void* workspace, StepParams* prm_out,
-                        int64_t* blocks_out) {
-    if (!grad_bufs || !hp || !overflow_flag) return fail(ZERO_ERR_ARG, "%s: NULL grad_bufs, hp or overflow_flag", fn);
-    if (world < 1 || world > ZERO_MAX_WORLD)
-        return fail(ZERO_ERR_ARG, "%s: world %d outside 1..%d", fn, world, ZERO_MAX_WORLD);
-    if (padded_numel < 0 || padded_numel % world != 0)
-        return fail(ZERO_ERR_ARG, "%s: padded_numel %lld is not a non-negative multiple of world %d", fn,
-                    (long long)padded_numel, world);
-    if (partition != ZERO_ALL_PARTITIONS && (partition < 0 || partition >= world))
-        return fail(ZERO_ERR_RANGE, "%s: partition %d outside 0..%d", fn, partition, world - 1);
-    if ((grad_dtype != ZERO_F16 && grad_dtype != ZERO_BF16) || (param_dtype != ZERO_F16 && param_dtype != ZERO_BF16))
-        return fail(ZERO_ERR_DTYPE, "%s: gradients and parameters must be ZERO_F16 or ZERO_BF16", fn);
-    if (!(hp->step >= 1)) return fail(ZERO_ERR_ARG, "%s: hp->step must be >= 1", fn);
-    if (!std::isfinite(hp->lr) || !std::isfinite(hp->eps) || !std::isfinite(hp->weight_decay) ||
-        !(hp->beta1 >= 0.0f && hp->beta1 < 1.0f) || !(hp->beta2 >= 0.0f && hp->beta2 < 1.0f) ||
-        !(hp->grad_divisor >= 0.0f) || !std::isfinite(hp->grad_divisor))
-        return fail(ZERO_ERR_ARG, "%s: hyper-parameters out of range", fn);
-    if (!(loss_scale > 0.0f) || !std::isfinite(loss_scale))
-        return fail(ZERO_ERR_ARG, "%s: loss_scale must be positive and finite", fn);
-    if (grad_sqnorm && !workspace) return fail(ZERO_ERR_ARG, "%s: grad_sqnorm needs a workspace", fn);
-    if (!aligned(overflow_flag, 4) || (grad_sqnorm && !aligned(grad_sqnorm, 8)) ||
-        (workspace && !aligned(workspace, 16)))
-        return fail(ZERO_ERR_ALIGN, "%s: flag, norm or workspace misaligned", fn);
-
-    const int64_t P = padded_numel / world;
-    const int64_t begin = partition == ZERO_ALL_PARTITIONS ? 0 : static_cast<int64_t>(partition) * P;
-    const int64_t count = partition == ZERO_ALL_PARTITIONS ? padded_numel : P;
-    if (count == 0) {
-        *blocks_out = 0;
-        return ZERO_OK;
-    }
-
-    const float* f_in[] = {master_in, m_in, v_in};
-    float* f_out[] = {master_out, m_out, v_out};
-    for (int i = 0; i < 3; ++i) {
-        if (!f_in[i] || !f_out[i]) return fail(ZERO_ERR_ARG, "%s: NULL state pointer", fn);
-        if (!aligned(f_in[i], 4) || !aligned(f_out[i], 4)) return fail(ZERO_ERR_ALIGN, "%s: fp32 state not 4-byte aligned", fn);
-    }
-    if (!param_out) return fail(ZERO_ERR_ARG, "%s: NULL param_out", fn);
-    if (!aligned(param_out, 2)) return fail(ZERO_ERR_ALIGN, "%s: param_out not 2-byte aligned", fn);
-    for (int k = 0; k < world; ++k) {
-        if (!grad_bufs[k]) return fail(ZERO_ERR_ARG, "%s: grad_bufs[%d] is NULL", fn, k);
-        if (!aligned(grad_bufs[k], 2)) return fail(ZERO_ERR_ALIGN, "%s: grad_bufs[%d] not 2-byte aligned", fn, k);
-    }
-    // outputs: each output either is its own input (in place) or overlaps
-    // nothing else; outputs never overlap each other or a gradient buffer
-    const int64_t fb = count * 4, pb = count * 2, gb = padded_numel * 2;
-    const void* outs[] = {master_out, m_out, v_out, param_out};
-    const int64_t out_bytes[] = {fb, fb, fb, pb};
-    for (int i = 0; i < 4; ++i) {
-        for (int j = i + 1; j < 4; ++j)
-            if (overlaps(outs[i], out_bytes[i], outs[j], out_bytes[j]))
-                return fail(ZERO_ERR_ARG, "%s: output arrays overlap", fn);
-        for (int j = 0; j < 3; ++j)
-            if (!(i == j && outs[i] == f_in[j]) && overlaps(outs[i], out_bytes[i], f_in[j], fb))
-                return fail(ZERO_ERR_ARG, "%s: an output overlaps an input it does not replace", fn);
-        for (int k = 0; k < world; ++k)
-            if (overlaps(outs[i], out_bytes[i], grad_bufs[k], gb))
-                return fail(ZERO_ERR_ARG, "%s: an output overlaps grad_bufs[%d]", fn, k);
-    }
-
-    StepParams prm{};
-    prm.world = world;
-    for (int k = 0; k < world; ++k) prm.grads[k] = static_cast<const uint16_t*>(grad_bufs[k]) + begin;
-    prm.count = count;
-    prm.master_in = master_in;
-    prm.m_in = m_in;
-    prm.v_in = v_in;
-    prm.master_out = master_out;
-    prm.m_out = m_out;
-    prm.v_out = v_out;
-    prm.param_out = param_out;
-    prm.overflow = overflow_flag;
-    prm.sqnorm = grad_sqnorm;
-    if (grad_sqnorm) {
-        prm.ticket = static_cast<unsigned int*>(workspace);
-        prm.partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + kWsPartialsOffset);
-    }
-    // constants: double, rounded once to float
-    const double divisor = hp->grad_divisor > 0.0f ? static_cast<double>(hp->grad_divisor) : static_cast<double>(world);
-    const double t = static_cast<double>(hp->step);
-    prm.c.lr = hp->lr;
-    prm.c.b1 = hp->beta1;
-    prm.c.b2 = hp->beta2;
-    prm.c.eps = hp->eps;
-    prm.c.inv = static_cast<float>(1.0 / (divisor * static_cast<double>(loss_scale)));
-    prm.c.omb1 = static_cast<float>(1.0 - static_cast<double>(hp->beta1));
-    prm.c.omb2 = static_cast<float>(1.0 - static_cast<double>(hp->beta2));
-    prm.c.rbc1 = static_cast<float>(1.0 / (1.0 - std::pow(static_cast<double>(hp->beta1), t)));
-    prm.c.rsbc2 = static_cast<float>(1.0 / std::sqrt(1.0 - std::pow(static_cast<double>(hp->beta2), t)));
-    prm.c.decay = static_cast<float>(1.0 - static_cast<double>(hp->lr) * static_cast<double>(hp->weight_decay));
-
-    const int64_t h = common_phase(prm);
-    if (h < 0 || h >= count) {
-        prm.head = count;
-        prm.nvec = 0;
-    } else {
-        prm.head = h;
-        prm.nvec = (count - h) / kVec;
-    }
-
-    int limit = 0;
-    if (int rc = grid_limit(grad_dtype, param_dtype, &limit)) return rc;
-    const int64_t work = prm.nvec > 0 ? prm.nvec : count;
-    int64_t blocks = (work + kThreads - 1) / kThreads;
-    if (blocks > limit) blocks = limit;
-    if (blocks < 1) blocks = 1;
-    *prm_out = prm;
-    *blocks_out = blocks;
-    return ZERO_OK;
-}
-
-// Enqueue the fused kernel prepared by prepare_step.
-inline int launch_step(const char* fn, const StepParams& prm, int64_t blocks, zero_dtype_t grad_dtype,
-                       zero_dtype_t param_dtype, zero_stream_t stream) {
-    if (blocks == 0) return ok();
-    KernelFn k = pick_kernel(grad_dtype, param_dtype);
-    k<<<static_cast<unsigned int>(blocks), kThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(prm);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return fail(ZERO_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
-    return ok();
-}
 
 }  // namespace
 }  // namespace fused

@@ -29,7 +29,7 @@
 //    block by a fixed shuffle tree, and the last block (atomic ticket, no
 //    grid barrier, no waiting) folds the per-block partials in block order in
 //    double, so the result is deterministic.
-#include "fused_step.cuh"
+#include "step_launch.h"
 
 using zero::fail;
 

@@ -1,0 +1,275 @@
+// Host side of the fused step: argument validation, kernel choice, grid
+// sizing and launch.  Included by every translation unit that launches the
+// kernels of fused_step.cuh.
+#pragma once
+
+#include "fused_step.cuh"
+
+namespace zero {
+namespace fused {
+namespace {
+
+constexpr uint32_t kPipeStageTarget = 80u * 1024u;  // bytes of one pipeline stage, aimed for
+constexpr uint32_t kPipeMinTile = 1536;             // elements: 3/4 of 4 x consumer threads
+constexpr uint32_t kPipeSmemMax = 220u * 1024u;     // dynamic shared memory cap
+
+using KernelFn = void (*)(StepParams);
+
+inline KernelFn pick_kernel(zero_dtype_t g, zero_dtype_t pd) {
+    if (g == ZERO_F16 && pd == ZERO_F16) return fused_step_kernel<__half, __half>;
+    if (g == ZERO_F16 && pd == ZERO_BF16) return fused_step_kernel<__half, __nv_bfloat16>;
+    if (g == ZERO_BF16 && pd == ZERO_F16) return fused_step_kernel<__nv_bfloat16, __half>;
+    return fused_step_kernel<__nv_bfloat16, __nv_bfloat16>;
+}
+
+inline KernelFn pick_pipe_kernel(zero_dtype_t g, zero_dtype_t pd) {
+    if (g == ZERO_F16 && pd == ZERO_F16) return fused_step_pipe_kernel<__half, __half>;
+    if (g == ZERO_F16 && pd == ZERO_BF16) return fused_step_pipe_kernel<__half, __nv_bfloat16>;
+    if (g == ZERO_BF16 && pd == ZERO_F16) return fused_step_pipe_kernel<__nv_bfloat16, __half>;
+    return fused_step_pipe_kernel<__nv_bfloat16, __nv_bfloat16>;
+}
+
+// Pipeline tile for N replicas: about kPipeStageTarget bytes per stage, a
+// multiple of 256 elements.  0 (the register kernel runs) when a tile would
+// keep fewer than 3/4 of the consumer threads busy (4 elements each): with
+// the stage target that is N > 20, where the register kernel is faster.
+inline int pipe_tile(int world) {
+    const uint32_t per_elem = 2u * static_cast<uint32_t>(world) + 12u;
+    uint32_t t = kPipeStageTarget / per_elem / 256u * 256u;
+    if (t > 8192u) t = 8192u;
+    if (t < kPipeMinTile) return 0;
+    if (static_cast<uint64_t>(kPipeStages) * t * per_elem > kPipeSmemMax) return 0;
+    return static_cast<int>(t);
+}
+
+inline uint32_t pipe_smem_bytes(int world, int tile) {
+    return static_cast<uint32_t>(kPipeStages) * static_cast<uint32_t>(tile) * (2u * static_cast<uint32_t>(world) + 12u);
+}
+
+struct DeviceInfo {
+    int sms = 0;
+    int blocks_per_sm[4] = {0, 0, 0, 0};
+    bool pipe_ready[4] = {false, false, false, false};
+};
+
+std::mutex g_dev_mu;
+DeviceInfo g_dev[64];
+
+inline int device_info(DeviceInfo** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return fail(ZERO_ERR_CUDA, "cudaGetDevice failed");
+    DeviceInfo& d = g_dev[dev];
+    if (d.sms == 0) {
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return fail(ZERO_ERR_CUDA, "cannot query the SM count");
+    }
+    *out = &d;
+    return ZERO_OK;
+}
+
+inline int grid_limit(zero_dtype_t g, zero_dtype_t pd, int* out) {
+    const int which = static_cast<int>(g) * 2 + static_cast<int>(pd);
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo* d = nullptr;
+    if (int rc = device_info(&d)) return rc;
+    if (d->blocks_per_sm[which] == 0) {
+        int n = 0;
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, pick_kernel(g, pd), kThreads, 0);
+        if (e != cudaSuccess || n < 1) return fail(ZERO_ERR_CUDA, "occupancy query failed: %s", cudaGetErrorString(e));
+        d->blocks_per_sm[which] = n;
+    }
+    int lim = d->sms * d->blocks_per_sm[which];
+    *out = lim < kMaxBlocks ? lim : kMaxBlocks;
+    return ZERO_OK;
+}
+
+// SM count, and the pipeline kernel's shared-memory limit raised once per
+// device and dtype pair.
+inline int pipe_setup(zero_dtype_t g, zero_dtype_t pd, int* sms) {
+    const int which = static_cast<int>(g) * 2 + static_cast<int>(pd);
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo* d = nullptr;
+    if (int rc = device_info(&d)) return rc;
+    if (!d->pipe_ready[which]) {
+        cudaError_t e = cudaFuncSetAttribute(pick_pipe_kernel(g, pd), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kPipeSmemMax));
+        if (e != cudaSuccess) return fail(ZERO_ERR_CUDA, "cannot raise the shared-memory limit: %s", cudaGetErrorString(e));
+        d->pipe_ready[which] = true;
+    }
+    *sms = d->sms;
+    return ZERO_OK;
+}
+
+// Smallest h in [0, kVec) at which every array sits on a 16-byte boundary,
+// or -1 if their phases never coincide.
+inline int64_t common_phase(const StepParams& p) {
+    for (int64_t h = 0; h < kVec; ++h) {
+        bool good = true;
+        for (int k = 0; k < p.world && good; ++k)
+            good = ((reinterpret_cast<uintptr_t>(p.grads[k]) + 2 * h) % 16) == 0;
+        const void* f32s[] = {p.master_in, p.m_in, p.v_in, p.master_out, p.m_out, p.v_out};
+        for (const void* a : f32s) good = good && ((reinterpret_cast<uintptr_t>(a) + 4 * h) % 16) == 0;
+        good = good && ((reinterpret_cast<uintptr_t>(p.param_out) + 2 * h) % 16) == 0;
+        if (good) return h;
+    }
+    return -1;
+}
+
+
+// Validate the arguments of a fused-step call and build its kernel
+// parameters and grid size.  `workspace` is the scratch used for the
+// gradient norm (ticket + per-block partials).  On success *blocks_out is the
+// number of blocks to launch (0: nothing to do).
+inline int prepare_step(const char* fn, const void* const* grad_bufs, int32_t world, int64_t padded_numel,
+                        int32_t partition, zero_dtype_t grad_dtype, const float* master_in, const float* m_in,
+                        const float* v_in, float* master_out, float* m_out, float* v_out, void* param_out,
+                        zero_dtype_t param_dtype, const zero_adam_hparams_t* hp, float loss_scale,
+                        int32_t* overflow_flag, double* grad_sqnorm, void* workspace, StepParams* prm_out,
+                        int64_t* blocks_out) {
+    if (!grad_bufs || !hp || !overflow_flag) return fail(ZERO_ERR_ARG, "%s: NULL grad_bufs, hp or overflow_flag", fn);
+    if (world < 1 || world > ZERO_MAX_WORLD)
+        return fail(ZERO_ERR_ARG, "%s: world %d outside 1..%d", fn, world, ZERO_MAX_WORLD);
+    if (padded_numel < 0 || padded_numel % world != 0)
+        return fail(ZERO_ERR_ARG, "%s: padded_numel %lld is not a non-negative multiple of world %d", fn,
+                    (long long)padded_numel, world);
+    if (partition != ZERO_ALL_PARTITIONS && (partition < 0 || partition >= world))
+        return fail(ZERO_ERR_RANGE, "%s: partition %d outside 0..%d", fn, partition, world - 1);
+    if ((grad_dtype != ZERO_F16 && grad_dtype != ZERO_BF16) || (param_dtype != ZERO_F16 && param_dtype != ZERO_BF16))
+        return fail(ZERO_ERR_DTYPE, "%s: gradients and parameters must be ZERO_F16 or ZERO_BF16", fn);
+    if (!(hp->step >= 1)) return fail(ZERO_ERR_ARG, "%s: hp->step must be >= 1", fn);
+    if (!std::isfinite(hp->lr) || !std::isfinite(hp->eps) || !std::isfinite(hp->weight_decay) ||
+        !(hp->beta1 >= 0.0f && hp->beta1 < 1.0f) || !(hp->beta2 >= 0.0f && hp->beta2 < 1.0f) ||
+        !(hp->grad_divisor >= 0.0f) || !std::isfinite(hp->grad_divisor))
+        return fail(ZERO_ERR_ARG, "%s: hyper-parameters out of range", fn);
+    if (!(loss_scale > 0.0f) || !std::isfinite(loss_scale))
+        return fail(ZERO_ERR_ARG, "%s: loss_scale must be positive and finite", fn);
+    if (grad_sqnorm && !workspace) return fail(ZERO_ERR_ARG, "%s: grad_sqnorm needs a workspace", fn);
+    if (!aligned(overflow_flag, 4) || (grad_sqnorm && !aligned(grad_sqnorm, 8)) ||
+        (workspace && !aligned(workspace, 16)))
+        return fail(ZERO_ERR_ALIGN, "%s: flag, norm or workspace misaligned", fn);
+
+    const int64_t P = padded_numel / world;
+    const int64_t begin = partition == ZERO_ALL_PARTITIONS ? 0 : static_cast<int64_t>(partition) * P;
+    const int64_t count = partition == ZERO_ALL_PARTITIONS ? padded_numel : P;
+    if (count == 0) {
+        *blocks_out = 0;
+        return ZERO_OK;
+    }
+
+    const float* f_in[] = {master_in, m_in, v_in};
+    float* f_out[] = {master_out, m_out, v_out};
+    for (int i = 0; i < 3; ++i) {
+        if (!f_in[i] || !f_out[i]) return fail(ZERO_ERR_ARG, "%s: NULL state pointer", fn);
+        if (!aligned(f_in[i], 4) || !aligned(f_out[i], 4)) return fail(ZERO_ERR_ALIGN, "%s: fp32 state not 4-byte aligned", fn);
+    }
+    if (!param_out) return fail(ZERO_ERR_ARG, "%s: NULL param_out", fn);
+    if (!aligned(param_out, 2)) return fail(ZERO_ERR_ALIGN, "%s: param_out not 2-byte aligned", fn);
+    for (int k = 0; k < world; ++k) {
+        if (!grad_bufs[k]) return fail(ZERO_ERR_ARG, "%s: grad_bufs[%d] is NULL", fn, k);
+        if (!aligned(grad_bufs[k], 2)) return fail(ZERO_ERR_ALIGN, "%s: grad_bufs[%d] not 2-byte aligned", fn, k);
+    }
+    // outputs: each output either is its own input (in place) or overlaps
+    // nothing else; outputs never overlap each other or a gradient buffer
+    const int64_t fb = count * 4, pb = count * 2, gb = padded_numel * 2;
+    const void* outs[] = {master_out, m_out, v_out, param_out};
+    const int64_t out_bytes[] = {fb, fb, fb, pb};
+    for (int i = 0; i < 4; ++i) {
+        for (int j = i + 1; j < 4; ++j)
+            if (overlaps(outs[i], out_bytes[i], outs[j], out_bytes[j]))
+                return fail(ZERO_ERR_ARG, "%s: output arrays overlap", fn);
+        for (int j = 0; j < 3; ++j)
+            if (!(i == j && outs[i] == f_in[j]) && overlaps(outs[i], out_bytes[i], f_in[j], fb))
+                return fail(ZERO_ERR_ARG, "%s: an output overlaps an input it does not replace", fn);
+        for (int k = 0; k < world; ++k)
+            if (overlaps(outs[i], out_bytes[i], grad_bufs[k], gb))
+                return fail(ZERO_ERR_ARG, "%s: an output overlaps grad_bufs[%d]", fn, k);
+    }
+
+    StepParams prm{};
+    prm.world = world;
+    for (int k = 0; k < world; ++k) prm.grads[k] = static_cast<const uint16_t*>(grad_bufs[k]) + begin;
+    prm.count = count;
+    prm.master_in = master_in;
+    prm.m_in = m_in;
+    prm.v_in = v_in;
+    prm.master_out = master_out;
+    prm.m_out = m_out;
+    prm.v_out = v_out;
+    prm.param_out = param_out;
+    prm.overflow = overflow_flag;
+    prm.sqnorm = grad_sqnorm;
+    if (grad_sqnorm) {
+        prm.ticket = static_cast<unsigned int*>(workspace);
+        prm.partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + kWsPartialsOffset);
+    }
+    // constants: double, rounded once to float
+    const double divisor = hp->grad_divisor > 0.0f ? static_cast<double>(hp->grad_divisor) : static_cast<double>(world);
+    const double t = static_cast<double>(hp->step);
+    prm.c.lr = hp->lr;
+    prm.c.b1 = hp->beta1;
+    prm.c.b2 = hp->beta2;
+    prm.c.eps = hp->eps;
+    prm.c.inv = static_cast<float>(1.0 / (divisor * static_cast<double>(loss_scale)));
+    prm.c.omb1 = static_cast<float>(1.0 - static_cast<double>(hp->beta1));
+    prm.c.omb2 = static_cast<float>(1.0 - static_cast<double>(hp->beta2));
+    prm.c.rbc1 = static_cast<float>(1.0 / (1.0 - std::pow(static_cast<double>(hp->beta1), t)));
+    prm.c.rsbc2 = static_cast<float>(1.0 / std::sqrt(1.0 - std::pow(static_cast<double>(hp->beta2), t)));
+    prm.c.decay = static_cast<float>(1.0 - static_cast<double>(hp->lr) * static_cast<double>(hp->weight_decay));
+
+    const int64_t h = common_phase(prm);
+    if (h < 0 || h >= count) {
+        prm.head = count;
+        prm.nvec = 0;
+    } else {
+        prm.head = h;
+        prm.nvec = (count - h) / kVec;
+    }
+    prm.tile = 0;
+
+    // The pipeline kernel takes calls whose arrays share a 16-byte phase and
+    // that give every SM at least two tiles; the rest use the register kernel.
+    int64_t blocks = 0;
+    const int tile = h >= 0 ? pipe_tile(world) : 0;
+    if (tile > 0) {
+        int sms = 0;
+        if (int rc = pipe_setup(grad_dtype, param_dtype, &sms)) return rc;
+        const int64_t ntiles = (count - h) / tile;
+        if (ntiles >= 2 * static_cast<int64_t>(sms)) {
+            prm.tile = tile;
+            prm.nvec = ntiles * tile / kVec;
+            blocks = sms;
+        }
+    }
+    if (prm.tile == 0) {
+        int limit = 0;
+        if (int rc = grid_limit(grad_dtype, param_dtype, &limit)) return rc;
+        const int64_t work = prm.nvec > 0 ? prm.nvec : count;
+        blocks = (work + kThreads - 1) / kThreads;
+        if (blocks > limit) blocks = limit;
+        if (blocks < 1) blocks = 1;
+    }
+    *prm_out = prm;
+    *blocks_out = blocks;
+    return ZERO_OK;
+}
+
+// Enqueue the fused kernel prepared by prepare_step.
+inline int launch_step(const char* fn, const StepParams& prm, int64_t blocks, zero_dtype_t grad_dtype,
+                       zero_dtype_t param_dtype, zero_stream_t stream) {
+    if (blocks == 0) return ok();
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (prm.tile > 0) {
+        pick_pipe_kernel(grad_dtype, param_dtype)<<<static_cast<unsigned int>(blocks), kPipeThreads,
+                                                     pipe_smem_bytes(prm.world, prm.tile), s>>>(prm);
+    } else {
+        pick_kernel(grad_dtype, param_dtype)<<<static_cast<unsigned int>(blocks), kThreads, 0, s>>>(prm);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(ZERO_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
+    return ok();
+}
+
+}  // namespace
+}  // namespace fused
+}  // namespace zero

@@ -121,7 +121,12 @@ class ZeroAdam:
         s = torch.cuda.current_stream() if stream is None else stream
         self.flag_host.copy_(self.flag, non_blocking=True)
         s.synchronize()
-        ovf = int(self.flag_host.item())
+        flag = int(self.flag_host.item())
+        ovf = int(flag != 0)
+        if flag & 2:
+            # the kernel abandoned its copy pipeline: the banks were not
+            # committed, but the device needs attention
+            raise RuntimeError("fused step kernel timed out waiting on its copy pipeline; step not committed")
         if not ovf:
             self.cur ^= 1
             self.t += 1
