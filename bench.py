@@ -214,8 +214,10 @@ def fill_workload(opt, w, seed_base: int):
         opt.params_bank[b][0].copy_(opt.master[b][0])
         for bank in (opt.m, opt.v):
             bank[b][0].zero_()
-        opt.master[b][1].copy_(opt.master[b][0])
-        opt.params_bank[b][1].copy_(opt.params_bank[b][0])
+        for extra in opt.master[b][1:]:
+            extra.copy_(opt.master[b][0])
+        for extra in opt.params_bank[b][1:]:
+            extra.copy_(opt.params_bank[b][0])
     torch.cuda.synchronize()
 
 
@@ -249,7 +251,7 @@ def run_gpu(args):
     gdt = torch.bfloat16 if args.grad_dtype == "bf16" else torch.float16
     opt = Z.ZeroAdam(w.numels, w.world, w.bucket_elems, lr=w.adam.lr, betas=(w.adam.beta1, w.adam.beta2),
                      eps=w.adam.eps, weight_decay=w.adam.weight_decay, loss_scale=w.loss_scale,
-                     grad_dtype=gdt, param_dtype=gdt)
+                     grad_dtype=gdt, param_dtype=gdt, mode=args.mode, max_grad_norm=args.max_grad_norm)
     L = opt.layout
     psi_p = sum(L.bucket_padded)
     fill_workload(opt, w, w.seed + 100 * rank)
@@ -321,6 +323,9 @@ def run_gpu(args):
                 "config": {"workload": w.name, "psi": sum(w.numels), "psi_padded": psi_p, "world": w.world,
                            "buckets": L.n_buckets, "bucket_elems": w.bucket_elems, "grad_dtype": args.grad_dtype,
                            "param_dtype": args.grad_dtype, "optimizer": "AdamW wd=0.01", "stage": 2,
+                           "mode": args.mode, "max_grad_norm": args.max_grad_norm,
+                           "passes": ("statistics pass (2N B/elem) + gated update" if opt.two_pass
+                                      else "single fused pass"),
                            "parallelism": f"{world_gpus} GPU(s) x {w.world} simulated replicas",
                            "l2": (f"inputs larger than L2: {psi_p * bpe / 1e9:.1f} GB of HBM traffic per step"
                                   if psi_p * bpe > 4 * 126e6 else "L2-influenced (footprint < 4x L2)")},
@@ -330,7 +335,7 @@ def run_gpu(args):
                              "kernel": "fused_step (shared-memory pipeline kernel for aligned calls of >= 2 tiles per SM)",
                              "bytes_per_elem": bpe,
                              "elems_per_launch": avg_elems, "launches_timed": len(launch_ms)},
-                "gpu_launches": args.steps * L.n_buckets,
+                "gpu_launches": args.steps * L.n_buckets * (2 if opt.two_pass else 1),
                 "applied_steps": applied,
                 "clocks": clock,
                 "e2e": e2e,
@@ -452,6 +457,9 @@ def main(argv=None):
     ap.add_argument("--world", type=int, default=8, help="simulated replicas of the flat workload")
     ap.add_argument("--grad-dtype", choices=["f16", "bf16"], default="f16")
     ap.add_argument("--sweep", action="store_true", help="flat bandwidth sweep, one JSON line per point")
+    ap.add_argument("--mode", choices=["banks", "inplace"], default="banks",
+                    help="banks: two state banks, one pass; inplace: one bank, statistics pass + gated update")
+    ap.add_argument("--max-grad-norm", type=float, default=None, help="clip gradients to this global norm")
     ap.add_argument("--sweep-dtype-only", action="store_true", help="sweep only --grad-dtype")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":

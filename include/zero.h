@@ -207,8 +207,9 @@ size_t zero_step_workspace_bytes(void);
  *              then OR into one flag for the whole step.
  * grad_sqnorm  device double or NULL; when not NULL, sum over the call's
  *              elements of g*g is ADDED to it (clear it at the start of a
- *              step).  Deterministic: per-block fp32 partial sums folded in a
- *              fixed order in double.
+ *              step).  Each g*g is exact in double; per-thread and per-block
+ *              sums in double, folded over blocks in a fixed order:
+ *              deterministic.
  * workspace    device, zero_step_workspace_bytes() bytes, zero-filled once
  *              before its first use; required when grad_sqnorm is not NULL
  *              (NULL allowed otherwise).  Each call leaves it zero-filled
@@ -229,6 +230,68 @@ int zero_reduce_scatter_adam_step(
     zero_stream_t stream);
 
 /*
+ * zero_grad_stats - the reduce-scatter's sums without the update: overflow
+ * flag and squared norm of one bucket's reduced gradients.
+ *
+ * Source: the reduce-scatter of ZeRO explainer, "Stage 2 - Gradient
+ * Partitioning (P_os+g)", taken alone.  For each processed element (same
+ * `partition` convention as zero_reduce_scatter_adam_step) it forms the
+ * rank-order fp32 sum s of the N replicas and g = s * fp32(1/(divisor *
+ * loss_scale)); it sets bit 0 of *overflow_flag when any s is inf or NaN
+ * (never clears it) and, when grad_sqnorm is not NULL, adds the sum of g*g
+ * (each g*g exact in double, summed in double, deterministic) to
+ * *grad_sqnorm.  It reads 2N bytes per element and writes no state.
+ *
+ * Purpose: decide skip and clipping for a whole step before any state is
+ * written.  Followed by zero_reduce_scatter_adam_step_gated, the update can
+ * run in place (one bank of states: the pages' 12 Psi / N bytes per rank)
+ * with an exact skip, for 4N + 26 bytes per element in total.
+ *
+ * grad_bufs, world, padded_numel, partition, grad_dtype: as for
+ *              zero_reduce_scatter_adam_step
+ * loss_scale   > 0, finite;  grad_divisor >= 0 (0 = world)
+ * overflow_flag device int32, OR-ed into
+ * grad_sqnorm  device double or NULL (added to; needs `workspace`)
+ * workspace    as for zero_reduce_scatter_adam_step
+ * Errors: ZERO_ERR_ARG, ZERO_ERR_RANGE, ZERO_ERR_DTYPE, ZERO_ERR_ALIGN,
+ * ZERO_ERR_CUDA.
+ */
+int zero_grad_stats(const void* const* grad_bufs, int32_t world, int64_t padded_numel, int32_t partition,
+                    zero_dtype_t grad_dtype, float loss_scale, float grad_divisor,
+                    int32_t* overflow_flag, double* grad_sqnorm, void* workspace, zero_stream_t stream);
+
+/*
+ * zero_reduce_scatter_adam_step_gated - zero_reduce_scatter_adam_step with
+ * a device-side gate and global-norm gradient clipping.
+ *
+ * Same arguments and results as zero_reduce_scatter_adam_step, plus:
+ * gate         device int32 or NULL.  When not NULL and non-zero when the
+ *              kernel starts, the call writes nothing at all (no state, no
+ *              parameters, no flag, no norm).  Pass the flag that
+ *              zero_grad_stats filled for the whole step: an overflowing
+ *              step then leaves in-place states bit-identical.  It must not
+ *              be this call's own overflow_flag, and nothing may write it
+ *              while the kernel runs.
+ * clip_sqnorm  device double or NULL.  When not NULL, the unscaled gradient
+ *              is multiplied by clip = min(1, max_norm / (sqrt(*clip_sqnorm)
+ *              + 1e-6)) (computed in double, rounded once to float):
+ *              g = (s * inv) * clip.  Pass the step's total squared norm from
+ *              zero_grad_stats.  Global-norm clipping is not on the pages.
+ * max_norm     > 0 and finite when clip_sqnorm is not NULL
+ * Errors: those of zero_reduce_scatter_adam_step.
+ */
+int zero_reduce_scatter_adam_step_gated(
+    const void* const* grad_bufs, int32_t world, int64_t padded_numel, int32_t partition,
+    zero_dtype_t grad_dtype,
+    const float* master_in, const float* m_in, const float* v_in,
+    float* master_out, float* m_out, float* v_out,
+    void* param_out, zero_dtype_t param_dtype,
+    const zero_adam_hparams_t* hp, float loss_scale,
+    int32_t* overflow_flag, double* grad_sqnorm, void* workspace,
+    const int32_t* gate, const double* clip_sqnorm, float max_norm,
+    zero_stream_t stream);
+
+/*
  * zero_reduce_scatter_adam_step_noalloc - zero_reduce_scatter_adam_step for
  * callers that cannot allocate device memory.
  *
@@ -239,7 +302,7 @@ int zero_reduce_scatter_adam_step(
  * that must not take cudaMalloc's implicit device synchronization, or a C
  * caller with no device allocator.  This entry point takes the same
  * arguments minus `workspace` and keeps that scratch in a fixed array in the
- * library's device image instead (16,640 bytes per GPU that loads the
+ * library's device image instead (33,024 bytes per GPU that loads the
  * library, held until exit); it calls no cudaMalloc, cudaFree or other
  * allocating routine.  Inputs and outputs are still the caller's.
  *

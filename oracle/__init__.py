@@ -94,6 +94,10 @@ def lib():
         L.orc_adam_constants.restype = None
         L.orc_adam_update.argtypes = [vp, i64, vp, vp, vp, vp, vp, ctypes.c_int]
         L.orc_adam_update.restype = None
+        L.orc_clip_coefficient.argtypes = [f64, f64]
+        L.orc_clip_coefficient.restype = f32
+        L.orc_adam_update_clipped.argtypes = [vp, i64, vp, f32, vp, vp, vp, vp, ctypes.c_int]
+        L.orc_adam_update_clipped.restype = None
         L.orc_allgather.argtypes = [vp, i32, i64, i64, vp]
         L.orc_allgather.restype = None
         L.orc_threads.restype = i32
@@ -285,6 +289,25 @@ def adam_update(s, consts, master, m, v, p16, pdtype: str = F16) -> None:
     s = np.ascontiguousarray(s, dtype=np.float32)
     lib().orc_adam_update(_ptr(s), s.size, _ptr(consts), _ptr(master), _ptr(m), _ptr(v),
                           _ptr(p16), _DT[pdtype])
+
+
+def clip_coefficient(total_sqnorm: float, max_norm: float) -> np.float32:
+    """Global-norm clipping factor min(1, max_norm / (sqrt(total) + 1e-6)).
+
+    Not on the pages (the usual rule of clipping by the global norm); the
+    coefficient is computed in double and rounded once to float.
+    """
+    return np.float32(lib().orc_clip_coefficient(float(total_sqnorm), float(max_norm)))
+
+
+def adam_update_clipped(s, consts, clip, master, m, v, p16, pdtype: str = F16) -> None:
+    """adam_update with g = (s * inv) * clip."""
+    for a in (master, m, v):
+        assert a.dtype == np.float32 and a.flags["C_CONTIGUOUS"] and a.size == s.size
+    assert p16.dtype == np.uint16 and p16.size == s.size and p16.flags["C_CONTIGUOUS"]
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    lib().orc_adam_update_clipped(_ptr(s), s.size, _ptr(consts), float(clip), _ptr(master), _ptr(m), _ptr(v),
+                                  _ptr(p16), _DT[pdtype])
 
 
 def allgather(shards, offset: int, part: int) -> np.ndarray:

@@ -257,6 +257,38 @@ void orc_adam_update(const float* s, int64_t count, const float* c,
     }
 }
 
+/* Global-norm gradient clipping (not on the pages; the usual rule): the
+ * unscaled gradient is multiplied by
+ *     clip = min(1, max_norm / (sqrt(total_sqnorm) + 1e-6)),
+ * computed in double and rounded once to float. */
+float orc_clip_coefficient(double total_sqnorm, double max_norm)
+{
+    double coef = max_norm / (sqrt(total_sqnorm) + 1e-6);
+    return coef < 1.0 ? (float)coef : 1.0f;
+}
+
+/* orc_adam_update with clipped gradients: g = (s * inv) * clip, the rest of
+ * the update unchanged.  clip == 1 reproduces orc_adam_update exactly. */
+void orc_adam_update_clipped(const float* s, int64_t count, const float* c, float clip,
+                             float* master, float* m, float* v, uint16_t* p16, int pdtype)
+{
+    const float lr = c[0], b1 = c[1], b2 = c[2], eps = c[3], inv = c[4];
+    const float omb1 = c[5], omb2 = c[6], rbc1 = c[7], rsbc2 = c[8], decay = c[9];
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < count; ++j) {
+        float g = (s[j] * inv) * clip;
+        float mn = fmaf(b1, m[j], omb1 * g);
+        float vn = fmaf(b2, v[j], (omb2 * g) * g);
+        float den = fmaf(sqrtf(vn), rsbc2, eps);
+        float u = (mn * rbc1) / den;
+        float pn = fmaf(-lr, u, master[j] * decay);
+        m[j] = mn;
+        v[j] = vn;
+        master[j] = pn;
+        p16[j] = from_f32(pn, pdtype);
+    }
+}
+
 /* ------------------------------------------------------------------------ */
 /* All-gather                                                               */
 /* ------------------------------------------------------------------------ */

@@ -43,7 +43,7 @@ def test_noalloc_entry_validates_like_the_regular_one():
     ok = list(args)
     ok[2] = 0
     assert Z.lib.zero_reduce_scatter_adam_step_noalloc(*ok) == 0    # nothing to do
-    assert Z.lib.zero_step_static_scratch_bytes() == 256 + 4 * 4096
+    assert Z.lib.zero_step_static_scratch_bytes() == 256 + 8 * 4096
 
 
 def _inputs(world, n, seed):

@@ -76,6 +76,13 @@ def _load():
     L.zero_reduce_scatter_adam_step_noalloc.restype = ctypes.c_int
     L.zero_step_static_scratch_bytes.argtypes = []
     L.zero_step_static_scratch_bytes.restype = ctypes.c_size_t
+    L.zero_grad_stats.argtypes = [ctypes.POINTER(vp), i32, i64, i32, ctypes.c_int, f32, f32, vp, vp, vp, vp]
+    L.zero_grad_stats.restype = ctypes.c_int
+    L.zero_reduce_scatter_adam_step_gated.argtypes = [
+        ctypes.POINTER(vp), i32, i64, i32, ctypes.c_int,
+        vp, vp, vp, vp, vp, vp, vp, ctypes.c_int,
+        ctypes.POINTER(AdamHParams), f32, vp, vp, vp, vp, vp, f32, vp]
+    L.zero_reduce_scatter_adam_step_gated.restype = ctypes.c_int
     L.zero_allgather_params.argtypes = [ctypes.POINTER(vp), i32, i64, i64, ctypes.c_int, vp, vp]
     L.zero_allgather_params.restype = ctypes.c_int
     L.zero_loss_scale_update.argtypes = [ctypes.POINTER(f32), ctypes.POINTER(i32), i32, i32, f32]
@@ -224,6 +231,29 @@ def zero_reduce_scatter_adam_step_noalloc(grad_bufs, padded_numel: int, partitio
         _ptr(master_in), _ptr(m_in), _ptr(v_in), _ptr(master_out), _ptr(m_out), _ptr(v_out),
         _ptr(param_out), _dtype_code(param_out), ctypes.byref(hp), float(loss_scale),
         _ptr(overflow_flag), _ptr(grad_sqnorm), _stream(stream)))
+
+
+def zero_grad_stats(grad_bufs, padded_numel: int, partition: int, loss_scale: float, overflow_flag,
+                    grad_sqnorm=None, workspace=None, grad_divisor: float = 0.0, stream=None) -> None:
+    """Overflow flag and squared norm of one bucket's reduced gradients (no update)."""
+    _check(lib.zero_grad_stats(_ptrs(grad_bufs), len(grad_bufs), padded_numel, partition,
+                               _dtype_code(grad_bufs[0]), float(loss_scale), float(grad_divisor),
+                               _ptr(overflow_flag), _ptr(grad_sqnorm), _ptr(workspace), _stream(stream)))
+
+
+def zero_reduce_scatter_adam_step_gated(grad_bufs, padded_numel: int, partition: int,
+                                        master_in, m_in, v_in, master_out, m_out, v_out, param_out,
+                                        hp: AdamHParams, loss_scale: float, overflow_flag,
+                                        grad_sqnorm=None, workspace=None, gate=None, clip_sqnorm=None,
+                                        max_norm: float = 0.0, stream=None) -> None:
+    """The fused step, skipped entirely when *gate != 0, with optional clipping."""
+    world = len(grad_bufs)
+    _check(lib.zero_reduce_scatter_adam_step_gated(
+        _ptrs(grad_bufs), world, padded_numel, partition, _dtype_code(grad_bufs[0]),
+        _ptr(master_in), _ptr(m_in), _ptr(v_in), _ptr(master_out), _ptr(m_out), _ptr(v_out),
+        _ptr(param_out), _dtype_code(param_out), ctypes.byref(hp), float(loss_scale),
+        _ptr(overflow_flag), _ptr(grad_sqnorm), _ptr(workspace), _ptr(gate), _ptr(clip_sqnorm),
+        float(max_norm), _stream(stream)))
 
 
 def zero_allgather_params(shards, shard_offset: int, part_numel: int, dst, stream=None) -> None:

@@ -23,12 +23,13 @@ constexpr int kVec = 8;          // elements per vector
 constexpr int kBatch = 8;        // replicas whose loads are issued together
 constexpr int kMaxBlocks = 8192; // per-block partials held by the workspace
 
-// Workspace: [ticket:uint32][pad to 256 B][partials: float x kMaxBlocks]
+// Workspace: [ticket:uint32][pad to 256 B][partials: double x kMaxBlocks]
 constexpr size_t kWsPartialsOffset = 256;
-constexpr size_t kWorkspaceBytes = kWsPartialsOffset + sizeof(float) * kMaxBlocks;
+constexpr size_t kWorkspaceBytes = kWsPartialsOffset + sizeof(double) * kMaxBlocks;
 
 struct Consts {
     float lr, b1, b2, eps, inv, omb1, omb2, rbc1, rsbc2, decay;
+    float clip;  // gradient multiplier of global-norm clipping; 1 when not clipping
 };
 
 struct StepParams {
@@ -48,8 +49,11 @@ struct StepParams {
     Consts c;
     int32_t* overflow;
     double* sqnorm;
-    float* partials;
+    double* partials;
     unsigned int* ticket;
+    const int32_t* gate;        // device; when not NULL and non-zero the kernel writes nothing
+    const double* clip_sqnorm;  // device; when not NULL, clip gradients to norm max_norm
+    double max_norm;
 };
 
 // ---------------------------------------------------------------- loads/stores
@@ -141,7 +145,7 @@ __device__ __forceinline__ void add8(const uint4& r, float* s) {
 // weight decay; every operation explicitly rounded so that no contraction
 // changes the result.  Returns the unscaled gradient g for the norm.
 __device__ __forceinline__ float adam(float s, float& p, float& m, float& v, const Consts& c) {
-    const float g = __fmul_rn(s, c.inv);
+    const float g = __fmul_rn(__fmul_rn(s, c.inv), c.clip);
     const float mn = __fmaf_rn(c.b1, m, __fmul_rn(c.omb1, g));
     const float vn = __fmaf_rn(c.b2, v, __fmul_rn(__fmul_rn(c.omb2, g), g));
     const float den = __fmaf_rn(__fsqrt_rn(vn), c.rsbc2, c.eps);
@@ -164,11 +168,25 @@ __device__ __forceinline__ double warp_sum_d(double x) {
     return x;
 }
 
+// Gate and clip, read once per thread from device memory: returns false
+// (write nothing) when the gate is set; otherwise sets c.clip from the
+// global squared norm, min(1, max_norm / (sqrt(sqnorm) + 1e-6)) computed in
+// double and rounded once to float.  Every thread of the grid takes the
+// same branch.
+__device__ __forceinline__ bool step_prologue(const StepParams& p, Consts& c) {
+    if (p.gate != nullptr && *reinterpret_cast<const volatile int32_t*>(p.gate) != 0) return false;
+    if (p.clip_sqnorm != nullptr) {
+        const double coef = p.max_norm / (sqrt(*p.clip_sqnorm) + 1e-6);
+        c.clip = coef < 1.0 ? static_cast<float>(coef) : 1.0f;
+    }
+    return true;
+}
+
 // Elements outside the vector (or tile) region: [0, head) and
 // [head + nvec*kVec, count), one element per thread and iteration.
 template <typename GT, typename PT>
 __device__ __forceinline__ void scalar_elements(const StepParams& p, const Consts& c, int64_t tid, int64_t nthreads,
-                                                bool& bad, float& sq) {
+                                                bool& bad, double& sq) {
     const int world = p.world;
     const int64_t vec_end = p.head + p.nvec * kVec;
     const int64_t nscalar = p.head + (p.count - vec_end);
@@ -180,7 +198,7 @@ __device__ __forceinline__ void scalar_elements(const StepParams& p, const Const
         float pw = p.master_in[e], mw = p.m_in[e], vw = p.v_in[e];
         bad |= !isfinite(s);
         const float g = adam(s, pw, mw, vw, c);
-        sq = __fmaf_rn(g, g, sq);
+        if (p.sqnorm) sq = fma(static_cast<double>(g), static_cast<double>(g), sq);
         p.master_out[e] = pw;
         p.m_out[e] = mw;
         p.v_out[e] = vw;
@@ -191,19 +209,19 @@ __device__ __forceinline__ void scalar_elements(const StepParams& p, const Const
 // Overflow vote and the optional deterministic norm fold.  Every thread of
 // the block must call it (it synchronizes the block).
 template <int NT>
-__device__ __forceinline__ void finish_block(const StepParams& p, bool bad, float sq) {
+__device__ __forceinline__ void finish_block(const StepParams& p, bool bad, double sq) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     // one atomic per warp that saw a non-finite sum
     if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.overflow, 1);
     if (p.sqnorm == nullptr) return;
-    __shared__ float wsum[NT / 32];
+    __shared__ double wsum[NT / 32];
     __shared__ bool last;
-    sq = warp_sum(sq);
+    sq = warp_sum_d(sq);
     if (lane == 0) wsum[warp] = sq;
     __syncthreads();
     if (warp == 0) {
-        float x = lane < NT / 32 ? wsum[lane] : 0.0f;
-        x = warp_sum(x);
+        double x = lane < NT / 32 ? wsum[lane] : 0.0;
+        x = warp_sum_d(x);
         if (lane == 0) {
             p.partials[blockIdx.x] = x;
             __threadfence();
@@ -215,7 +233,7 @@ __device__ __forceinline__ void finish_block(const StepParams& p, bool bad, floa
     if (last && warp == 0) {
         __threadfence();
         double acc = 0.0;
-        for (unsigned int b = lane; b < gridDim.x; b += 32) acc += static_cast<double>(__ldcg(p.partials + b));
+        for (unsigned int b = lane; b < gridDim.x; b += 32) acc += __ldcg(p.partials + b);
         acc = warp_sum_d(acc);
         if (lane == 0) {
             *p.sqnorm += acc;
@@ -232,9 +250,10 @@ __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_const
     const int64_t tid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
     const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
     const int world = p.world;
-    const Consts c = p.c;
+    Consts c = p.c;
+    if (!step_prologue(p, c)) return;
     bool bad = false;
-    float sq = 0.0f;
+    double sq = 0.0;
 
     // ---- vector path: kVec elements per iteration, 16-byte accesses
     for (int64_t vi = tid; vi < p.nvec; vi += nthreads) {
@@ -272,7 +291,7 @@ __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_const
         for (int e = 0; e < kVec; ++e) {
             bad |= !isfinite(s[e]);
             const float g = adam(s[e], pw[e], mw[e], vw[e], c);
-            sq = __fmaf_rn(g, g, sq);
+            if (p.sqnorm) sq = fma(static_cast<double>(g), static_cast<double>(g), sq);
         }
         st_state16(p.master_out + e0, pw[0], pw[1], pw[2], pw[3]);
         st_state16(p.master_out + e0 + 4, pw[4], pw[5], pw[6], pw[7]);
@@ -289,6 +308,67 @@ __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_const
     }
 
     scalar_elements<GT, PT>(p, c, tid, nthreads, bad, sq);
+    finish_block<kThreads>(p, bad, sq);
+}
+
+// Statistics pre-pass: the rank-order fp32 sum of the N replicas, the
+// overflow test and, when p.sqnorm is set, the squared norm of the unscaled
+// gradient g = s * inv, without reading or writing any optimizer state.
+// 2N bytes per element.  Lets a caller decide skip and clipping for a whole
+// step before any state is written (in-place update with an exact skip).
+template <typename GT>
+__global__ void __launch_bounds__(kThreads) grad_stats_kernel(const __grid_constant__ StepParams p) {
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
+    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
+    const int world = p.world;
+    const float inv = p.c.inv;
+    const bool want_sq = p.sqnorm != nullptr;
+    bool bad = false;
+    double sq = 0.0;
+    for (int64_t vi = tid; vi < p.nvec; vi += nthreads) {
+        const int64_t e0 = p.head + vi * kVec;
+        float s[kVec];
+        {
+            uint4 r[kBatch];
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b)
+                if (b < world) r[b] = ld_grad16(static_cast<const uint16_t*>(p.grads[b]) + e0);
+            cvt8<GT>(r[0], s);
+#pragma unroll
+            for (int b = 1; b < kBatch; ++b)
+                if (b < world) add8<GT>(r[b], s);
+        }
+        for (int k0 = kBatch; k0 < world; k0 += kBatch) {
+            uint4 r[kBatch];
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b)
+                if (k0 + b < world) r[b] = ld_grad16(static_cast<const uint16_t*>(p.grads[k0 + b]) + e0);
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b)
+                if (k0 + b < world) add8<GT>(r[b], s);
+        }
+#pragma unroll
+        for (int e = 0; e < kVec; ++e) {
+            bad |= !isfinite(s[e]);
+            if (want_sq) {
+                const float g = __fmul_rn(s[e], inv);
+                sq = fma(static_cast<double>(g), static_cast<double>(g), sq);
+            }
+        }
+    }
+    const int64_t vec_end = p.head + p.nvec * kVec;
+    const int64_t nscalar = p.head + (p.count - vec_end);
+    for (int64_t q = tid; q < nscalar; q += nthreads) {
+        const int64_t e = q < p.head ? q : vec_end + (q - p.head);
+        float s = Fmt<GT>::one(static_cast<const uint16_t*>(p.grads[0])[e]);
+        for (int k = 1; k < world; ++k)
+            s = __fadd_rn(s, Fmt<GT>::one(static_cast<const uint16_t*>(p.grads[k])[e]));
+        bad |= !isfinite(s);
+        if (want_sq) {
+            const float g = __fmul_rn(s, inv);
+            sq = fma(static_cast<double>(g), static_cast<double>(g), sq);
+        }
+    }
     finish_block<kThreads>(p, bad, sq);
 }
 
@@ -377,6 +457,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1) fused_step_pipe_kernel(const 
     const uint32_t stage = static_cast<uint32_t>(world) * gbytes + 3u * sbytes;
     const int64_t ntiles = p.nvec * kVec / T;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    Consts c = p.c;
+    if (!step_prologue(p, c)) return;   // uniform over the grid: before any barrier is set up
     if (threadIdx.x == 0) {
         for (int s = 0; s < kPipeStages; ++s) {
             mbar_init(&full[s], 1);
@@ -386,9 +468,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1) fused_step_pipe_kernel(const 
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
-    const Consts c = p.c;
     bool bad = false;
-    float sq = 0.0f;
+    double sq = 0.0;
 
     if (warp == kPipeConsumerWarps) {
         // ---- producer warp: lane 0 arms the stage, all lanes issue copies
@@ -473,15 +554,16 @@ __global__ void __launch_bounds__(kPipeThreads, 1) fused_step_pipe_kernel(const 
                 float4 mw = *reinterpret_cast<const float4*>(sm_m + j);
                 float4 vw = *reinterpret_cast<const float4*>(sm_v + j);
                 bad |= !isfinite(sacc[0]) | !isfinite(sacc[1]) | !isfinite(sacc[2]) | !isfinite(sacc[3]);
-                float g;
-                g = adam(sacc[0], pw.x, mw.x, vw.x, c);
-                sq = __fmaf_rn(g, g, sq);
-                g = adam(sacc[1], pw.y, mw.y, vw.y, c);
-                sq = __fmaf_rn(g, g, sq);
-                g = adam(sacc[2], pw.z, mw.z, vw.z, c);
-                sq = __fmaf_rn(g, g, sq);
-                g = adam(sacc[3], pw.w, mw.w, vw.w, c);
-                sq = __fmaf_rn(g, g, sq);
+                const float g0 = adam(sacc[0], pw.x, mw.x, vw.x, c);
+                const float g1 = adam(sacc[1], pw.y, mw.y, vw.y, c);
+                const float g2 = adam(sacc[2], pw.z, mw.z, vw.z, c);
+                const float g3 = adam(sacc[3], pw.w, mw.w, vw.w, c);
+                if (p.sqnorm) {
+                    sq = fma(static_cast<double>(g0), static_cast<double>(g0), sq);
+                    sq = fma(static_cast<double>(g1), static_cast<double>(g1), sq);
+                    sq = fma(static_cast<double>(g2), static_cast<double>(g2), sq);
+                    sq = fma(static_cast<double>(g3), static_cast<double>(g3), sq);
+                }
                 st_state16(p.master_out + base + j, pw.x, pw.y, pw.z, pw.w);
                 st_state16(p.m_out + base + j, mw.x, mw.y, mw.z, mw.w);
                 st_state16(p.v_out + base + j, vw.x, vw.y, vw.z, vw.w);

@@ -22,6 +22,10 @@ inline KernelFn pick_kernel(zero_dtype_t g, zero_dtype_t pd) {
     return fused_step_kernel<__nv_bfloat16, __nv_bfloat16>;
 }
 
+inline KernelFn pick_stats_kernel(zero_dtype_t g) {
+    return g == ZERO_F16 ? grad_stats_kernel<__half> : grad_stats_kernel<__nv_bfloat16>;
+}
+
 inline KernelFn pick_pipe_kernel(zero_dtype_t g, zero_dtype_t pd) {
     if (g == ZERO_F16 && pd == ZERO_F16) return fused_step_pipe_kernel<__half, __half>;
     if (g == ZERO_F16 && pd == ZERO_BF16) return fused_step_pipe_kernel<__half, __nv_bfloat16>;
@@ -49,6 +53,7 @@ inline uint32_t pipe_smem_bytes(int world, int tile) {
 struct DeviceInfo {
     int sms = 0;
     int blocks_per_sm[4] = {0, 0, 0, 0};
+    int stats_blocks_per_sm[2] = {0, 0};
     bool pipe_ready[4] = {false, false, false, false};
 };
 
@@ -80,6 +85,22 @@ inline int grid_limit(zero_dtype_t g, zero_dtype_t pd, int* out) {
         d->blocks_per_sm[which] = n;
     }
     int lim = d->sms * d->blocks_per_sm[which];
+    *out = lim < kMaxBlocks ? lim : kMaxBlocks;
+    return ZERO_OK;
+}
+
+inline int stats_grid_limit(zero_dtype_t g, int* out) {
+    const int which = static_cast<int>(g);
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo* d = nullptr;
+    if (int rc = device_info(&d)) return rc;
+    if (d->stats_blocks_per_sm[which] == 0) {
+        int n = 0;
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, pick_stats_kernel(g), kThreads, 0);
+        if (e != cudaSuccess || n < 1) return fail(ZERO_ERR_CUDA, "occupancy query failed: %s", cudaGetErrorString(e));
+        d->stats_blocks_per_sm[which] = n;
+    }
+    int lim = d->sms * d->stats_blocks_per_sm[which];
     *out = lim < kMaxBlocks ? lim : kMaxBlocks;
     return ZERO_OK;
 }
@@ -201,7 +222,7 @@ inline int prepare_step(const char* fn, const void* const* grad_bufs, int32_t wo
     prm.sqnorm = grad_sqnorm;
     if (grad_sqnorm) {
         prm.ticket = static_cast<unsigned int*>(workspace);
-        prm.partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + kWsPartialsOffset);
+        prm.partials = reinterpret_cast<double*>(static_cast<char*>(workspace) + kWsPartialsOffset);
     }
     // constants: double, rounded once to float
     const double divisor = hp->grad_divisor > 0.0f ? static_cast<double>(hp->grad_divisor) : static_cast<double>(world);
@@ -216,6 +237,10 @@ inline int prepare_step(const char* fn, const void* const* grad_bufs, int32_t wo
     prm.c.rbc1 = static_cast<float>(1.0 / (1.0 - std::pow(static_cast<double>(hp->beta1), t)));
     prm.c.rsbc2 = static_cast<float>(1.0 / std::sqrt(1.0 - std::pow(static_cast<double>(hp->beta2), t)));
     prm.c.decay = static_cast<float>(1.0 - static_cast<double>(hp->lr) * static_cast<double>(hp->weight_decay));
+    prm.c.clip = 1.0f;
+    prm.gate = nullptr;
+    prm.clip_sqnorm = nullptr;
+    prm.max_norm = 0.0;
 
     const int64_t h = common_phase(prm);
     if (h < 0 || h >= count) {
@@ -251,6 +276,107 @@ inline int prepare_step(const char* fn, const void* const* grad_bufs, int32_t wo
     }
     *prm_out = prm;
     *blocks_out = blocks;
+    return ZERO_OK;
+}
+
+// Validate a statistics call and build its kernel parameters (the state
+// pointers stay NULL: the statistics kernel reads gradients only).
+inline int prepare_stats(const char* fn, const void* const* grad_bufs, int32_t world, int64_t padded_numel,
+                         int32_t partition, zero_dtype_t grad_dtype, float loss_scale, float grad_divisor,
+                         int32_t* overflow_flag, double* grad_sqnorm, void* workspace, StepParams* prm_out,
+                         int64_t* blocks_out) {
+    if (!grad_bufs || !overflow_flag) return fail(ZERO_ERR_ARG, "%s: NULL grad_bufs or overflow_flag", fn);
+    if (world < 1 || world > ZERO_MAX_WORLD)
+        return fail(ZERO_ERR_ARG, "%s: world %d outside 1..%d", fn, world, ZERO_MAX_WORLD);
+    if (padded_numel < 0 || padded_numel % world != 0)
+        return fail(ZERO_ERR_ARG, "%s: padded_numel %lld is not a non-negative multiple of world %d", fn,
+                    (long long)padded_numel, world);
+    if (partition != ZERO_ALL_PARTITIONS && (partition < 0 || partition >= world))
+        return fail(ZERO_ERR_RANGE, "%s: partition %d outside 0..%d", fn, partition, world - 1);
+    if (grad_dtype != ZERO_F16 && grad_dtype != ZERO_BF16)
+        return fail(ZERO_ERR_DTYPE, "%s: gradients must be ZERO_F16 or ZERO_BF16", fn);
+    if (!(loss_scale > 0.0f) || !std::isfinite(loss_scale))
+        return fail(ZERO_ERR_ARG, "%s: loss_scale must be positive and finite", fn);
+    if (!(grad_divisor >= 0.0f) || !std::isfinite(grad_divisor))
+        return fail(ZERO_ERR_ARG, "%s: grad_divisor must be >= 0 and finite", fn);
+    if (grad_sqnorm && !workspace) return fail(ZERO_ERR_ARG, "%s: grad_sqnorm needs a workspace", fn);
+    if (!aligned(overflow_flag, 4) || (grad_sqnorm && !aligned(grad_sqnorm, 8)) ||
+        (workspace && !aligned(workspace, 16)))
+        return fail(ZERO_ERR_ALIGN, "%s: flag, norm or workspace misaligned", fn);
+    for (int k = 0; k < world; ++k) {
+        if (!grad_bufs[k]) return fail(ZERO_ERR_ARG, "%s: grad_bufs[%d] is NULL", fn, k);
+        if (!aligned(grad_bufs[k], 2)) return fail(ZERO_ERR_ALIGN, "%s: grad_bufs[%d] not 2-byte aligned", fn, k);
+    }
+    const int64_t P = padded_numel / world;
+    const int64_t begin = partition == ZERO_ALL_PARTITIONS ? 0 : static_cast<int64_t>(partition) * P;
+    const int64_t count = partition == ZERO_ALL_PARTITIONS ? padded_numel : P;
+    if (count == 0) {
+        *blocks_out = 0;
+        return ZERO_OK;
+    }
+    StepParams prm{};
+    prm.world = world;
+    for (int k = 0; k < world; ++k) prm.grads[k] = static_cast<const uint16_t*>(grad_bufs[k]) + begin;
+    prm.count = count;
+    prm.overflow = overflow_flag;
+    prm.sqnorm = grad_sqnorm;
+    if (grad_sqnorm) {
+        prm.ticket = static_cast<unsigned int*>(workspace);
+        prm.partials = reinterpret_cast<double*>(static_cast<char*>(workspace) + kWsPartialsOffset);
+    }
+    const double divisor = grad_divisor > 0.0f ? static_cast<double>(grad_divisor) : static_cast<double>(world);
+    prm.c.inv = static_cast<float>(1.0 / (divisor * static_cast<double>(loss_scale)));
+    prm.c.clip = 1.0f;
+    // gradients only: the first element at which every replica is 16-byte aligned
+    int64_t h = -1;
+    for (int64_t c = 0; c < kVec && h < 0; ++c) {
+        bool good = true;
+        for (int k = 0; k < world && good; ++k)
+            good = ((reinterpret_cast<uintptr_t>(prm.grads[k]) + 2 * c) % 16) == 0;
+        if (good) h = c;
+    }
+    if (h < 0 || h >= count) {
+        prm.head = count;
+        prm.nvec = 0;
+    } else {
+        prm.head = h;
+        prm.nvec = (count - h) / kVec;
+    }
+    int limit = 0;
+    if (int rc = stats_grid_limit(grad_dtype, &limit)) return rc;
+    const int64_t work = prm.nvec > 0 ? prm.nvec : count;
+    int64_t blocks = (work + kThreads - 1) / kThreads;
+    if (blocks > limit) blocks = limit;
+    if (blocks < 1) blocks = 1;
+    *prm_out = prm;
+    *blocks_out = blocks;
+    return ZERO_OK;
+}
+
+inline int launch_stats(const char* fn, const StepParams& prm, int64_t blocks, zero_dtype_t grad_dtype,
+                        zero_stream_t stream) {
+    if (blocks == 0) return ok();
+    pick_stats_kernel(grad_dtype)<<<static_cast<unsigned int>(blocks), kThreads, 0,
+                                    reinterpret_cast<cudaStream_t>(stream)>>>(prm);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(ZERO_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
+    return ok();
+}
+
+// Add the gate and the clipping inputs to prepared step parameters.
+inline int add_gate_and_clip(const char* fn, StepParams* prm, const int32_t* gate, const double* clip_sqnorm,
+                             float max_norm) {
+    if (gate && !aligned(gate, 4)) return fail(ZERO_ERR_ALIGN, "%s: gate misaligned", fn);
+    if (gate && gate == prm->overflow)
+        return fail(ZERO_ERR_ARG, "%s: gate must not be the call's own overflow_flag", fn);
+    if (clip_sqnorm) {
+        if (!aligned(clip_sqnorm, 8)) return fail(ZERO_ERR_ALIGN, "%s: clip_sqnorm misaligned", fn);
+        if (!(max_norm > 0.0f) || !std::isfinite(max_norm))
+            return fail(ZERO_ERR_ARG, "%s: max_norm must be positive and finite", fn);
+    }
+    prm->gate = gate;
+    prm->clip_sqnorm = clip_sqnorm;
+    prm->max_norm = static_cast<double>(max_norm);
     return ZERO_OK;
 }
 

@@ -12,8 +12,8 @@
 // and allocates nothing.
 //
 // Limits and rules:
-//  - the array holds the ticket and kStaticMaxBlocks (4096) partial sums,
-//    16,640 bytes; every GPU that loads the library holds it until exit;
+//  - the array holds the ticket and kStaticMaxBlocks (4096) fp64 partial
+//    sums, 33,024 bytes; every GPU that loads the library holds it until exit;
 //  - the fused kernels' grids are at most SM count x resident blocks (148 or
 //    296 blocks on a B200), so any input size fits; a call whose grid would
 //    need more than 4096 blocks is rejected with ZERO_ERR_RANGE;
@@ -29,7 +29,7 @@ namespace zero {
 namespace {
 
 constexpr int64_t kStaticMaxBlocks = 4096;
-constexpr size_t kStaticScratchBytes = fused::kWsPartialsOffset + sizeof(float) * kStaticMaxBlocks;
+constexpr size_t kStaticScratchBytes = fused::kWsPartialsOffset + sizeof(double) * kStaticMaxBlocks;
 
 // Ticket word at offset 0, per-block partial sums from kWsPartialsOffset,
 // the same layout as the caller-provided workspace.
@@ -95,7 +95,7 @@ extern "C" int zero_reduce_scatter_adam_step_noalloc(
         cudaError_t e = cudaMemsetAsync(scratch, 0, sizeof(unsigned int), reinterpret_cast<cudaStream_t>(stream));
         if (e != cudaSuccess) return fail(ZERO_ERR_CUDA, "%s: clearing the ticket failed: %s", fn, cudaGetErrorString(e));
         prm.ticket = static_cast<unsigned int*>(scratch);
-        prm.partials = reinterpret_cast<float*>(static_cast<char*>(scratch) + kWsPartialsOffset);
+        prm.partials = reinterpret_cast<double*>(static_cast<char*>(scratch) + kWsPartialsOffset);
     }
     return launch_step(fn, prm, blocks, grad_dtype, param_dtype, stream);
 }

@@ -1,30 +1,36 @@
 """ZeroAdam: a ZeRO-2 partitioned mixed-precision Adam step on one GPU.
 
 N data-parallel replicas are simulated by N resident gradient buffers per
-bucket.  A step runs the fused reduce-scatter + Adam kernel over every bucket,
-reads the overflow flag, and commits or skips:
+bucket.  Two ways to run a step, both with an exact skip on overflow:
 
-  - the fp32 master / momentum / variance states and the low-precision
-    parameters live in two banks; a step reads bank `cur` and writes bank
-    `cur ^ 1`, and the bank flips only when no reduced gradient of the whole
-    step was inf or NaN, so a skipped step leaves every state bit-identical;
-  - the loss scale follows zero_loss_scale_update (halve on overflow, double
-    after `growth_interval` good steps) and the Adam step count t advances
-    only on applied updates.
+  mode="banks" (default): the fused reduce-scatter + Adam kernel runs once
+    over every bucket, reading bank `cur` of the fp32 master / momentum /
+    variance states and low-precision parameters and writing bank `cur ^ 1`;
+    the bank flips only when no reduced gradient of the whole step was inf or
+    NaN.  One pass over HBM (2N + 26 bytes per element); the second bank
+    doubles the 12 Psi/N bytes of optimizer state that ZeRO keeps per rank
+    (ZeRO explainer, "Stage 1 - Optimizer State Partitioning").
+  mode="inplace": a statistics pass over every bucket (rank-order sums,
+    overflow flag, squared norm) and then the update in place, gated on the
+    device by that flag: one bank, the pages' 12 Psi/N, for 4N + 26 bytes per
+    element.
 
-The second bank doubles the 12 Psi/N bytes of optimizer state that ZeRO
-keeps per rank (ZeRO explainer, "Stage 1 - Optimizer State Partitioning");
-it buys a single pass over HBM per step with an exact skip.
+max_grad_norm (either mode) clips the unscaled gradients to that global
+norm, with the coefficient computed on the device from the statistics pass
+(banks mode then also takes the two-pass route).
 
-This class only allocates buffers and sequences library calls; all
-arithmetic is in libzero's kernels.
+The loss scale follows zero_loss_scale_update (halve on overflow, double
+after `growth_interval` good steps) and the Adam step count t advances only
+on applied updates.  This class only allocates buffers and sequences library
+calls; all arithmetic is in libzero's kernels.
 """
 from __future__ import annotations
 
 import torch
 
-from . import (ZERO_ALL_PARTITIONS, hparams, zero_flatten_bucket, zero_loss_scale_update,
-               zero_partition_layout, zero_reduce_scatter_adam_step, zero_step_workspace_bytes)
+from . import (ZERO_ALL_PARTITIONS, hparams, zero_flatten_bucket, zero_grad_stats, zero_loss_scale_update,
+               zero_partition_layout, zero_reduce_scatter_adam_step, zero_reduce_scatter_adam_step_gated,
+               zero_step_workspace_bytes)
 
 
 class ZeroAdam:
@@ -32,7 +38,14 @@ class ZeroAdam:
                  lr: float = 1e-3, betas=(0.9, 0.999), eps: float = 1e-8, weight_decay: float = 0.0,
                  grad_dtype=torch.float16, param_dtype=torch.float16, loss_scale: float = 65536.0,
                  growth_interval: int = 1000, min_scale: float = 1.0, grad_divisor: float = 0.0,
-                 track_grad_norm: bool = False, device="cuda"):
+                 track_grad_norm: bool = False, mode: str = "banks", max_grad_norm: float | None = None,
+                 device="cuda"):
+        if mode not in ("banks", "inplace"):
+            raise ValueError("mode must be 'banks' or 'inplace'")
+        if max_grad_norm is not None and not max_grad_norm > 0:
+            raise ValueError("max_grad_norm must be positive")
+        self.mode, self.max_grad_norm = mode, max_grad_norm
+        self.two_pass = mode == "inplace" or max_grad_norm is not None
         self.layout = zero_partition_layout(list(numels), world, bucket_elems, align_elems)
         self.world = world
         self.device = torch.device(device)
@@ -44,19 +57,24 @@ class ZeroAdam:
         self.cur = 0
         L, dev = self.layout, self.device
         f32 = dict(dtype=torch.float32, device=dev)
-        self.master = [[torch.zeros(L.bucket_padded[b], **f32) for _ in range(2)] for b in range(L.n_buckets)]
-        self.m = [[torch.zeros(L.bucket_padded[b], **f32) for _ in range(2)] for b in range(L.n_buckets)]
-        self.v = [[torch.zeros(L.bucket_padded[b], **f32) for _ in range(2)] for b in range(L.n_buckets)]
-        self.params_bank = [[torch.zeros(L.bucket_padded[b], dtype=param_dtype, device=dev) for _ in range(2)]
+        nbank = 1 if mode == "inplace" else 2
+        self.master = [[torch.zeros(L.bucket_padded[b], **f32) for _ in range(nbank)] for b in range(L.n_buckets)]
+        self.m = [[torch.zeros(L.bucket_padded[b], **f32) for _ in range(nbank)] for b in range(L.n_buckets)]
+        self.v = [[torch.zeros(L.bucket_padded[b], **f32) for _ in range(nbank)] for b in range(L.n_buckets)]
+        self.params_bank = [[torch.zeros(L.bucket_padded[b], dtype=param_dtype, device=dev) for _ in range(nbank)]
                             for b in range(L.n_buckets)]
         self.grads = [[torch.zeros(L.bucket_padded[b], dtype=grad_dtype, device=dev) for _ in range(world)]
                       for b in range(L.n_buckets)]
-        self.flag = torch.zeros(1, dtype=torch.int32, device=dev)
-        self.flag_host = torch.zeros(1, dtype=torch.int32, pin_memory=True)
+        # flags[0]: the step's overflow flag (read by the host, the gate of
+        # the two-pass update); flags[1]: the gated update's own flag
+        self.flags = torch.zeros(2, dtype=torch.int32, device=dev)
+        self.flag = self.flags[0:1]
+        self.flag_host = torch.zeros(2, dtype=torch.int32, pin_memory=True)
         self.track_grad_norm = track_grad_norm
-        self.sqnorm = torch.zeros(1, dtype=torch.float64, device=dev) if track_grad_norm else None
+        need_norm = track_grad_norm or max_grad_norm is not None
+        self.sqnorm = torch.zeros(1, dtype=torch.float64, device=dev) if need_norm else None
         self.workspace = (torch.zeros(zero_step_workspace_bytes(), dtype=torch.uint8, device=dev)
-                          if track_grad_norm else None)
+                          if need_norm else None)
         self.last_overflow = 0
 
     # ------------------------------------------------------------ state access
@@ -73,10 +91,11 @@ class ZeroAdam:
             zero_flatten_bucket(self.layout, b, master, self.master[b][0], stream)
             zero_flatten_bucket(self.layout, b, params, self.params_bank[b][0], stream)
             for bank in (self.master, self.params_bank):
-                bank[b][1].copy_(bank[b][0])
+                for extra in bank[b][1:]:
+                    extra.copy_(bank[b][0])
             for bank in (self.m, self.v):
-                bank[b][0].zero_()
-                bank[b][1].zero_()
+                for t in bank[b]:
+                    t.zero_()
         self.cur = 0
         self.t = 0
 
@@ -99,11 +118,13 @@ class ZeroAdam:
         if stream is not None:
             with torch.cuda.stream(stream):
                 return self.launch(None, on_launch)
-        self.flag.zero_()
+        self.flags.zero_()
         if self.sqnorm is not None:
             self.sqnorm.zero_()
         hp = hparams(self.lr, self.betas[0], self.betas[1], self.eps, self.weight_decay,
                      self.t + 1, self.grad_divisor)
+        if self.two_pass:
+            return self._launch_two_pass(hp, on_launch)
         c, n = self.cur, self.cur ^ 1
         for b in range(self.layout.n_buckets):
             if on_launch is not None:
@@ -116,19 +137,41 @@ class ZeroAdam:
             if on_launch is not None:
                 on_launch(b, "after")
 
+    def _launch_two_pass(self, hp, on_launch) -> None:
+        """Statistics over every bucket, then the gated (and clipped) update."""
+        L = self.layout
+        for b in range(L.n_buckets):
+            zero_grad_stats(self.grads[b], L.bucket_padded[b], ZERO_ALL_PARTITIONS, self.scale, self.flag,
+                            self.sqnorm, self.workspace, self.grad_divisor)
+        c = self.cur
+        n = c if self.mode == "inplace" else c ^ 1
+        clip = self.sqnorm if self.max_grad_norm is not None else None
+        for b in range(L.n_buckets):
+            if on_launch is not None:
+                on_launch(b, "before")
+            zero_reduce_scatter_adam_step_gated(
+                self.grads[b], L.bucket_padded[b], ZERO_ALL_PARTITIONS,
+                self.master[b][c], self.m[b][c], self.v[b][c],
+                self.master[b][n], self.m[b][n], self.v[b][n], self.params_bank[b][n],
+                hp, self.scale, self.flags[1:2], None, None, gate=self.flag, clip_sqnorm=clip,
+                max_norm=self.max_grad_norm or 0.0)
+            if on_launch is not None:
+                on_launch(b, "after")
+
     def commit(self, stream=None) -> bool:
         """Read the overflow flag (device -> host), flip banks or skip, update the scale."""
         s = torch.cuda.current_stream() if stream is None else stream
-        self.flag_host.copy_(self.flag, non_blocking=True)
+        self.flag_host.copy_(self.flags, non_blocking=True)
         s.synchronize()
-        flag = int(self.flag_host.item())
+        flag, step_flag = int(self.flag_host[0]), int(self.flag_host[1])
         ovf = int(flag != 0)
-        if flag & 2:
+        if (flag | step_flag) & 2:
             # the kernel abandoned its copy pipeline: the banks were not
             # committed, but the device needs attention
             raise RuntimeError("fused step kernel timed out waiting on its copy pipeline; step not committed")
         if not ovf:
-            self.cur ^= 1
+            if self.mode == "banks":
+                self.cur ^= 1
             self.t += 1
         self.scale, self.good_steps = zero_loss_scale_update(self.scale, self.good_steps, bool(ovf),
                                                              self.growth_interval, self.min_scale)
