@@ -187,6 +187,25 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------- multi-rank helpers
+
+def max_over_ranks(value: float, device) -> float:
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gparams(elems_per_rank: int, n_ranks: int, ms_per_step: float) -> float:
+    """Elements updated per second by all ranks together (weak scaling: every
+    rank runs the same workload), in Gparams/s, from the slowest rank's time."""
+    return n_ranks * elems_per_rank / (ms_per_step * 1e-3) / 1e9
+
+
 # --------------------------------------------------------------- GPU side
 
 def fill_workload(opt, w, seed_base: int):
@@ -291,12 +310,9 @@ def run_gpu(args):
         for i in range(0, len(es), 2):
             launch_ms.append(es[i].elapsed_time(es[i + 1]))
             launch_elems.append(L.bucket_padded[b])
-    if world_gpus > 1:
-        tt = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms, "cuda")
     ms_per_step = ms / args.steps
-    value = world_gpus * psi_p / (ms_per_step * 1e-3) / 1e9
+    value = whole_job_gparams(psi_p, world_gpus, ms_per_step)
     bpe = bytes_per_elem(w.world)
     peak, peak_kind = peaks()
     kern_bytes = sum(launch_elems) * bpe
@@ -429,15 +445,10 @@ def run_e2e(opt, args, stream, barrier, world_gpus):
         opt.step_from_host(host)
     t1.record(stream)
     barrier()
-    ms = t0.elapsed_time(t1)
-    if world_gpus > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), "cuda")
     psi_p = sum(opt.layout.bucket_padded)
     del host
-    return {"value": world_gpus * psi_p * steps / (ms * 1e-3) / 1e9, "unit": UNIT,
+    return {"value": whole_job_gparams(psi_p, world_gpus, ms / steps), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4, "steps": steps,
             "ms_per_step": ms / steps}
 

@@ -355,6 +355,23 @@ int zero_allgather_params(const void* const* shards, int32_t world, int64_t shar
                           int64_t part_numel, zero_dtype_t dtype, void* dst,
                           zero_stream_t stream);
 
+/*
+ * zero_test_wait_timeout - self-test of the bounded device waits.
+ *
+ * The paper has no counterpart: a test hook of this library.  The
+ * shared-memory pipeline of the fused step waits on mbarriers that its own
+ * bulk copies complete, each wait limited to 2 s of wall time; when a limit
+ * runs out the kernel ORs 2 into the overflow flag, stops, and returns.
+ * This call runs the same wait routine on an mbarrier that nothing ever
+ * arrives at, with the limit `limit_ns`: after about that long it ORs 2 into
+ * *status and the kernel returns, so a caller can check that a stuck wait
+ * ends with a status instead of a hang.
+ * status    device int32, OR-ed into
+ * limit_ns  0 .. 1e10
+ * Errors: ZERO_ERR_ARG, ZERO_ERR_ALIGN, ZERO_ERR_CUDA.
+ */
+int zero_test_wait_timeout(int32_t* status, int64_t limit_ns, zero_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Host helpers                                                              */
 /* ------------------------------------------------------------------------ */

@@ -169,3 +169,9 @@ def test_allgather_and_flatten_reject_bad_arguments():
     assert L.zero_flatten_bucket(ctypes.byref(lay), 0, tp, 5, 0x30000, None) == -3
     assert L.zero_flatten_bucket(ctypes.byref(lay), 0, tp, 2, 0x30002, None) == -2
     assert L.zero_flatten_bucket(ctypes.byref(lay), 0, tp, 0, 0x10004, None) == -1
+
+
+def test_wait_timeout_rejects_bad_arguments():
+    assert Z.lib.zero_test_wait_timeout(None, 1000, None) == -1
+    assert Z.lib.zero_test_wait_timeout(0x10002, 1000, None) == -2
+    assert Z.lib.zero_test_wait_timeout(0x10000, -1, None) == -1

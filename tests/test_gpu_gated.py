@@ -225,3 +225,35 @@ def test_zeroadam_banks_mode_with_clipping():
         master, m, v, p = opt.state(b)
         assert assert_f32_close(host_f32(master), states[b].master, "master") == 0
         assert assert_u16_close(host_u16(p), states[b].params, "params") == 0
+
+
+@pytest.mark.parametrize("mode", ["banks", "inplace"])
+def test_checkpoint_resume_bit_identical(mode):
+    """Save after step 2, reload into a fresh optimizer: steps 3-5 (one with
+    an injected overflow) are bit-identical to the uninterrupted run."""
+    numels = [400_000, 13, 900_001]
+    N = 4
+    adam = workloads.AdamConfig(weight_decay=0.01)
+    L, opt, _ = _opt_and_oracle(numels, N, 500_000, adam, mode)
+    grads = {}
+    for step in range(1, 6):
+        G = _grads_for(L, N, step, 65536.0 if step < 5 else 32768.0)
+        if step == 4:
+            workloads.inject(G[0][1], np.array([2]), np.array([False]))
+        grads[step] = G
+    for step in (1, 2):
+        _upload(opt, grads[step])
+        opt.step()
+    sd = opt.state_dict()
+    for step in (3, 4, 5):
+        _upload(opt, grads[step])
+        opt.step()
+    L2, opt2, _ = _opt_and_oracle(numels, N, 500_000, adam, mode)
+    opt2.load_state_dict(sd)
+    for step in (3, 4, 5):
+        _upload(opt2, grads[step])
+        opt2.step()
+    assert (opt.t, opt.scale, opt.good_steps) == (opt2.t, opt2.scale, opt2.good_steps) == (4, 32768.0, 1)
+    for b in range(L.n_buckets):
+        for x, y in zip(opt.state(b), opt2.state(b)):
+            assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))

@@ -1,0 +1,78 @@
+"""The benchmark's multi-rank path on the CPU: world_size 2 over gloo.
+
+Under torchrun every GPU runs its own instance of the workload (the N data-
+parallel replicas are simulated inside each GPU, so no data crosses GPUs);
+the ranks only agree on the timing: the step time is the maximum over ranks
+and the whole-job value sums every rank's elements.  These tests run that
+host logic in two gloo processes, and the reference arm's rank rule (rank 0
+alone prints, the others exit 0 without work).
+"""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        ms = [12.5, 10.0][rank]               # rank 0 is the slow one
+        got = bench.max_over_ranks(ms, "cpu")
+        value = bench.whole_job_gparams(1_000_000_000, world, got)
+        q.put((rank, got, value))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_whole_job_value_gloo():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    assert [r[1] for r in res] == [12.5, 12.5]
+    assert all(abs(r[2] - 2 * 1e9 / 12.5e-3 / 1e9) < 1e-9 for r in res)
+
+
+def test_helpers_without_process_group():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(3.0, "cpu") == 3.0
+    assert bench.whole_job_gparams(1_557_611_200, 1, 9.72) == pytest.approx(160.25, rel=1e-3)
+
+
+def test_reference_arm_two_ranks_only_rank0_prints():
+    env = dict(os.environ, PYTHONPATH=ROOT)
+    outs = []
+    for rank in (0, 1):
+        e = dict(env, RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank))
+        r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                            "--steps", "1", "--warmup", "0", "--ref-sample", "65536"],
+                           env=e, capture_output=True, text=True, timeout=300)
+        assert r.returncode == 0, r.stderr
+        outs.append(r.stdout.strip())
+    assert outs[1] == ""
+    line = json.loads(outs[0].splitlines()[-1])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"

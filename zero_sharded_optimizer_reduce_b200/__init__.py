@@ -83,6 +83,8 @@ def _load():
         vp, vp, vp, vp, vp, vp, vp, ctypes.c_int,
         ctypes.POINTER(AdamHParams), f32, vp, vp, vp, vp, vp, f32, vp]
     L.zero_reduce_scatter_adam_step_gated.restype = ctypes.c_int
+    L.zero_test_wait_timeout.argtypes = [vp, i64, vp]
+    L.zero_test_wait_timeout.restype = ctypes.c_int
     L.zero_allgather_params.argtypes = [ctypes.POINTER(vp), i32, i64, i64, ctypes.c_int, vp, vp]
     L.zero_allgather_params.restype = ctypes.c_int
     L.zero_loss_scale_update.argtypes = [ctypes.POINTER(f32), ctypes.POINTER(i32), i32, i32, f32]
@@ -269,6 +271,11 @@ def zero_loss_scale_update(scale: float, good_steps: int, overflow: bool,
     _check(lib.zero_loss_scale_update(ctypes.byref(s), ctypes.byref(g), int(bool(overflow)),
                                       growth_interval, min_scale))
     return s.value, g.value
+
+
+def zero_test_wait_timeout(status, limit_ns: int, stream=None) -> None:
+    """Run the bounded-wait self-test: ORs 2 into status after ~limit_ns."""
+    _check(lib.zero_test_wait_timeout(_ptr(status), int(limit_ns), _stream(stream)))
 
 
 def version() -> str:

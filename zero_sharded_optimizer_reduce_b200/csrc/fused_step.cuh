@@ -374,6 +374,9 @@ __global__ void __launch_bounds__(kThreads) grad_stats_kernel(const __grid_const
 
 // ------------------------------------------------------- bulk-copy pipeline
 
+// (the pipeline's helpers follow; wait_timeout_kernel below exercises the
+// bounded wait on its own)
+
 __device__ __forceinline__ uint32_t smem_addr(const void* ptr) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(ptr));
 }
@@ -407,17 +410,17 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
-// Wait for the phase of `bar` with the given parity, for at most
-// kWaitLimitNs of wall time.  Returns false when the limit ran out.
+// Wait for the phase of `bar` with the given parity, for at most `limit_ns`
+// of wall time (%globaltimer).  Returns false when the limit ran out.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
         for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
     }
 }
 
@@ -583,6 +586,18 @@ __global__ void __launch_bounds__(kPipeThreads, 1) fused_step_pipe_kernel(const 
 }
 
 // ------------------------------------------------------------------ host side
+
+// Self-test of the bounded wait: one thread waits on an mbarrier that
+// nothing ever arrives at, with a short limit.  It must give up, record
+// kFlagDeviceTimeout in *status and return; the CTA's shared memory holds no
+// copy in flight, so nothing else needs draining.
+__global__ void wait_timeout_kernel(int32_t* status, uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (!mbar_wait_bounded(&bar, 0u, limit_ns)) atomicOr(status, kFlagDeviceTimeout);
+}
 
 }  // namespace
 }  // namespace fused

@@ -43,3 +43,4 @@ extern "C" int zero_reduce_scatter_adam_step_gated(
     if (int rc = add_gate_and_clip(fn, &prm, gate, clip_sqnorm, max_norm)) return rc;
     return launch_step(fn, prm, blocks, grad_dtype, param_dtype, stream);
 }
+

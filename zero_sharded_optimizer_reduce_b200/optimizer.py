@@ -191,6 +191,33 @@ class ZeroAdam:
                     self.grads[b][k].copy_(host_grads[b][k], non_blocking=True)
             return self.step()
 
+    # -------------------------------------------------------------- checkpoint
+    def state_dict(self) -> dict:
+        """Host copy of everything a resumed run needs: the committed master,
+        m, v and parameters of every bucket, t, the loss scale and the
+        good-step count, plus the layout they belong to."""
+        L = self.layout
+        return {
+            "world": self.world, "bucket_padded": list(L.bucket_padded), "mode": self.mode,
+            "t": self.t, "scale": self.scale, "good_steps": self.good_steps,
+            "buckets": [{name: x.detach().cpu().clone() for name, x in zip(("master", "m", "v", "params"),
+                                                                            self.state(b))}
+                        for b in range(L.n_buckets)],
+        }
+
+    def load_state_dict(self, sd: dict) -> None:
+        """Restore a state_dict taken from an optimizer with the same layout."""
+        L = self.layout
+        if sd["world"] != self.world or list(sd["bucket_padded"]) != list(L.bucket_padded):
+            raise ValueError("checkpoint layout does not match this optimizer")
+        for b, bucket in enumerate(sd["buckets"]):
+            for bank_list, name in ((self.master, "master"), (self.m, "m"), (self.v, "v"),
+                                    (self.params_bank, "params")):
+                for t in bank_list[b]:
+                    t.copy_(bucket[name].view(t.dtype) if bucket[name].dtype != t.dtype else bucket[name])
+        self.cur = 0
+        self.t, self.scale, self.good_steps = int(sd["t"]), float(sd["scale"]), int(sd["good_steps"])
+
     def grad_sqnorm(self) -> float:
         """Sum of squared unscaled gradients of the last step (if tracked)."""
         return float(self.sqnorm.item()) if self.sqnorm is not None else float("nan")
