@@ -373,6 +373,43 @@ int zero_allgather_params(const void* const* shards, int32_t world, int64_t shar
 int zero_test_wait_timeout(int32_t* status, int64_t limit_ns, zero_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Multi-process ranks: sharing gradient and parameter buffers               */
+/* ------------------------------------------------------------------------ */
+
+/* Opaque CUDA IPC handle (the bytes of a cudaIpcMemHandle_t). */
+typedef struct {
+    unsigned char bytes[64];
+} zero_ipc_handle_t;
+
+/*
+ * zero_ipc_export / zero_ipc_import / zero_ipc_close - share device buffers
+ * between the processes (ranks) of one node.
+ *
+ * Source: ZeRO explainer, "Stage 2 - Gradient Partitioning (P_os+g)": each
+ * rank needs, from every other rank, only the gradient slice of its own
+ * partition.  With the peers' buffers mapped, a rank passes them (in rank
+ * order, its own included) as `grad_bufs` to zero_reduce_scatter_adam_step
+ * with partition = its rank: the kernel itself performs the reduce-scatter by
+ * reading each peer's slice (NVLink P2P loads across GPUs), in fixed rank
+ * order.  The updated parameter slots are then gathered the same way with
+ * zero_allgather_params.  The ranks must synchronise on the host (a barrier)
+ * between writing gradients and the step, and after the gather.
+ *
+ * zero_ipc_export: `ptr` any device address inside an allocation of the
+ *   current process; fills `handle` (of the whole allocation) and `offset`
+ *   (bytes from the allocation's start to ptr).  Host only.
+ * zero_ipc_import: maps a handle exported by another process on this node
+ *   (any device; peer access is enabled as needed); *ptr = mapped base +
+ *   offset; *base is what zero_ipc_close takes.  Not for handles of the
+ *   calling process itself.
+ * zero_ipc_close: unmaps a base returned by zero_ipc_import.
+ * Errors: ZERO_ERR_ARG, ZERO_ERR_CUDA.
+ */
+int zero_ipc_export(const void* ptr, zero_ipc_handle_t* handle, int64_t* offset);
+int zero_ipc_import(const zero_ipc_handle_t* handle, int64_t offset, void** ptr, void** base);
+int zero_ipc_close(void* base);
+
+/* ------------------------------------------------------------------------ */
 /* Host helpers                                                              */
 /* ------------------------------------------------------------------------ */
 

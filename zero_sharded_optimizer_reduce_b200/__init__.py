@@ -43,6 +43,21 @@ class _Layout(ctypes.Structure):
                 ("tensor_offset", ctypes.POINTER(ctypes.c_int64))]
 
 
+class IpcHandle(ctypes.Structure):
+    _fields_ = [("bytes", ctypes.c_ubyte * 64)]
+
+
+class DevicePtr:
+    """A raw device address with a dtype, accepted wherever a tensor is
+    (for buffers mapped from another process)."""
+
+    def __init__(self, ptr: int, dtype):
+        self.ptr, self.dtype = int(ptr), dtype
+
+    def data_ptr(self) -> int:
+        return self.ptr
+
+
 class AdamHParams(ctypes.Structure):
     _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
                 ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float),
@@ -83,6 +98,12 @@ def _load():
         vp, vp, vp, vp, vp, vp, vp, ctypes.c_int,
         ctypes.POINTER(AdamHParams), f32, vp, vp, vp, vp, vp, f32, vp]
     L.zero_reduce_scatter_adam_step_gated.restype = ctypes.c_int
+    L.zero_ipc_export.argtypes = [vp, ctypes.POINTER(IpcHandle), ctypes.POINTER(i64)]
+    L.zero_ipc_export.restype = ctypes.c_int
+    L.zero_ipc_import.argtypes = [ctypes.POINTER(IpcHandle), i64, ctypes.POINTER(vp), ctypes.POINTER(vp)]
+    L.zero_ipc_import.restype = ctypes.c_int
+    L.zero_ipc_close.argtypes = [vp]
+    L.zero_ipc_close.restype = ctypes.c_int
     L.zero_test_wait_timeout.argtypes = [vp, i64, vp]
     L.zero_test_wait_timeout.restype = ctypes.c_int
     L.zero_allgather_params.argtypes = [ctypes.POINTER(vp), i32, i64, i64, ctypes.c_int, vp, vp]
@@ -278,8 +299,30 @@ def zero_test_wait_timeout(status, limit_ns: int, stream=None) -> None:
     _check(lib.zero_test_wait_timeout(_ptr(status), int(limit_ns), _stream(stream)))
 
 
+def zero_ipc_export(tensor) -> tuple:
+    """(handle bytes, byte offset) of a device buffer, for another process."""
+    h = IpcHandle()
+    off = ctypes.c_int64()
+    _check(lib.zero_ipc_export(_ptr(tensor), ctypes.byref(h), ctypes.byref(off)))
+    return bytes(h.bytes), int(off.value)
+
+
+def zero_ipc_import(handle: bytes, offset: int) -> tuple:
+    """Map another process's buffer: returns (device address, mapping base)."""
+    h = IpcHandle()
+    ctypes.memmove(h.bytes, handle, 64)
+    ptr, base = ctypes.c_void_p(), ctypes.c_void_p()
+    _check(lib.zero_ipc_import(ctypes.byref(h), int(offset), ctypes.byref(ptr), ctypes.byref(base)))
+    return int(ptr.value), int(base.value)
+
+
+def zero_ipc_close(base: int) -> None:
+    _check(lib.zero_ipc_close(ctypes.c_void_p(base)))
+
+
 def version() -> str:
     return lib.zero_version().decode()
 
 
 from .optimizer import ZeroAdam  # noqa: E402  (uses the bindings above)
+from .distributed import DistributedZeroAdam  # noqa: E402

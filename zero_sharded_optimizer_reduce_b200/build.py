@@ -21,7 +21,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libzero.so")
 
-SOURCES = ["step.cu", "step_static.cu", "stats.cu", "selftest.cu", "copy.cu", "host.cpp"]
+SOURCES = ["step.cu", "step_static.cu", "stats.cu", "selftest.cu", "copy.cu", "host.cpp", "ipc.cpp"]
 HEADERS = [os.path.join(CSRC, n) for n in ("common.h", "fused_step.cuh", "step_launch.h")] + [os.path.join(INCLUDE, "zero.h")]
 
 NVCC_FLAGS = [
