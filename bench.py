@@ -419,6 +419,53 @@ def run_sweep(args):
     return 0
 
 
+def run_stage3(args):
+    """Layer-wise ZeRO-3 step on the 6.7B GPT shape (32 layers + embedding
+    unit, N = 8): two gathers per unit plus the per-unit statistics and gated
+    in-place update, timed with and without gather prefetch.  One JSON line."""
+    import torch
+    import zero_sharded_optimizer_reduce_b200 as Z
+    torch.cuda.set_device(0)
+    w = workloads.gpt_6p7b_layerwise()
+    out = {}
+    for prefetch in (False, True):
+        s3 = Z.ZeroStage3(w.numels, w.world, lr=w.adam.lr, betas=(w.adam.beta1, w.adam.beta2), eps=w.adam.eps,
+                          weight_decay=w.adam.weight_decay, loss_scale=w.loss_scale, prefetch=prefetch)
+        gen = torch.Generator(device="cuda")
+        for u in range(s3.U):
+            gen.manual_seed(4000 + u)
+            s3.master[u].normal_(0.0, w.master_std, generator=gen)
+            s3.master[u][s3.layout.bucket_numel[u]:].zero_()
+        for k, g in enumerate(s3.grads):
+            gen.manual_seed(5000 + k)
+            g.copy_(torch.randn(g.numel(), generator=gen, device="cuda").mul_(w.grad_std * w.loss_scale))
+        s3.load(list(s3.master))
+        for _ in range(args.warmup):
+            s3.step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            s3.step()
+        e1.record()
+        torch.cuda.synchronize()
+        out[prefetch] = e0.elapsed_time(e1) / args.steps
+        del s3
+        torch.cuda.empty_cache()
+    psi = sum(Z.zero_partition_layout(w.numels, w.world, 1, 8).bucket_padded)
+    N = w.world
+    step_bytes = psi * (8 + 4 * N + 26)      # 2 gathers x (2 read + 2 write) + statistics + update
+    peak, peak_kind = peaks()
+    line = {"metric": "ZeRO-3 layer-wise step (gathers + statistics + gated in-place update)", "unit": "Gparams/s",
+            "value": psi / (out[True] * 1e-3) / 1e9, "ms_per_step": out[True], "ms_per_step_no_prefetch": out[False],
+            "prefetch_gain": out[False] / out[True] - 1.0, "steps": args.steps, "warmup": args.warmup,
+            "config": {"workload": w.name, "psi_padded": psi, "world": N, "units": len(w.numels)},
+            "hbm_gbs": step_bytes / (out[True] * 1e-3) / 1e9, "bytes_per_elem": 8 + 4 * N + 26,
+            "frac_measured": step_bytes / (out[True] * 1e-3) / 1e9 / peak, "peak_kind": peak_kind}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_e2e(opt, args, stream, barrier, world_gpus):
     """Same step through ZeroAdam.step_from_host: every step copies the N
     replicas' gradients from pinned host memory and reads the flag back."""
@@ -468,6 +515,7 @@ def main(argv=None):
     ap.add_argument("--world", type=int, default=8, help="simulated replicas of the flat workload")
     ap.add_argument("--grad-dtype", choices=["f16", "bf16"], default="f16")
     ap.add_argument("--sweep", action="store_true", help="flat bandwidth sweep, one JSON line per point")
+    ap.add_argument("--stage3", action="store_true", help="layer-wise ZeRO-3 step on the 6.7B shape, prefetch on/off")
     ap.add_argument("--mode", choices=["banks", "inplace"], default="banks",
                     help="banks: two state banks, one pass; inplace: one bank, statistics pass + gated update")
     ap.add_argument("--max-grad-norm", type=float, default=None, help="clip gradients to this global norm")
@@ -479,6 +527,8 @@ def main(argv=None):
         return run_reference(args)
     if args.sweep:
         return run_sweep(args)
+    if args.stage3:
+        return run_stage3(args)
     return run_gpu(args)
 
 
