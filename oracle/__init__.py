@@ -66,45 +66,50 @@ def build(force: bool = False) -> str:
 _lib = None
 
 
+def load_library(path: str):
+    """Load a compiled oracle library and declare its C signatures."""
+    L = ctypes.CDLL(path)
+    i64, i32, f32, f64 = ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_double
+    vp = ctypes.c_void_p
+    L.orc_f16_to_f32.restype = f32
+    L.orc_f16_to_f32.argtypes = [ctypes.c_uint16]
+    L.orc_bf16_to_f32.restype = f32
+    L.orc_bf16_to_f32.argtypes = [ctypes.c_uint16]
+    L.orc_f32_to_f16.restype = ctypes.c_uint16
+    L.orc_f32_to_f16.argtypes = [f32]
+    L.orc_f32_to_bf16.restype = ctypes.c_uint16
+    L.orc_f32_to_bf16.argtypes = [f32]
+    for n in ("orc_f16_to_f32_array", "orc_bf16_to_f32_array",
+              "orc_f32_to_f16_array", "orc_f32_to_bf16_array"):
+        getattr(L, n).argtypes = [vp, vp, i64]
+        getattr(L, n).restype = None
+    L.orc_reduce.argtypes = [vp, i32, ctypes.c_int, i64, i64, vp]
+    L.orc_reduce.restype = None
+    L.orc_any_nonfinite.argtypes = [vp, i64]
+    L.orc_any_nonfinite.restype = i32
+    L.orc_grad_sqnorm.argtypes = [vp, i64, f32]
+    L.orc_grad_sqnorm.restype = f64
+    L.orc_adam_constants.argtypes = [f32, f32, f32, f32, f32, i64, f64, f32, vp]
+    L.orc_adam_constants.restype = None
+    L.orc_adam_update.argtypes = [vp, i64, vp, vp, vp, vp, vp, ctypes.c_int]
+    L.orc_adam_update.restype = None
+    L.orc_clip_coefficient.argtypes = [f64, f64]
+    L.orc_clip_coefficient.restype = f32
+    L.orc_adam_update_clipped.argtypes = [vp, i64, vp, f32, vp, vp, vp, vp, ctypes.c_int]
+    L.orc_adam_update_clipped.restype = None
+    L.orc_allgather.argtypes = [vp, i32, i64, i64, vp]
+    L.orc_allgather.restype = None
+    L.orc_threads.restype = i32
+    L.orc_threads.argtypes = []
+    L.orc_set_threads.restype = None
+    L.orc_set_threads.argtypes = [i32]
+    return L
+
+
 def lib():
     global _lib
     if _lib is None:
-        L = ctypes.CDLL(build())
-        i64, i32, f32, f64 = ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_double
-        vp = ctypes.c_void_p
-        L.orc_f16_to_f32.restype = f32
-        L.orc_f16_to_f32.argtypes = [ctypes.c_uint16]
-        L.orc_bf16_to_f32.restype = f32
-        L.orc_bf16_to_f32.argtypes = [ctypes.c_uint16]
-        L.orc_f32_to_f16.restype = ctypes.c_uint16
-        L.orc_f32_to_f16.argtypes = [f32]
-        L.orc_f32_to_bf16.restype = ctypes.c_uint16
-        L.orc_f32_to_bf16.argtypes = [f32]
-        for n in ("orc_f16_to_f32_array", "orc_bf16_to_f32_array",
-                  "orc_f32_to_f16_array", "orc_f32_to_bf16_array"):
-            getattr(L, n).argtypes = [vp, vp, i64]
-            getattr(L, n).restype = None
-        L.orc_reduce.argtypes = [vp, i32, ctypes.c_int, i64, i64, vp]
-        L.orc_reduce.restype = None
-        L.orc_any_nonfinite.argtypes = [vp, i64]
-        L.orc_any_nonfinite.restype = i32
-        L.orc_grad_sqnorm.argtypes = [vp, i64, f32]
-        L.orc_grad_sqnorm.restype = f64
-        L.orc_adam_constants.argtypes = [f32, f32, f32, f32, f32, i64, f64, f32, vp]
-        L.orc_adam_constants.restype = None
-        L.orc_adam_update.argtypes = [vp, i64, vp, vp, vp, vp, vp, ctypes.c_int]
-        L.orc_adam_update.restype = None
-        L.orc_clip_coefficient.argtypes = [f64, f64]
-        L.orc_clip_coefficient.restype = f32
-        L.orc_adam_update_clipped.argtypes = [vp, i64, vp, f32, vp, vp, vp, vp, ctypes.c_int]
-        L.orc_adam_update_clipped.restype = None
-        L.orc_allgather.argtypes = [vp, i32, i64, i64, vp]
-        L.orc_allgather.restype = None
-        L.orc_threads.restype = i32
-        L.orc_threads.argtypes = []
-        L.orc_set_threads.restype = None
-        L.orc_set_threads.argtypes = [i32]
-        _lib = L
+        _lib = load_library(build())
     return _lib
 
 

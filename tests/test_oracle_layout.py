@@ -105,3 +105,12 @@ def test_layout_rejects_bad_arguments():
         oracle.partition_layout([3], 2, -1)
     with pytest.raises(ValueError):
         oracle.partition_layout([-1], 2)
+
+
+def test_allgather_with_offset_brute_force():
+    rng = np.random.Generator(np.random.PCG64(8))
+    shards = [rng.integers(0, 65536, 50).astype(np.uint16) for _ in range(3)]
+    for off, part in [(0, 50), (7, 11), (49, 1), (13, 0)]:
+        got = oracle.allgather(shards, off, part)
+        ref = np.concatenate([sh[off:off + part] for sh in shards])
+        assert np.array_equal(got, ref)

@@ -79,3 +79,14 @@ def test_grad_sqnorm_matches_fp64_sum():
     inv = np.float32(1.0 / 4096.0)
     ref = float(np.sum((s.astype(np.float64) * float(inv)) ** 2))
     assert abs(oracle.grad_sqnorm(s, inv) - ref) <= 1e-12 * ref
+
+
+def test_nan_alone_sets_the_flag():
+    G = [workloads.grads(64, 95 + k, 1e-3, 1024.0) for k in range(3)]
+    G[1][17] = workloads.F16_NAN
+    s = oracle.reduce(G)
+    assert np.isnan(s[17]) and oracle.any_nonfinite(s) == 1
+    G[1][17] = workloads.F16_POS_INF
+    G[2][17] = 0xFC00                          # -inf: inf + (-inf) is NaN
+    s = oracle.reduce(G)
+    assert np.isnan(s[17]) and oracle.any_nonfinite(s) == 1
