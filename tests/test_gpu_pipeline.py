@@ -2,8 +2,8 @@
 
 Calls whose arrays share a 16-byte phase and that give every SM at least two
 tiles run the bulk-copy pipeline kernel; these sizes are chosen above that
-threshold (tile = about 80 KB of inputs per stage, i.e. 5632 elements at
-N = 1 down to 768 at N = 64, on 148 SMs), with ragged tails, a shifted
+threshold (two stages of at most 180 KB: 6144 elements per tile at N = 1
+down to 2048 at N = 16, on 148 SMs), with ragged tails, a shifted
 common phase (scalar head), single partitions, bf16 and N up to 64.
 """
 import numpy as np
@@ -21,8 +21,12 @@ SMS = 148
 
 
 def _tile(world):
-    t = (81920 // (2 * world + 12)) // 256 * 256
-    return max(768, min(8192, t))
+    """The pipeline tile for N replicas (N <= 20): the largest multiple of 512
+    whose two stages fit in 180 KB.  Above N = 20 the register kernel runs;
+    the size then only has to be large."""
+    if world > 20:
+        return 1536
+    return min(8192, (180 * 1024 // (2 * (2 * world + 12))) // 512 * 512)
 
 
 @pytest.mark.parametrize("world", [1, 2, 3, 4, 8, 16, 64])

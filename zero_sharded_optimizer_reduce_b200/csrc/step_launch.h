@@ -9,9 +9,10 @@ namespace zero {
 namespace fused {
 namespace {
 
-constexpr uint32_t kPipeStageTarget = 80u * 1024u;  // bytes of one pipeline stage, aimed for
+constexpr uint32_t kPipeSmemTarget = 180u * 1024u;  // shared memory of both stages, at most
 constexpr uint32_t kPipeMinTile = 1536;             // elements: 3/4 of 4 x consumer threads
 constexpr uint32_t kPipeSmemMax = 220u * 1024u;     // dynamic shared memory cap
+constexpr int kPipeMaxWorld = 20;                   // largest N measured to gain from the pipeline
 
 using KernelFn = void (*)(StepParams);
 
@@ -33,13 +34,16 @@ inline KernelFn pick_pipe_kernel(zero_dtype_t g, zero_dtype_t pd) {
     return fused_step_pipe_kernel<__nv_bfloat16, __nv_bfloat16>;
 }
 
-// Pipeline tile for N replicas: about kPipeStageTarget bytes per stage, a
-// multiple of 256 elements.  0 (the register kernel runs) when a tile would
-// keep fewer than 3/4 of the consumer threads busy (4 elements each): with
-// the stage target that is N > 20, where the register kernel is faster.
+// Pipeline tile for N replicas: the largest multiple of 512 elements whose
+// two stages fit in kPipeSmemTarget, for N <= kPipeMaxWorld; 0 (the
+// register kernel runs) otherwise.  Measured on B200: large stages and tiles
+// that split evenly into rounds of 4 elements per consumer thread run
+// fastest (N = 8: T = 3072, 6.96 TB/s; T = 2304, 6.07 TB/s); above N = 20
+// the register kernel is faster than the small tiles that would fit.
 inline int pipe_tile(int world) {
+    if (world > kPipeMaxWorld) return 0;
     const uint32_t per_elem = 2u * static_cast<uint32_t>(world) + 12u;
-    uint32_t t = kPipeStageTarget / per_elem / 256u * 256u;
+    uint32_t t = kPipeSmemTarget / (static_cast<uint32_t>(kPipeStages) * per_elem) / 512u * 512u;
     if (t > 8192u) t = 8192u;
     if (t < kPipeMinTile) return 0;
     if (static_cast<uint64_t>(kPipeStages) * t * per_elem > kPipeSmemMax) return 0;
