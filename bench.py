@@ -95,7 +95,9 @@ class ClockSampler:
         self.fh.close()
         sm, mx, reasons = [], 0.0, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
+        with open(self.path) as f:
+            lines = f.readlines()
+        for line in lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
@@ -118,7 +120,8 @@ class ClockSampler:
 def source_digest() -> str:
     h = hashlib.sha256()
     p = os.path.join(ROOT, "zero_sharded_optimizer_reduce_b200", "csrc", "fused_step.cuh")
-    h.update(open(p, "rb").read())
+    with open(p, "rb") as f:
+        h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -127,7 +130,8 @@ def profiled_traffic(elems_per_launch: float):
     if it was taken on the current kernel source; else None."""
     p = os.path.join(ROOT, "profiles", "fused_step_traffic.json")
     try:
-        d = json.load(open(p))
+        with open(p) as f:
+            d = json.load(f)
     except Exception:
         return None
     if d.get("kernel_source_sha256_16") != source_digest():

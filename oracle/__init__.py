@@ -335,13 +335,16 @@ def loss_scale_update(scale: float, good_steps: int, overflow: bool,
 
     Overflow: the update is skipped, the scale halves (not below min_scale)
     and the good-step counter restarts.  Otherwise the counter grows and the
-    scale doubles after `growth_interval` consecutive good steps.
+    scale doubles after `growth_interval` consecutive good steps, unless the
+    doubled fp32 scale would be infinite.
     """
     if overflow:
         return max(scale / 2.0, min_scale), 0
     good_steps += 1
     if good_steps >= growth_interval:
-        return scale * 2.0, 0
+        twice = scale * 2.0
+        fits = twice <= float(np.finfo(np.float32).max)   # the scale is an fp32 value
+        return (twice if fits else scale), 0
     return scale, good_steps
 
 

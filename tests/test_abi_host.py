@@ -21,7 +21,8 @@ HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))
 
 
 def _declared_functions():
-    text = open(HEADER).read()
+    with open(HEADER) as f:
+        text = f.read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(zero_[a-z0-9_]+)\s*\(", text)))
 
@@ -175,3 +176,10 @@ def test_wait_timeout_rejects_bad_arguments():
     assert Z.lib.zero_test_wait_timeout(None, 1000, None) == -1
     assert Z.lib.zero_test_wait_timeout(0x10002, 1000, None) == -2
     assert Z.lib.zero_test_wait_timeout(0x10000, -1, None) == -1
+
+
+def test_loss_scale_growth_stops_below_inf():
+    big = float(np.float32(3.0e38))
+    s, g = Z.zero_loss_scale_update(big, 0, False, growth_interval=1)
+    so, go = oracle.loss_scale_update(big, 0, False, growth_interval=1)
+    assert (s, g) == (so, go) == (big, 0)

@@ -315,3 +315,37 @@ def test_zeroadam_multi_bucket_matches_stage2_with_overflow_skip():
                 for x, y in zip(before[b], opt.state(b)):
                     assert torch.equal(x.view(torch.uint8) if x.dtype != torch.uint8 else x,
                                        y.view(torch.uint8) if y.dtype != torch.uint8 else y)
+
+
+def test_flatten_many_tensors_spans_several_launches():
+    # 150 tensors in one bucket: the copy kernel takes 64 segments per launch
+    rng = np.random.Generator(np.random.PCG64(13))
+    numels = rng.integers(1, 3000, 150).tolist()
+    lay = Z.zero_partition_layout(numels, 8, 0)
+    olay = oracle.partition_layout(numels, 8, 0)
+    host = [rng.integers(0, 2 ** 16, n, dtype=np.uint64).astype(np.uint16) for n in numels]
+    dev = [torch.from_numpy(h.view(np.int16).copy()).cuda().view(torch.float16) for h in host]
+    buf = Guarded(lay.bucket_padded[0], torch.float16)
+    Z.zero_flatten_bucket(lay, 0, dev, buf.t)
+    torch.cuda.synchronize()
+    buf.check()
+    assert np.array_equal(host_u16(buf.t), oracle.flatten_bucket(olay, 0, host))
+
+
+def test_allgather_more_than_64_ranks():
+    rng = np.random.Generator(np.random.PCG64(14))
+    world, part = 100, 1031
+    host = [rng.integers(0, 2 ** 16, part + 5, dtype=np.uint64).astype(np.uint16) for _ in range(world)]
+    dev = [torch.from_numpy(h.view(np.int16).copy()).cuda().view(torch.bfloat16) for h in host]
+    dst = Guarded(world * part, torch.bfloat16)
+    Z.zero_allgather_params(dev, 5, part, dst.t)
+    torch.cuda.synchronize()
+    dst.check()
+    assert np.array_equal(host_u16(dst.t), oracle.allgather(host, 5, part))
+
+
+def test_step_with_128_replicas():
+    c = Case(128 * 1001, 128, seed=15)
+    c.run(_adam())
+    ref, _, _ = c.expect(_adam())
+    assert c.compare(ref) == [0, 0, 0, 0]

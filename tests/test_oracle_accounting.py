@@ -16,7 +16,8 @@ import pytest
 import oracle
 import workloads
 
-GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "zero_explainer_figures.json")))
+with open(os.path.join(os.path.dirname(__file__), "golden", "zero_explainer_figures.json")) as _f:
+    GOLD = json.load(_f)
 
 
 @pytest.mark.parametrize("N", [1, 2, 4, 8, 16, 64])

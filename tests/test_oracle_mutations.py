@@ -87,7 +87,8 @@ def _build_mutant(src_text: str, workdir: str) -> str:
 
 @pytest.mark.parametrize("name,find,repl", MUTANTS, ids=[m[0] for m in MUTANTS])
 def test_every_mutant_is_caught(name, find, repl):
-    text = open(SRC).read()
+    with open(SRC) as f:
+        text = f.read()
     assert find in text, f"mutation target not found: {find!r}"
     mutated = text.replace(find, repl)
     with tempfile.TemporaryDirectory() as d:

@@ -16,6 +16,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <mutex>
 #include <vector>
 
 #include "common.h"
@@ -81,15 +82,24 @@ __global__ void __launch_bounds__(kThreads) copy_segments_kernel(const __grid_co
     for (; i < nvec; i += nt) __stcs(d4 + i, __ldcs(s4 + i));
 }
 
-int g_sms_cached = 0;
+std::mutex g_sms_mu;
+int g_sms[64] = {};
+
+// SM count of the current device, queried once per device.
+int device_sms(const char* fn, int* sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return fail(ZERO_ERR_CUDA, "%s: cannot query the device", fn);
+    std::lock_guard<std::mutex> lk(g_sms_mu);
+    if (g_sms[dev] == 0 && cudaDeviceGetAttribute(&g_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return fail(ZERO_ERR_CUDA, "%s: cannot query the SM count", fn);
+    *sms = g_sms[dev];
+    return ZERO_OK;
+}
 
 int launch_segments(const std::vector<Seg>& segs, int esize, cudaStream_t stream, const char* fn) {
-    if (g_sms_cached == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&g_sms_cached, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return fail(ZERO_ERR_CUDA, "%s: cannot query the device", fn);
-    }
+    int sms = 0;
+    if (int rc = device_sms(fn, &sms)) return rc;
     for (size_t first = 0; first < segs.size(); first += kMaxSegs) {
         const size_t n = std::min<size_t>(kMaxSegs, segs.size() - first);
         CopyParams prm{};
@@ -103,7 +113,7 @@ int launch_segments(const std::vector<Seg>& segs, int esize, cudaStream_t stream
         // enough blocks to cover the largest segment with kUnroll 16-byte
         // accesses per thread, at most ~8 resident blocks per SM in total
         int64_t want = (max_bytes + int64_t(kThreads) * 16 * kUnroll - 1) / (int64_t(kThreads) * 16 * kUnroll);
-        int64_t cap = std::max<int64_t>(1, int64_t(g_sms_cached) * 8 / int64_t(n));
+        int64_t cap = std::max<int64_t>(1, int64_t(sms) * 8 / int64_t(n));
         const unsigned int gx = static_cast<unsigned int>(std::max<int64_t>(1, std::min(want, cap)));
         copy_segments_kernel<<<dim3(gx, static_cast<unsigned int>(n)), kThreads, 0, stream>>>(prm);
         cudaError_t e = cudaGetLastError();

@@ -152,7 +152,8 @@ int zero_loss_scale_update(float* scale, int32_t* good_steps, int32_t overflow,
         *scale = half < min_scale ? min_scale : half;
         *good_steps = 0;
     } else if (++*good_steps >= growth_interval) {
-        *scale = *scale * 2.0f;
+        const float twice = *scale * 2.0f;
+        if (std::isfinite(twice)) *scale = twice;   // the scale never grows to inf
         *good_steps = 0;
     }
     return zero::ok();
