@@ -9,6 +9,7 @@
 import ctypes
 import os
 import re
+import subprocess
 
 import numpy as np
 import pytest
@@ -183,3 +184,37 @@ def test_loss_scale_growth_stops_below_inf():
     s, g = Z.zero_loss_scale_update(big, 0, False, growth_interval=1)
     so, go = oracle.loss_scale_update(big, 0, False, growth_interval=1)
     assert (s, g) == (so, go) == (big, 0)
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include "zero.h"
+int main(void) {
+    int64_t numels[3] = {5, 7, 11};
+    zero_layout_t L = {0};
+    if (zero_partition_layout(numels, 3, 4, 10, 1, &L) != ZERO_OK) return 1;
+    printf("%lld %lld %lld\n", (long long)L.n_buckets, (long long)L.bucket_padded[0], (long long)L.bucket_padded[1]);
+    zero_layout_free(&L);
+    float scale = 8.0f; int32_t good = 0;
+    if (zero_loss_scale_update(&scale, &good, 1, 1000, 1.0f) != ZERO_OK || scale != 4.0f) return 2;
+    if (zero_reduce_scatter_adam_step(NULL, 2, 64, ZERO_ALL_PARTITIONS, ZERO_F16, NULL, NULL, NULL, NULL, NULL,
+                                      NULL, NULL, ZERO_F16, NULL, 1.0f, NULL, NULL, NULL, NULL) != ZERO_ERR_ARG) return 3;
+    printf("%s|%s\n", zero_strerror(ZERO_ERR_ARG), zero_last_error());
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    src = tmp_path / "use_zero.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "use_zero"
+    inc = os.path.join(os.path.dirname(HEADER))
+    libdir = os.path.dirname(Z.LIB_PATH)
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-I", inc, str(src), "-o", str(exe),
+                           "-L", libdir, "-lzero", f"-Wl,-rpath,{libdir}"])
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    lines = out.stdout.splitlines()
+    assert lines[0] == "3 8 8"          # buckets [5], [7], [11] padded to multiples of 4
+    assert lines[1].startswith("invalid argument|zero_reduce_scatter_adam_step")

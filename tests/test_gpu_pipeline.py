@@ -102,3 +102,17 @@ def test_pipeline_deterministic():
     for o in outs[1:]:
         for a, b in zip(outs[0], o):
             assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+
+
+def test_pipeline_single_partition_with_head():
+    # P = 4 (mod 8): rank r's gradient slice starts 8 bytes off the 16-byte
+    # phase for odd r, the state arrays at phase 0; the common phase is
+    # element 4, so the pipeline kernel runs with a 4-element scalar head
+    world = 4
+    T = _tile(world)
+    P = 2 * SMS * T + 8 * 100 + 4
+    for r in (1, 2):
+        c = Case(world * P, world, seed=370 + r, partition=r)
+        ref, _, _ = c.expect(_adam())
+        c.run(_adam())
+        assert c.compare(ref) == [0, 0, 0, 0]
