@@ -257,3 +257,30 @@ def test_checkpoint_resume_bit_identical(mode):
     for b in range(L.n_buckets):
         for x, y in zip(opt.state(b), opt2.state(b)):
             assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
+
+
+def _stats_tile(world):
+    return min(8192, (180 * 1024 // (2 * 2 * world)) // 512 * 512)
+
+
+@pytest.mark.parametrize("world,dtype,goff", [(8, oracle.F16, 0), (8, oracle.F16, 3), (16, oracle.BF16, 0),
+                                              (1, oracle.F16, 5), (3, oracle.BF16, 1)])
+def test_stats_pipeline(world, dtype, goff):
+    """Sizes that give every SM at least two tiles: the statistics pipeline
+    kernel runs, with ragged tails and (goff > 0) a scalar head."""
+    T = _stats_tile(world)
+    per_rank = (2 * 148 * T + 777) // world + 3
+    c = Case(world * per_rank, world, gdtype=dtype, pdtype=dtype, seed=460 + world, goff=goff, scale=65536.0)
+    flag, norm = _stats(c)
+    ovf, sq, _, _ = _oracle_stats(c)
+    assert flag == ovf == 0 and abs(norm - sq) <= _norm_tol(c.n) * sq
+    n = c.n
+    for pos, is_inf in [(np.array([n // 3]), np.array([True])), (np.array([n - 2]), np.array([False])),
+                        (np.array([1]), np.array([False]))]:
+        g = c.G[world - 1].copy()
+        workloads.inject(c.G[world - 1], pos, is_inf, dtype)
+        to_dev_u16(c.G[world - 1], TD[dtype], buf=c.g_dev[world - 1])
+        flag, _ = _stats(c)
+        assert flag == 1 == _oracle_stats(c)[0]
+        c.G[world - 1] = g
+        to_dev_u16(g, TD[dtype], buf=c.g_dev[world - 1])

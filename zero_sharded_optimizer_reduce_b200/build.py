@@ -22,7 +22,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libzero.so")
 
 SOURCES = ["step.cu", "step_static.cu", "stats.cu", "selftest.cu", "copy.cu", "host.cpp", "ipc.cpp"]
-HEADERS = [os.path.join(CSRC, n) for n in ("common.h", "fused_step.cuh", "step_launch.h")] + [os.path.join(INCLUDE, "zero.h")]
+HEADERS = [os.path.join(CSRC, n) for n in ("common.h", "fused_step.cuh", "grad_stats.cuh", "step_launch.h")] + [os.path.join(INCLUDE, "zero.h")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

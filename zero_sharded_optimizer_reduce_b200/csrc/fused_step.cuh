@@ -311,67 +311,6 @@ __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_const
     finish_block<kThreads>(p, bad, sq);
 }
 
-// Statistics pre-pass: the rank-order fp32 sum of the N replicas, the
-// overflow test and, when p.sqnorm is set, the squared norm of the unscaled
-// gradient g = s * inv, without reading or writing any optimizer state.
-// 2N bytes per element.  Lets a caller decide skip and clipping for a whole
-// step before any state is written (in-place update with an exact skip).
-template <typename GT>
-__global__ void __launch_bounds__(kThreads) grad_stats_kernel(const __grid_constant__ StepParams p) {
-    const int64_t tid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
-    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
-    const int world = p.world;
-    const float inv = p.c.inv;
-    const bool want_sq = p.sqnorm != nullptr;
-    bool bad = false;
-    double sq = 0.0;
-    for (int64_t vi = tid; vi < p.nvec; vi += nthreads) {
-        const int64_t e0 = p.head + vi * kVec;
-        float s[kVec];
-        {
-            uint4 r[kBatch];
-#pragma unroll
-            for (int b = 0; b < kBatch; ++b)
-                if (b < world) r[b] = ld_grad16(static_cast<const uint16_t*>(p.grads[b]) + e0);
-            cvt8<GT>(r[0], s);
-#pragma unroll
-            for (int b = 1; b < kBatch; ++b)
-                if (b < world) add8<GT>(r[b], s);
-        }
-        for (int k0 = kBatch; k0 < world; k0 += kBatch) {
-            uint4 r[kBatch];
-#pragma unroll
-            for (int b = 0; b < kBatch; ++b)
-                if (k0 + b < world) r[b] = ld_grad16(static_cast<const uint16_t*>(p.grads[k0 + b]) + e0);
-#pragma unroll
-            for (int b = 0; b < kBatch; ++b)
-                if (k0 + b < world) add8<GT>(r[b], s);
-        }
-#pragma unroll
-        for (int e = 0; e < kVec; ++e) {
-            bad |= !isfinite(s[e]);
-            if (want_sq) {
-                const float g = __fmul_rn(s[e], inv);
-                sq = fma(static_cast<double>(g), static_cast<double>(g), sq);
-            }
-        }
-    }
-    const int64_t vec_end = p.head + p.nvec * kVec;
-    const int64_t nscalar = p.head + (p.count - vec_end);
-    for (int64_t q = tid; q < nscalar; q += nthreads) {
-        const int64_t e = q < p.head ? q : vec_end + (q - p.head);
-        float s = Fmt<GT>::one(static_cast<const uint16_t*>(p.grads[0])[e]);
-        for (int k = 1; k < world; ++k)
-            s = __fadd_rn(s, Fmt<GT>::one(static_cast<const uint16_t*>(p.grads[k])[e]));
-        bad |= !isfinite(s);
-        if (want_sq) {
-            const float g = __fmul_rn(s, inv);
-            sq = fma(static_cast<double>(g), static_cast<double>(g), sq);
-        }
-    }
-    finish_block<kThreads>(p, bad, sq);
-}
-
 // ------------------------------------------------------- bulk-copy pipeline
 
 // (the pipeline's helpers follow; wait_timeout_kernel below exercises the

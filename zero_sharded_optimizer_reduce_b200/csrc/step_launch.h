@@ -4,6 +4,7 @@
 #pragma once
 
 #include "fused_step.cuh"
+#include "grad_stats.cuh"
 
 namespace zero {
 namespace fused {
@@ -25,6 +26,10 @@ inline KernelFn pick_kernel(zero_dtype_t g, zero_dtype_t pd) {
 
 inline KernelFn pick_stats_kernel(zero_dtype_t g) {
     return g == ZERO_F16 ? grad_stats_kernel<__half> : grad_stats_kernel<__nv_bfloat16>;
+}
+
+inline KernelFn pick_stats_pipe_kernel(zero_dtype_t g) {
+    return g == ZERO_F16 ? grad_stats_pipe_kernel<__half> : grad_stats_pipe_kernel<__nv_bfloat16>;
 }
 
 inline KernelFn pick_pipe_kernel(zero_dtype_t g, zero_dtype_t pd) {
@@ -50,6 +55,21 @@ inline int pipe_tile(int world) {
     return static_cast<int>(t);
 }
 
+// Tile of the statistics pipeline (stages hold gradients only, 2N bytes per
+// element): the same rule as pipe_tile.
+inline int stats_pipe_tile(int world) {
+    if (world > kPipeMaxWorld) return 0;
+    const uint32_t per_elem = 2u * static_cast<uint32_t>(world);
+    uint32_t t = kPipeSmemTarget / (static_cast<uint32_t>(kPipeStages) * per_elem) / 512u * 512u;
+    if (t > 8192u) t = 8192u;
+    if (t < kPipeMinTile) return 0;
+    return static_cast<int>(t);
+}
+
+inline uint32_t stats_pipe_smem_bytes(int world, int tile) {
+    return static_cast<uint32_t>(kPipeStages) * static_cast<uint32_t>(tile) * 2u * static_cast<uint32_t>(world);
+}
+
 inline uint32_t pipe_smem_bytes(int world, int tile) {
     return static_cast<uint32_t>(kPipeStages) * static_cast<uint32_t>(tile) * (2u * static_cast<uint32_t>(world) + 12u);
 }
@@ -59,6 +79,7 @@ struct DeviceInfo {
     int blocks_per_sm[4] = {0, 0, 0, 0};
     int stats_blocks_per_sm[2] = {0, 0};
     bool pipe_ready[4] = {false, false, false, false};
+    bool stats_pipe_ready[2] = {false, false};
 };
 
 std::mutex g_dev_mu;
@@ -283,6 +304,22 @@ inline int prepare_step(const char* fn, const void* const* grad_bufs, int32_t wo
     return ZERO_OK;
 }
 
+// SM count, and the statistics pipeline kernel's shared-memory limit.
+inline int stats_pipe_setup(zero_dtype_t g, int* sms) {
+    const int which = static_cast<int>(g);
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo* d = nullptr;
+    if (int rc = device_info(&d)) return rc;
+    if (!d->stats_pipe_ready[which]) {
+        cudaError_t e = cudaFuncSetAttribute(pick_stats_pipe_kernel(g), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kPipeSmemMax));
+        if (e != cudaSuccess) return fail(ZERO_ERR_CUDA, "cannot raise the shared-memory limit: %s", cudaGetErrorString(e));
+        d->stats_pipe_ready[which] = true;
+    }
+    *sms = d->sms;
+    return ZERO_OK;
+}
+
 // Validate a statistics call and build its kernel parameters (the state
 // pointers stay NULL: the statistics kernel reads gradients only).
 inline int prepare_stats(const char* fn, const void* const* grad_bufs, int32_t world, int64_t padded_numel,
@@ -346,12 +383,27 @@ inline int prepare_stats(const char* fn, const void* const* grad_bufs, int32_t w
         prm.head = h;
         prm.nvec = (count - h) / kVec;
     }
-    int limit = 0;
-    if (int rc = stats_grid_limit(grad_dtype, &limit)) return rc;
-    const int64_t work = prm.nvec > 0 ? prm.nvec : count;
-    int64_t blocks = (work + kThreads - 1) / kThreads;
-    if (blocks > limit) blocks = limit;
-    if (blocks < 1) blocks = 1;
+    prm.tile = 0;
+    int64_t blocks = 0;
+    const int tile = h >= 0 ? stats_pipe_tile(world) : 0;
+    if (tile > 0) {
+        int sms = 0;
+        if (int rc = stats_pipe_setup(grad_dtype, &sms)) return rc;
+        const int64_t ntiles = (count - h) / tile;
+        if (ntiles >= 2 * static_cast<int64_t>(sms)) {
+            prm.tile = tile;
+            prm.nvec = ntiles * tile / kVec;
+            blocks = sms;
+        }
+    }
+    if (prm.tile == 0) {
+        int limit = 0;
+        if (int rc = stats_grid_limit(grad_dtype, &limit)) return rc;
+        const int64_t work = prm.nvec > 0 ? prm.nvec : count;
+        blocks = (work + kThreads - 1) / kThreads;
+        if (blocks > limit) blocks = limit;
+        if (blocks < 1) blocks = 1;
+    }
     *prm_out = prm;
     *blocks_out = blocks;
     return ZERO_OK;
@@ -360,8 +412,13 @@ inline int prepare_stats(const char* fn, const void* const* grad_bufs, int32_t w
 inline int launch_stats(const char* fn, const StepParams& prm, int64_t blocks, zero_dtype_t grad_dtype,
                         zero_stream_t stream) {
     if (blocks == 0) return ok();
-    pick_stats_kernel(grad_dtype)<<<static_cast<unsigned int>(blocks), kThreads, 0,
-                                    reinterpret_cast<cudaStream_t>(stream)>>>(prm);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (prm.tile > 0) {
+        pick_stats_pipe_kernel(grad_dtype)<<<static_cast<unsigned int>(blocks), kPipeThreads,
+                                             stats_pipe_smem_bytes(prm.world, prm.tile), s>>>(prm);
+    } else {
+        pick_stats_kernel(grad_dtype)<<<static_cast<unsigned int>(blocks), kThreads, 0, s>>>(prm);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(ZERO_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
     return ok();
