@@ -284,3 +284,22 @@ def test_stats_pipeline(world, dtype, goff):
         assert flag == 1 == _oracle_stats(c)[0]
         c.G[world - 1] = g
         to_dev_u16(g, TD[dtype], buf=c.g_dev[world - 1])
+
+
+@pytest.mark.parametrize("mode", ["banks", "inplace"])
+def test_step_from_host_matches_device_step(mode):
+    """The end-to-end entry (pinned host gradients, per-bucket copy stream)
+    gives the same bits as writing the gradients on the device first."""
+    numels = [700_001, 3, 900_000]
+    N = 4
+    adam = workloads.AdamConfig(weight_decay=0.01)
+    L, a, _ = _opt_and_oracle(numels, N, 800_000, adam, mode)
+    _, b, _ = _opt_and_oracle(numels, N, 800_000, adam, mode)
+    for step in range(1, 4):
+        G = _grads_for(L, N, step, 65536.0)
+        host = [[torch.from_numpy(g.view(np.int16)).view(torch.float16).pin_memory() for g in per] for per in G]
+        _upload(a, G)
+        assert a.step() and b.step_from_host(host)
+    for bk in range(L.n_buckets):
+        for x, y in zip(a.state(bk), b.state(bk)):
+            assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))

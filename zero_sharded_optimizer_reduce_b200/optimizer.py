@@ -109,24 +109,28 @@ class ZeroAdam:
         return self.grads[b]
 
     # -------------------------------------------------------------------- step
-    def launch(self, stream=None, on_launch=None) -> None:
+    def launch(self, stream=None, on_launch=None, before_bucket=None) -> None:
         """Enqueue the fused kernel over every bucket (no host synchronization).
 
         `on_launch(bucket, phase)` is called with phase "before" / "after"
-        around each kernel launch (used to record timing events).
+        around each kernel launch (used to record timing events);
+        `before_bucket(bucket)` runs before bucket b's first kernel is
+        enqueued (used to make the stream wait for that bucket's inputs).
         """
         if stream is not None:
             with torch.cuda.stream(stream):
-                return self.launch(None, on_launch)
+                return self.launch(None, on_launch, before_bucket)
         self.flags.zero_()
         if self.sqnorm is not None:
             self.sqnorm.zero_()
         hp = hparams(self.lr, self.betas[0], self.betas[1], self.eps, self.weight_decay,
                      self.t + 1, self.grad_divisor)
         if self.two_pass:
-            return self._launch_two_pass(hp, on_launch)
+            return self._launch_two_pass(hp, on_launch, before_bucket)
         c, n = self.cur, self.cur ^ 1
         for b in range(self.layout.n_buckets):
+            if before_bucket is not None:
+                before_bucket(b)
             if on_launch is not None:
                 on_launch(b, "before")
             zero_reduce_scatter_adam_step(
@@ -137,10 +141,12 @@ class ZeroAdam:
             if on_launch is not None:
                 on_launch(b, "after")
 
-    def _launch_two_pass(self, hp, on_launch) -> None:
+    def _launch_two_pass(self, hp, on_launch, before_bucket=None) -> None:
         """Statistics over every bucket, then the gated (and clipped) update."""
         L = self.layout
         for b in range(L.n_buckets):
+            if before_bucket is not None:
+                before_bucket(b)
             zero_grad_stats(self.grads[b], L.bucket_padded[b], ZERO_ALL_PARTITIONS, self.scale, self.flag,
                             self.sqnorm, self.workspace, self.grad_divisor)
         c = self.cur
@@ -184,12 +190,27 @@ class ZeroAdam:
         return self.commit(stream)
 
     def step_from_host(self, host_grads, stream=None) -> bool:
-        """Copy host gradients (host_grads[b][k], pinned) in, then step."""
-        with torch.cuda.stream(stream if stream is not None else torch.cuda.current_stream()):
+        """Copy host gradients (host_grads[b][k], pinned) in, then step.
+
+        The copies run bucket by bucket on a separate copy stream; bucket b's
+        kernel waits only for bucket b's copies, so it overlaps the copies of
+        the buckets after it."""
+        main = stream if stream is not None else torch.cuda.current_stream()
+        if not hasattr(self, "_copy_stream"):
+            self._copy_stream = torch.cuda.Stream(device=self.device)
+        cs = self._copy_stream
+        cs.wait_stream(main)           # the previous step's kernels are done reading the buffers
+        ready = []
+        with torch.cuda.stream(cs):
             for b in range(self.layout.n_buckets):
                 for k in range(self.world):
                     self.grads[b][k].copy_(host_grads[b][k], non_blocking=True)
-            return self.step()
+                ev = torch.cuda.Event()
+                ev.record(cs)
+                ready.append(ev)
+        with torch.cuda.stream(main):
+            self.launch(before_bucket=lambda b: main.wait_event(ready[b]))
+            return self.commit()
 
     # -------------------------------------------------------------- checkpoint
     def state_dict(self) -> dict:
