@@ -1,5 +1,7 @@
-// Device code of the fused ZeRO-2 step kernel and the host helpers that
-// size its grid; included by every translation unit that launches it.
+// Device code of the fused ZeRO-2 step: the register-streaming and the
+// shared-memory pipeline kernels, the device helpers they share with the
+// statistics kernels, and the bounded-wait self-test kernel.  Host-side
+// validation, kernel choice and launch live in step_launch.h.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -8,7 +10,6 @@
 
 #include <cmath>
 #include <cstdint>
-#include <mutex>
 
 #include "common.h"
 

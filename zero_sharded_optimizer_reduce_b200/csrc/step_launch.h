@@ -3,6 +3,8 @@
 // kernels of fused_step.cuh.
 #pragma once
 
+#include <mutex>
+
 #include "fused_step.cuh"
 #include "grad_stats.cuh"
 
