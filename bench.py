@@ -459,6 +459,18 @@ def run_stage3(args):
         e1.record()
         torch.cuda.synchronize()
         out[prefetch] = e0.elapsed_time(e1) / args.steps
+        if prefetch:
+            # the all-gather alone: unit 0 from the 8 shards into a layer buffer
+            for _ in range(3):
+                s3.unit_params(0, s3.layer[0][:s3.layout.bucket_padded[0]])
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(20):
+                s3.unit_params(0, s3.layer[0][:s3.layout.bucket_padded[0]])
+            e1.record()
+            torch.cuda.synchronize()
+            gather_ms = e0.elapsed_time(e1) / 20
+            gather_elems = s3.layout.bucket_padded[0]
         del s3
         torch.cuda.empty_cache()
     psi = sum(Z.zero_partition_layout(w.numels, w.world, 1, 8).bucket_padded)
@@ -470,7 +482,11 @@ def run_stage3(args):
             "prefetch_gain": out[False] / out[True] - 1.0, "steps": args.steps, "warmup": args.warmup,
             "config": {"workload": w.name, "psi_padded": psi, "world": N, "units": len(w.numels)},
             "hbm_gbs": step_bytes / (out[True] * 1e-3) / 1e9, "bytes_per_elem": 8 + 4 * N + 26,
-            "frac_measured": step_bytes / (out[True] * 1e-3) / 1e9 / peak, "peak_kind": peak_kind}
+            "frac_measured": step_bytes / (out[True] * 1e-3) / 1e9 / peak, "peak_kind": peak_kind,
+            "allgather": {"elements": gather_elems, "ms": gather_ms, "bytes_per_elem": 4,
+                          "gbs": gather_elems * 4 / (gather_ms * 1e-3) / 1e9,
+                          "frac_measured": gather_elems * 4 / (gather_ms * 1e-3) / 1e9 / peak,
+                          "note": "2 B read + 2 B write per element; one unit (201M elements) from 8 shards"}}
     print(json.dumps(line), flush=True)
     return 0
 

@@ -251,8 +251,12 @@ def test_stage3_layerwise_6p7b(dtype):
 
 
 @pytest.mark.parametrize("psi,world,dtype", [(1 << 20, 64, oracle.F16), (16 << 20, 16, oracle.BF16),
-                                             (256 << 20, 8, oracle.F16), (256 << 20, 2, oracle.BF16)])
+                                             (256 << 20, 8, oracle.F16), (256 << 20, 2, oracle.BF16),
+                                             (1 << 30, 16, oracle.BF16), (2 << 30, 4, oracle.F16)])
 def test_sweep_points_windows(psi, world, dtype):
+    need = psi * (2 * world + 30) / 1e9 + 2
+    if _free_gb() < need:
+        pytest.skip(f"needs {need:.0f} GB of HBM")
     tdt = TD[dtype]
     grads = [torch.empty(psi, dtype=tdt, device="cuda") for _ in range(world)]
     for k in range(world):
