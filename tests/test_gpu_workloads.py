@@ -32,6 +32,7 @@ TD = {oracle.F16: torch.float16, oracle.BF16: torch.bfloat16}
 
 
 def _free_gb():
+    torch.cuda.empty_cache()          # blocks cached by earlier tests count as free
     free, _ = torch.cuda.mem_get_info()
     return free / 1e9
 

@@ -1,0 +1,44 @@
+"""Property-based tests (hypothesis, derandomized): random layouts through
+the C ABI against the oracle on the CPU, and random small configurations of
+the fused step on the GPU against the oracle, bit for bit."""
+import numpy as np
+import pytest
+import torch
+from hypothesis import given, settings
+from hypothesis import strategies as st
+
+import oracle
+import workloads
+import zero_sharded_optimizer_reduce_b200 as Z
+
+
+@settings(max_examples=300, deadline=None, derandomize=True)
+@given(numels=st.lists(st.integers(0, 10_000), max_size=40), world=st.integers(1, 128),
+       cap=st.integers(0, 50_000), align=st.integers(1, 16))
+def test_layout_matches_oracle(numels, world, cap, align):
+    a = Z.zero_partition_layout(numels, world, cap, align)
+    b = oracle.partition_layout(numels, world, cap, align)
+    assert list(a.bucket_numel) == b.bucket_numel and list(a.bucket_padded) == b.bucket_padded
+    assert list(a.bucket_offset) == b.bucket_offset
+    assert list(a.tensor_bucket) == b.tensor_bucket and list(a.tensor_offset) == b.tensor_offset
+
+
+@pytest.mark.gpu
+@settings(max_examples=40, deadline=None, derandomize=True)
+@given(world=st.integers(1, 17), per_rank=st.integers(1, 5000),
+       dtypes=st.sampled_from([(oracle.F16, oracle.F16), (oracle.BF16, oracle.BF16), (oracle.F16, oracle.BF16),
+                               (oracle.BF16, oracle.F16)]),
+       offs=st.tuples(st.integers(0, 7), st.integers(0, 7), st.integers(0, 7)),
+       part=st.integers(-1, 16), inplace=st.booleans(), wd=st.sampled_from([0.0, 0.01, 0.1]),
+       t=st.integers(1, 50), seed=st.integers(0, 10_000))
+def test_step_matches_oracle(world, per_rank, dtypes, offs, part, inplace, wd, t, seed):
+    from test_gpu_step import Case
+    gd, pd = dtypes
+    partition = part if part < world else -1
+    c = Case(world * per_rank, world, gdtype=gd, pdtype=pd, seed=seed, partition=partition, goff=offs[0],
+             soff=offs[1], poff=offs[2], inplace=inplace)
+    adam = workloads.AdamConfig(weight_decay=wd)
+    ref, ovf, _ = c.expect(adam, t=t)
+    c.run(adam, t=t)
+    assert int(c.flag.item()) == ovf == 0
+    assert c.compare(ref) == [0, 0, 0, 0]
