@@ -318,7 +318,9 @@ def run_gpu(args):
     for b, es in ev.items():
         for i in range(0, len(es), 2):
             launch_ms.append(es[i].elapsed_time(es[i + 1]))
-            launch_elems.append(L.bucket_padded[b])
+            # b = -1: the runner's whole step (every bucket's kernel, the flag
+            # clear and its 4-byte read-back) between one pair of events
+            launch_elems.append(psi_p if b < 0 else L.bucket_padded[b])
     ms = max_over_ranks(ms, "cuda")
     ms_per_step = ms / args.steps
     value = whole_job_gparams(psi_p, world_gpus, ms_per_step)
@@ -357,9 +359,13 @@ def run_gpu(args):
                 "hbm_gbs": value * 1e9 * bpe / world_gpus / 1e9,
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
                              "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
-                             "kernel": "fused_step (shared-memory pipeline kernel for aligned calls of >= 2 tiles per SM)",
+                             "kernel": ("fused_step (shared-memory pipeline kernel for aligned calls of >= 2 tiles per SM); "
+                                        "timed per step over all buckets" if -1 in ev else
+                                        "fused_step (shared-memory pipeline kernel for aligned calls of >= 2 tiles per SM)"),
                              "bytes_per_elem": bpe,
-                             "elems_per_launch": avg_elems, "launches_timed": len(launch_ms)},
+                             "elems_per_launch": avg_elems, "launches_timed": len(launch_ms),
+                             "timed_unit": ("one step: all buckets' kernels + flag clear + 4-byte read-back"
+                                            if -1 in ev else "one bucket's kernel")},
                 "gpu_launches": args.steps * L.n_buckets * (2 if opt.two_pass else 1),
                 "applied_steps": applied,
                 "clocks": clock,
@@ -528,7 +534,7 @@ def run_e2e(opt, args, stream, barrier, world_gpus):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=3)

@@ -373,6 +373,67 @@ int zero_allgather_params(const void* const* shards, int32_t world, int64_t shar
 int zero_test_wait_timeout(int32_t* status, int64_t limit_ns, zero_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Step runner: the whole step over every bucket                             */
+/* ------------------------------------------------------------------------ */
+
+/* One bucket as the runner sees it; every pointer is caller-owned device
+ * memory.  Bank b of the states is master[b], m[b], v[b] (fp32, padded_numel
+ * elements each) and params[b] (param dtype). */
+typedef struct {
+    int64_t padded_numel;           /* multiple of world */
+    const void* const* grad_bufs;   /* host array of `world` device pointers; copied by create */
+    float* master[2];
+    float* m[2];
+    float* v[2];
+    void* params[2];
+} zero_bucket_banks_t;
+
+typedef struct zero_runner zero_runner_t;   /* opaque, host memory */
+
+/*
+ * zero_runner_create / _launch / _commit / _state / _set_state / _destroy -
+ * the ZeRO-2 step over a list of buckets with an exact skip.
+ *
+ * Source: ZeRO explainer, "Stage 2 - Gradient Partitioning (P_os+g)" (every
+ * bucket's reduce-scatter + update of the partitions) and "Constant-size
+ * buffers" (the buckets); the skip on overflow and the dynamic loss scale are
+ * not on the pages (zero_loss_scale_update).
+ *
+ * zero_runner_launch enqueues on `stream`, without waiting: clear
+ * *flag_dev (and *grad_sqnorm), the fused step over every bucket reading bank
+ * `cur` and writing bank `cur ^ 1` with hyper-parameters hp (step = t + 1)
+ * and the current loss scale, and a copy of *flag_dev into *flag_host.
+ * zero_runner_commit waits for the stream, reads *flag_host and, when it is
+ * 0, makes bank `cur ^ 1` current and advances t; it then applies
+ * zero_loss_scale_update and reports *applied (1 = update applied).  A launch
+ * must be followed by a commit before the next launch.
+ *
+ * create: buckets[n_buckets] (copied; the pointer arrays too), world 1 ..
+ *   ZERO_MAX_WORLD, dtypes and hp as for zero_reduce_scatter_adam_step
+ *   (hp->step is the t of the first update), loss_scale > 0, growth_interval
+ *   >= 1, min_scale > 0; flag_dev device int32; flag_host host int32 (pinned,
+ *   e.g. cudaHostAlloc); grad_sqnorm device double or NULL (with workspace as
+ *   for zero_reduce_scatter_adam_step).  Every bucket is validated for both
+ *   bank directions.  Allocates only the host-side runner object.
+ * state / set_state: t (applied updates), loss scale, good-step count and the
+ *   current bank, to read or to restore (e.g. from a checkpoint).
+ * Errors: those of zero_reduce_scatter_adam_step; ZERO_ERR_ARG for a launch
+ * without commit or a commit without launch; ZERO_ERR_CUDA from commit when
+ * the kernel reported a pipeline timeout (flag bit 1): nothing is committed.
+ */
+int zero_runner_create(const zero_bucket_banks_t* buckets, int64_t n_buckets, int32_t world,
+                       zero_dtype_t grad_dtype, zero_dtype_t param_dtype, const zero_adam_hparams_t* hp,
+                       float loss_scale, int32_t growth_interval, float min_scale,
+                       int32_t* flag_dev, int32_t* flag_host, double* grad_sqnorm, void* workspace,
+                       zero_runner_t** out);
+int zero_runner_launch(zero_runner_t* runner, zero_stream_t stream);
+int zero_runner_commit(zero_runner_t* runner, zero_stream_t stream, int32_t* applied);
+int zero_runner_state(const zero_runner_t* runner, int64_t* t, float* loss_scale, int32_t* good_steps,
+                      int32_t* bank);
+int zero_runner_set_state(zero_runner_t* runner, int64_t t, float loss_scale, int32_t good_steps, int32_t bank);
+void zero_runner_destroy(zero_runner_t* runner);
+
+/* ------------------------------------------------------------------------ */
 /* Multi-process ranks: sharing gradient and parameter buffers               */
 /* ------------------------------------------------------------------------ */
 

@@ -303,3 +303,36 @@ def test_step_from_host_matches_device_step(mode):
     for bk in range(L.n_buckets):
         for x, y in zip(a.state(bk), b.state(bk)):
             assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
+
+
+def test_runner_protocol_and_state():
+    """The native runner: launch/commit alternate, state round-trips, and a
+    step through it equals a step through the per-bucket calls."""
+    numels = [500_000, 11]
+    N = 4
+    adam = workloads.AdamConfig(weight_decay=0.01)
+    L, a, _ = _opt_and_oracle(numels, N, 0, adam, "banks")
+    assert a._runner is not None
+    G = _grads_for(L, N, 1, 65536.0)
+    _upload(a, G)
+    r = a._runner
+    r.launch()
+    with pytest.raises(Z.ZeroError):
+        r.launch()                      # the launched step is not committed yet
+    assert r.commit() is True
+    with pytest.raises(Z.ZeroError):
+        r.commit()                      # nothing launched
+    t, scale, good, bank = r.state()
+    assert (t, scale, good, bank) == (1, 65536.0, 1, 1)
+    r.set_state(t, scale, good, bank)
+    with pytest.raises(Z.ZeroError):
+        r.set_state(1, -1.0, 0, 0)
+    # the same step through the per-bucket Python path on a fresh optimizer
+    _, b, _ = _opt_and_oracle(numels, N, 0, adam, "banks")
+    _upload(b, G)
+    b.launch()
+    assert b.commit()
+    for bk in range(L.n_buckets):
+        a_state = [x.clone() for x in (a.master[bk][bank], a.m[bk][bank], a.v[bk][bank], a.params_bank[bk][bank])]
+        for x, y in zip(a_state, b.state(bk)):
+            assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))

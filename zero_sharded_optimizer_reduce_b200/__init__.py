@@ -58,6 +58,12 @@ class DevicePtr:
         return self.ptr
 
 
+class BucketBanks(ctypes.Structure):
+    _fields_ = [("padded_numel", ctypes.c_int64), ("grad_bufs", ctypes.POINTER(ctypes.c_void_p)),
+                ("master", ctypes.c_void_p * 2), ("m", ctypes.c_void_p * 2), ("v", ctypes.c_void_p * 2),
+                ("params", ctypes.c_void_p * 2)]
+
+
 class AdamHParams(ctypes.Structure):
     _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
                 ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float),
@@ -104,6 +110,21 @@ def _load():
     L.zero_ipc_import.restype = ctypes.c_int
     L.zero_ipc_close.argtypes = [vp]
     L.zero_ipc_close.restype = ctypes.c_int
+    L.zero_runner_create.argtypes = [ctypes.POINTER(BucketBanks), i64, i32, ctypes.c_int, ctypes.c_int,
+                                     ctypes.POINTER(AdamHParams), f32, i32, f32, vp, vp, vp, vp,
+                                     ctypes.POINTER(vp)]
+    L.zero_runner_create.restype = ctypes.c_int
+    L.zero_runner_launch.argtypes = [vp, vp]
+    L.zero_runner_launch.restype = ctypes.c_int
+    L.zero_runner_commit.argtypes = [vp, vp, ctypes.POINTER(i32)]
+    L.zero_runner_commit.restype = ctypes.c_int
+    L.zero_runner_state.argtypes = [vp, ctypes.POINTER(i64), ctypes.POINTER(f32), ctypes.POINTER(i32),
+                                    ctypes.POINTER(i32)]
+    L.zero_runner_state.restype = ctypes.c_int
+    L.zero_runner_set_state.argtypes = [vp, i64, f32, i32, i32]
+    L.zero_runner_set_state.restype = ctypes.c_int
+    L.zero_runner_destroy.argtypes = [vp]
+    L.zero_runner_destroy.restype = None
     L.zero_test_wait_timeout.argtypes = [vp, i64, vp]
     L.zero_test_wait_timeout.restype = ctypes.c_int
     L.zero_allgather_params.argtypes = [ctypes.POINTER(vp), i32, i64, i64, ctypes.c_int, vp, vp]
@@ -292,6 +313,59 @@ def zero_loss_scale_update(scale: float, good_steps: int, overflow: bool,
     _check(lib.zero_loss_scale_update(ctypes.byref(s), ctypes.byref(g), int(bool(overflow)),
                                       growth_interval, min_scale))
     return s.value, g.value
+
+
+class Runner:
+    """zero_runner_*: the step over every bucket in two C calls (launch, commit).
+
+    `buckets`: list of (grad_bufs, [master0, master1], [m0, m1], [v0, v1],
+    [params0, params1]) tensors; flag_dev a device int32 tensor, flag_host a
+    pinned int32 tensor; the tensors must outlive the runner.
+    """
+
+    def __init__(self, buckets, hp: AdamHParams, loss_scale: float, flag_dev, flag_host, grad_sqnorm=None,
+                 workspace=None, growth_interval: int = 1000, min_scale: float = 1.0):
+        descs = (BucketBanks * max(1, len(buckets)))()
+        self._keep = []
+        world = len(buckets[0][0]) if buckets else 1
+        for i, (grads, master, m, v, params) in enumerate(buckets):
+            arr = _ptrs(grads)
+            self._keep.append(arr)
+            d = descs[i]
+            d.padded_numel = grads[0].numel()
+            d.grad_bufs = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+            for b in range(2):
+                d.master[b], d.m[b], d.v[b], d.params[b] = (_ptr(master[b]), _ptr(m[b]), _ptr(v[b]),
+                                                            _ptr(params[b]))
+        gd = _dtype_code(buckets[0][0][0]) if buckets else ZERO_F16
+        pd = _dtype_code(buckets[0][4][0]) if buckets else ZERO_F16
+        h = ctypes.c_void_p()
+        _check(lib.zero_runner_create(descs, len(buckets), world, gd, pd, ctypes.byref(hp), float(loss_scale),
+                                      growth_interval, min_scale, _ptr(flag_dev), _ptr(flag_host),
+                                      _ptr(grad_sqnorm), _ptr(workspace), ctypes.byref(h)))
+        self._h = h
+
+    def launch(self, stream=None) -> None:
+        _check(lib.zero_runner_launch(self._h, _stream(stream)))
+
+    def commit(self, stream=None) -> bool:
+        applied = ctypes.c_int32()
+        _check(lib.zero_runner_commit(self._h, _stream(stream), ctypes.byref(applied)))
+        return bool(applied.value)
+
+    def state(self):
+        t, s, g, b = ctypes.c_int64(), ctypes.c_float(), ctypes.c_int32(), ctypes.c_int32()
+        _check(lib.zero_runner_state(self._h, ctypes.byref(t), ctypes.byref(s), ctypes.byref(g), ctypes.byref(b)))
+        return t.value, s.value, g.value, b.value
+
+    def set_state(self, t: int, scale: float, good: int, bank: int) -> None:
+        _check(lib.zero_runner_set_state(self._h, t, scale, good, bank))
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            lib.zero_runner_destroy(h)
+            self._h = None
 
 
 def zero_test_wait_timeout(status, limit_ns: int, stream=None) -> None:

@@ -28,7 +28,7 @@ from __future__ import annotations
 
 import torch
 
-from . import (ZERO_ALL_PARTITIONS, hparams, zero_flatten_bucket, zero_grad_stats, zero_loss_scale_update,
+from . import (ZERO_ALL_PARTITIONS, Runner, hparams, zero_flatten_bucket, zero_grad_stats, zero_loss_scale_update,
                zero_partition_layout, zero_reduce_scatter_adam_step, zero_reduce_scatter_adam_step_gated,
                zero_step_workspace_bytes)
 
@@ -76,6 +76,21 @@ class ZeroAdam:
         self.workspace = (torch.zeros(zero_step_workspace_bytes(), dtype=torch.uint8, device=dev)
                           if need_norm else None)
         self.last_overflow = 0
+        # the single-pass banks mode runs through the native step runner:
+        # one C call enqueues the whole step, one commits it
+        self._runner = None
+        if not self.two_pass and L.n_buckets > 0:
+            self._flag_pinned = torch.zeros(1, dtype=torch.int32, pin_memory=True)
+            buckets = [(self.grads[b], self.master[b], self.m[b], self.v[b], self.params_bank[b])
+                       for b in range(L.n_buckets)]
+            self._runner = Runner(buckets, hparams(lr, betas[0], betas[1], eps, weight_decay, 1, grad_divisor),
+                                  self.scale, self.flag, self._flag_pinned, self.sqnorm, self.workspace,
+                                  growth_interval, min_scale)
+
+    def _sync_runner(self) -> None:
+        """Hand the Python-side step state to the runner."""
+        if self._runner is not None:
+            self._runner.set_state(self.t, self.scale, self.good_steps, self.cur)
 
     # ------------------------------------------------------------ state access
     def load(self, params, master=None, stream=None) -> None:
@@ -98,6 +113,7 @@ class ZeroAdam:
                     t.zero_()
         self.cur = 0
         self.t = 0
+        self._sync_runner()
 
     def state(self, b: int):
         """Committed (master, m, v, params) of bucket b."""
@@ -182,12 +198,31 @@ class ZeroAdam:
         self.scale, self.good_steps = zero_loss_scale_update(self.scale, self.good_steps, bool(ovf),
                                                              self.growth_interval, self.min_scale)
         self.last_overflow = ovf
+        self._sync_runner()
         return not ovf
 
     def step(self, stream=None, on_launch=None) -> bool:
-        """One whole step over all buckets; returns True if the update was applied."""
-        self.launch(stream, on_launch)
-        return self.commit(stream)
+        """One whole step over all buckets; returns True if the update was applied.
+
+        In the single-pass banks mode the native runner enqueues and commits
+        the step; `on_launch(-1, phase)` then brackets the whole step's device
+        work (flag clear, every bucket's kernel, the flag read-back).
+        Otherwise `on_launch(b, phase)` brackets each bucket's kernel."""
+        if self._runner is None:
+            self.launch(stream, on_launch)
+            return self.commit(stream)
+        with torch.cuda.stream(stream if stream is not None else torch.cuda.current_stream()):
+            if on_launch is not None:
+                on_launch(-1, "before")
+            self._runner.launch()
+            if on_launch is not None:
+                on_launch(-1, "after")
+            try:
+                applied = self._runner.commit()
+            finally:
+                self.t, self.scale, self.good_steps, self.cur = self._runner.state()
+        self.last_overflow = int(not applied)
+        return applied
 
     def step_from_host(self, host_grads, stream=None) -> bool:
         """Copy host gradients (host_grads[b][k], pinned) in, then step.
@@ -238,6 +273,7 @@ class ZeroAdam:
                     t.copy_(bucket[name].view(t.dtype) if bucket[name].dtype != t.dtype else bucket[name])
         self.cur = 0
         self.t, self.scale, self.good_steps = int(sd["t"]), float(sd["scale"]), int(sd["good_steps"])
+        self._sync_runner()
 
     def grad_sqnorm(self) -> float:
         """Sum of squared unscaled gradients of the last step (if tracked)."""
