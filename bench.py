@@ -36,8 +36,6 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-import numpy as np  # noqa: E402
-
 import workloads  # noqa: E402
 
 METRIC = "fused ZeRO step: Gparams/s and achieved HBM GB/s vs B200 peak (1 GPU)"

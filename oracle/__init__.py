@@ -31,7 +31,6 @@ from __future__ import annotations
 
 import ctypes
 import dataclasses
-import math
 import os
 import subprocess
 import tempfile

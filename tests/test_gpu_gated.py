@@ -18,7 +18,7 @@ import torch
 import oracle
 import workloads
 import zero_sharded_optimizer_reduce_b200 as Z
-from _gpu import Guarded, assert_f32_close, assert_u16_close, host_f32, host_u16, to_dev_u16
+from _gpu import assert_f32_close, assert_u16_close, host_f32, host_u16, to_dev_u16
 from test_gpu_step import TD, Case, _adam, _hp
 
 pytestmark = pytest.mark.gpu

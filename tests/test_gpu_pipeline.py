@@ -12,7 +12,6 @@ import torch
 
 import oracle
 import workloads
-import zero_sharded_optimizer_reduce_b200 as Z
 from test_gpu_step import Case, _adam
 
 pytestmark = pytest.mark.gpu

@@ -75,10 +75,6 @@ def _windows(padded, world, n_random=64, width=65_536, seed=0):
     return merged
 
 
-def _take(t, wins):
-    return [t[a:b] for a, b in wins]
-
-
 def _u16(t):
     return host_u16(t)
 

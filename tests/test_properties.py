@@ -3,7 +3,6 @@ the C ABI against the oracle on the CPU, and random small configurations of
 the fused step on the GPU against the oracle, bit for bit."""
 import numpy as np
 import pytest
-import torch
 from hypothesis import given, settings
 from hypothesis import strategies as st
 

@@ -363,8 +363,11 @@ class Runner:
 
     def __del__(self):
         h = getattr(self, "_h", None)
-        if h is not None and h.value:
-            lib.zero_runner_destroy(h)
+        if h is not None and h.value and lib is not None:
+            try:
+                lib.zero_runner_destroy(h)
+            except Exception:      # interpreter shutdown: the library may be gone
+                pass
             self._h = None
 
 

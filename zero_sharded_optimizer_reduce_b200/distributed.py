@@ -29,7 +29,7 @@ from __future__ import annotations
 import torch
 import torch.distributed as dist
 
-from . import (ZERO_ALL_PARTITIONS, DevicePtr, hparams, zero_allgather_params, zero_ipc_close,
+from . import (DevicePtr, hparams, zero_allgather_params, zero_ipc_close,
                zero_ipc_export, zero_ipc_import, zero_loss_scale_update, zero_partition_layout,
                zero_reduce_scatter_adam_step)
 
