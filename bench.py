@@ -145,23 +145,35 @@ def profiled_traffic(elems_per_launch: float):
 # --------------------------------------------------------------- CPU side
 
 def cpu_baseline(w: workloads.Workload, sample_elems: int, min_seconds: float = 10.0, max_seconds: float = 30.0):
-    """The oracle on this host's cores on a contiguous slice of bucket 0."""
+    """The oracle on this host's cores on a contiguous slice of bucket 0
+    (OpenMP over every core), plus the same slice on one thread."""
     import oracle
     N = w.world
     G = [workloads.grads(sample_elems, workloads.seed_for(w.seed, 1, k), w.grad_std, w.loss_scale)
          for k in range(N)]
-    st = oracle.initial_state(workloads.master(sample_elems, 7 * w.seed))
-    done, t0, t = 0, time.perf_counter(), 0
-    while True:
-        t += 1
-        oracle.flat_step(G, st, w.adam, t, w.loss_scale, float(N))
-        done += sample_elems
-        el = time.perf_counter() - t0
-        if el >= min_seconds or el >= max_seconds:
-            break
-    return {"value": done / el / 1e9, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
-            "sample": f"{t} oracle steps (reduce-scatter, overflow test, AdamW) over a {sample_elems:,}-element "
-                      f"slice of bucket 0 with N={N} replicas, {el:.1f} s"}
+
+    def timed(seconds):
+        st = oracle.initial_state(workloads.master(sample_elems, 7 * w.seed))
+        done, t0, t = 0, time.perf_counter(), 0
+        while True:
+            t += 1
+            oracle.flat_step(G, st, w.adam, t, w.loss_scale, float(N))
+            done += sample_elems
+            el = time.perf_counter() - t0
+            if el >= seconds or el >= max_seconds:
+                return done / el / 1e9, t, el
+
+    cores = oracle.threads()
+    value, steps, el = timed(min_seconds)
+    oracle.set_threads(1)
+    try:
+        single, _, _ = timed(min(5.0, min_seconds))
+    finally:
+        oracle.set_threads(cores)
+    return {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "single_thread_value": single,
+            "sample": f"{steps} oracle steps (reduce-scatter, overflow test, AdamW) over a {sample_elems:,}-element "
+                      f"slice of bucket 0 with N={N} replicas, {el:.1f} s on {cores} threads; "
+                      f"single_thread_value: the same slice on 1 thread"}
 
 
 def run_reference(args):
