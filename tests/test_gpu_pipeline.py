@@ -3,8 +3,10 @@
 Calls whose arrays share a 16-byte phase and that give every SM at least two
 tiles run the bulk-copy pipeline kernel; these sizes are chosen above that
 threshold (two stages of at most 180 KB: 6144 elements per tile at N = 1
-down to 2048 at N = 16, on 148 SMs), with ragged tails, a shifted
-common phase (scalar head), single partitions, bf16 and N up to 64.
+down to 1536 at N = 20, on 148 SMs), with ragged tails, a shifted
+common phase (scalar head), single partitions, bf16 and overflow.  Above
+N = 20 the register kernel runs at the same sizes; those cases (N up to 128)
+check that the kernel choice at the boundary keeps parity.
 """
 import numpy as np
 import pytest
@@ -28,7 +30,7 @@ def _tile(world):
     return min(8192, (180 * 1024 // (2 * (2 * world + 12))) // 512 * 512)
 
 
-@pytest.mark.parametrize("world", [1, 2, 3, 4, 8, 16, 64])
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 8, 16, 20, 21, 32, 40, 48, 64, 100, 128])
 def test_pipeline_ragged(world):
     T = _tile(world)
     per_rank = (2 * SMS * T + T // 2 + 5 + world - 1) // world
@@ -86,8 +88,8 @@ def test_pipeline_overflow_flag_and_in_place():
     assert ovf == 1 and int(c.flag.item()) == 1
 
 
-def test_pipeline_deterministic():
-    world = 8
+@pytest.mark.parametrize("world", [8, 64])
+def test_pipeline_deterministic(world):
     T = _tile(world)
     n = world * ((2 * SMS * T + 4099) // world)
     c = Case(n, world, seed=360, norm=True)
@@ -115,3 +117,29 @@ def test_pipeline_single_partition_with_head():
         ref, _, _ = c.expect(_adam())
         c.run(_adam())
         assert c.compare(ref) == [0, 0, 0, 0]
+
+
+@pytest.mark.parametrize("world,gd,pd", [(32, oracle.BF16, oracle.BF16), (64, oracle.F16, oracle.BF16),
+                                         (128, oracle.BF16, oracle.F16)])
+def test_pipeline_large_world_bf16_and_partition(world, gd, pd):
+    # the register kernel above N = 20, both dtypes, whole bucket and one partition
+    T = _tile(world)
+    P = 2 * SMS * T + 8 * 31
+    for r in (-1, world - 1):
+        c = Case(world * P, world, gdtype=gd, pdtype=pd, seed=380 + world, partition=r, scale=65536.0)
+        ref, _, _ = c.expect(_adam(0.01), t=3)
+        c.run(_adam(0.01), t=3)
+        assert c.compare(ref) == [0, 0, 0, 0]
+
+
+@pytest.mark.parametrize("world", [32, 64])
+def test_pipeline_large_world_overflow(world):
+    T = _tile(world)
+    n = world * ((2 * SMS * T + 77) // world)
+    c = Case(n, world, seed=390 + world)
+    workloads.inject(c.G[world - 1], np.array([n // 3]), np.array([False]))
+    from _gpu import to_dev_u16
+    to_dev_u16(c.G[world - 1], torch.float16, buf=c.g_dev[world - 1])
+    ref, ovf, _ = c.expect(_adam())
+    c.run(_adam())
+    assert ovf == 1 and int(c.flag.item()) == 1
