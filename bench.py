@@ -57,6 +57,27 @@ def bytes_per_elem(world: int) -> int:
     return 2 * world + 26
 
 
+def step_bytes_per_elem(world: int, mode: str, clipped: bool) -> int:
+    """Algorithmic HBM bytes per element of a whole step: the fused single
+    pass (2N + 26), statistics + gated update (4N + 26), or the staged
+    reduce-scatter (2N + 4) + update from the reduced gradients (30)."""
+    if mode == "staged":
+        return 2 * world + 34
+    if mode == "inplace" or clipped:
+        return 4 * world + 26
+    return 2 * world + 26
+
+
+def update_bytes_per_elem(world: int, mode: str) -> int:
+    """Algorithmic bytes per element of the kernel the roofline times (the
+    step's update kernel)."""
+    return 30 if mode == "staged" else 2 * world + 26
+
+
+PASSES = {"banks": "single fused pass", "inplace": "statistics pass (2N B/elem) + gated update (2N + 26)",
+          "staged": "reduce-scatter to fp32 (2N + 4 B/elem) + gated update from it (30)"}
+
+
 # ----------------------------------------------------------------- helpers
 
 class ClockSampler:
@@ -334,13 +355,14 @@ def run_gpu(args):
     ms = max_over_ranks(ms, "cuda")
     ms_per_step = ms / args.steps
     value = whole_job_gparams(psi_p, world_gpus, ms_per_step)
-    bpe = bytes_per_elem(w.world)
+    bpe = step_bytes_per_elem(w.world, args.mode, args.max_grad_norm is not None)
+    kbpe = update_bytes_per_elem(w.world, args.mode)
     peak, peak_kind = peaks()
-    kern_bytes = sum(launch_elems) * bpe
+    kern_bytes = sum(launch_elems) * kbpe
     kern_s = sum(launch_ms) * 1e-3
     achieved = kern_bytes / kern_s / 1e9
     avg_elems = sum(launch_elems) / len(launch_elems)
-    traffic = profiled_traffic(avg_elems)
+    traffic = profiled_traffic(avg_elems) if args.mode == "banks" else None
 
     # ---- end to end through the public API: host gradients in, flag out
     e2e = None
@@ -361,8 +383,8 @@ def run_gpu(args):
                            "buckets": L.n_buckets, "bucket_elems": w.bucket_elems, "grad_dtype": args.grad_dtype,
                            "param_dtype": args.grad_dtype, "optimizer": "AdamW wd=0.01", "stage": 2,
                            "mode": args.mode, "max_grad_norm": args.max_grad_norm,
-                           "passes": ("statistics pass (2N B/elem) + gated update" if opt.two_pass
-                                      else "single fused pass"),
+                           "passes": (PASSES[args.mode] if args.mode != "banks" or not opt.two_pass
+                                      else "statistics pass (2N B/elem) + clipped update (2N + 26)"),
                            "parallelism": f"{world_gpus} GPU(s) x {w.world} simulated replicas",
                            "l2": (f"inputs larger than L2: {psi_p * bpe / 1e9:.1f} GB of HBM traffic per step"
                                   if psi_p * bpe > 4 * 126e6 else "L2-influenced (footprint < 4x L2)")},
@@ -371,8 +393,10 @@ def run_gpu(args):
                              "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                              "kernel": ("fused_step (shared-memory pipeline kernel for aligned calls of >= 2 tiles per SM); "
                                         "timed per step over all buckets" if -1 in ev else
+                                        "adam_reduced_kernel (update from the fp32 reduced gradients)"
+                                        if args.mode == "staged" else
                                         "fused_step (shared-memory pipeline kernel for aligned calls of >= 2 tiles per SM)"),
-                             "bytes_per_elem": bpe,
+                             "bytes_per_elem": kbpe,
                              "elems_per_launch": avg_elems, "launches_timed": len(launch_ms),
                              "timed_unit": ("one step: all buckets' kernels + flag clear + 4-byte read-back"
                                             if -1 in ev else "one bucket's kernel")},
@@ -557,8 +581,9 @@ def main(argv=None):
     ap.add_argument("--grad-dtype", choices=["f16", "bf16"], default="f16")
     ap.add_argument("--sweep", action="store_true", help="flat bandwidth sweep, one JSON line per point")
     ap.add_argument("--stage3", action="store_true", help="layer-wise ZeRO-3 step on the 6.7B shape, prefetch on/off")
-    ap.add_argument("--mode", choices=["banks", "inplace"], default="banks",
-                    help="banks: two state banks, one pass; inplace: one bank, statistics pass + gated update")
+    ap.add_argument("--mode", choices=["banks", "inplace", "staged"], default="banks",
+                    help="banks: two state banks, one pass; inplace: one bank, statistics pass + gated update; "
+                         "staged: one bank, reduce-scatter to fp32 + gated update")
     ap.add_argument("--max-grad-norm", type=float, default=None, help="clip gradients to this global norm")
     ap.add_argument("--sweep-dtype-only", action="store_true", help="sweep only --grad-dtype")
     args = ap.parse_args(argv)

@@ -292,6 +292,62 @@ int zero_reduce_scatter_adam_step_gated(
     zero_stream_t stream);
 
 /*
+ * zero_reduce_scatter_grads - the reduce-scatter of a staged step: store
+ * each processed element's reduced, unscaled gradient in fp32.
+ *
+ * Source: ZeRO explainer (azimuth.plus), "Stage 2 - Gradient Partitioning
+ * (P_os+g)": the gradients are reduce-scattered so that each rank keeps the
+ * reduced gradients of its own partition only.  For each processed element
+ * (same `partition` convention as zero_reduce_scatter_adam_step) it forms
+ * the rank-order fp32 sum s of the N replicas and stores
+ * g = s * fp32(1/(divisor * loss_scale)) to reduced_out; the flag and the
+ * norm are those of zero_grad_stats.  2N + 4 bytes per element.
+ *
+ * reduced_out  device fp32, one element per processed element (P elements
+ *              for one partition, padded_numel for ZERO_ALL_PARTITIONS),
+ *              4-byte aligned (16-byte aligned at the same element as the
+ *              gradient buffers for the vector path); must not overlap a
+ *              gradient buffer.  Caller-owned.
+ * other arguments: as for zero_grad_stats.
+ * Errors: those of zero_grad_stats; ZERO_ERR_ARG for a NULL reduced_out.
+ */
+int zero_reduce_scatter_grads(const void* const* grad_bufs, int32_t world, int64_t padded_numel, int32_t partition,
+                              zero_dtype_t grad_dtype, float loss_scale, float grad_divisor, float* reduced_out,
+                              int32_t* overflow_flag, double* grad_sqnorm, void* workspace, zero_stream_t stream);
+
+/*
+ * zero_adam_step_reduced - the update of a staged step: Adam/AdamW on a
+ * partition from the reduced gradients that zero_reduce_scatter_grads
+ * stored.
+ *
+ * Source: ZeRO explainer, "Stage 2 - Gradient Partitioning (P_os+g)" (each
+ * rank updates its own partition from its reduced gradients); the update is
+ * the one of zero_reduce_scatter_adam_step with g read from reduced_grad
+ * instead of formed from the replicas, so both give identical bits for the
+ * same inputs.  Reads 16 and writes 14 bytes per element.
+ *
+ * reduced_grad  device fp32, `count` elements (unscaled gradients)
+ * count         elements, >= 0 (0: nothing is launched)
+ * master_in .. param_out, param_dtype, hp: as for
+ *               zero_reduce_scatter_adam_step, `count` elements each
+ *               (hp->grad_divisor is not used: the gradients are already
+ *               unscaled); in place when each *_out equals its *_in
+ * gate, clip_sqnorm, max_norm: as for zero_reduce_scatter_adam_step_gated
+ *               (pass the flag and the norm of the step's
+ *               zero_reduce_scatter_grads calls: an overflowing step then
+ *               writes nothing)
+ * No flag or norm is produced.
+ * Errors: ZERO_ERR_ARG, ZERO_ERR_DTYPE, ZERO_ERR_ALIGN, ZERO_ERR_CUDA.
+ */
+int zero_adam_step_reduced(const float* reduced_grad, int64_t count,
+                           const float* master_in, const float* m_in, const float* v_in,
+                           float* master_out, float* m_out, float* v_out,
+                           void* param_out, zero_dtype_t param_dtype,
+                           const zero_adam_hparams_t* hp,
+                           const int32_t* gate, const double* clip_sqnorm, float max_norm,
+                           zero_stream_t stream);
+
+/*
  * zero_reduce_scatter_adam_step_noalloc - zero_reduce_scatter_adam_step for
  * callers that cannot allocate device memory.
  *

@@ -88,6 +88,8 @@ def load_library(path: str):
     L.orc_any_nonfinite.restype = i32
     L.orc_grad_sqnorm.argtypes = [vp, i64, f32]
     L.orc_grad_sqnorm.restype = f64
+    L.orc_unscale.argtypes = [vp, i64, f32, vp]
+    L.orc_unscale.restype = None
     L.orc_adam_constants.argtypes = [f32, f32, f32, f32, f32, i64, f64, f32, vp]
     L.orc_adam_constants.restype = None
     L.orc_adam_update.argtypes = [vp, i64, vp, vp, vp, vp, vp, ctypes.c_int]
@@ -275,6 +277,14 @@ def any_nonfinite(s: np.ndarray) -> int:
 def grad_sqnorm(s: np.ndarray, inv: float) -> float:
     s = np.ascontiguousarray(s, dtype=np.float32)
     return float(lib().orc_grad_sqnorm(_ptr(s), s.size, float(inv)))
+
+
+def unscale(s: np.ndarray, inv: float) -> np.ndarray:
+    """The reduced, unscaled fp32 gradient g = s * inv of a rank's partition."""
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    g = np.empty_like(s)
+    lib().orc_unscale(_ptr(s), s.size, float(inv), _ptr(g))
+    return g
 
 
 def adam_constants(adam, t: int, divisor: float, loss_scale: float) -> np.ndarray:

@@ -208,6 +208,14 @@ double orc_grad_sqnorm(const float* s, int64_t count, float inv)
     return acc;
 }
 
+/* The reduced gradient a rank keeps after the reduce-scatter (ZeRO explainer,
+ * "Stage 2 - Gradient Partitioning (P_os+g)"), unscaled: g[j] = s[j]*inv in
+ * fp32, the same g the update and the norm use. */
+void orc_unscale(const float* s, int64_t count, float inv, float* g)
+{
+    for (int64_t j = 0; j < count; ++j) g[j] = s[j] * inv;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Adam                                                                     */
 /* ------------------------------------------------------------------------ */

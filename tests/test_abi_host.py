@@ -152,6 +152,54 @@ def test_step_with_nothing_to_do_is_ok():
     assert _step_call(n=0) == 0
 
 
+def _reduced_call(**kw):
+    """zero_adam_step_reduced with fake (never dereferenced) pointers."""
+    base = 0x7000_0000
+    f = lambda i: kw.get(f"p{i}", base + 0x100_0000 * i)
+    hp = kw.get("hp", Z.hparams())
+    return Z.lib.zero_adam_step_reduced(
+        kw.get("red", base + 0x100_0000 * 12), kw.get("n", 64), f(1), f(2), f(3), f(4), f(5), f(6), f(7),
+        kw.get("pd", 0), None if hp is None else ctypes.byref(hp), kw.get("gate", None), kw.get("clip", None),
+        kw.get("max_norm", 0.0), None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(hp=None), -1),
+    (dict(n=-1), -1),
+    (dict(pd=2), -3),
+    (dict(hp=Z.hparams(step=0)), -1),
+    (dict(red=0), -1),                              # NULL reduced gradient
+    (dict(red=0x7C00_0002), -2),                    # reduced gradient not 4-byte aligned
+    (dict(p2=0), -1),                               # NULL m_in
+    (dict(p6=0x7600_0002), -2),                     # v_out misaligned
+    (dict(p7=0x7700_0001), -2),                     # param_out misaligned
+    (dict(red=0x7400_0000 + 4), -1),                # reduced gradient overlaps master_out
+    (dict(p5=0x7100_0000), -1),                     # m_out is master_in
+    (dict(gate=0x7D00_0002), -2),                   # misaligned gate
+    (dict(clip=0x7E00_0000, max_norm=0.0), -1),     # clipping without a positive max_norm
+])
+def test_reduced_update_rejects_bad_arguments(kw, code):
+    assert _reduced_call(**kw) == code
+    assert Z.lib.zero_last_error() != b""
+
+
+def test_reduced_update_with_nothing_to_do_is_ok():
+    assert _reduced_call(n=0) == 0
+
+
+def test_staged_reduce_scatter_rejects_bad_arguments():
+    L = Z.lib
+    g = (ctypes.c_void_p * 2)(0x10000, 0x20000)
+    flag = 0x7000_0000
+    assert L.zero_reduce_scatter_grads(g, 2, 64, -1, 0, 1.0, 0.0, None, flag, None, None, None) == -1
+    assert L.zero_reduce_scatter_grads(g, 2, 64, -1, 0, 1.0, 0.0, 0x30002, flag, None, None, None) == -2
+    assert L.zero_reduce_scatter_grads(g, 2, 64, -1, 0, 1.0, 0.0, 0x10040, flag, None, None, None) == -1
+    assert L.zero_reduce_scatter_grads(g, 2, 63, -1, 0, 1.0, 0.0, 0x30000, flag, None, None, None) == -1
+    assert L.zero_reduce_scatter_grads(g, 2, 64, 3, 0, 1.0, 0.0, 0x30000, flag, None, None, None) == -4
+    assert L.zero_reduce_scatter_grads(g, 2, 64, -1, 2, 1.0, 0.0, 0x30000, flag, None, None, None) == -3
+    assert L.zero_reduce_scatter_grads(g, 2, 0, -1, 0, 1.0, 0.0, 0x30000, flag, None, None, None) == 0
+
+
 def test_allgather_and_flatten_reject_bad_arguments():
     L = Z.lib
     sh = (ctypes.c_void_p * 2)(0x10000, 0x20000)

@@ -160,12 +160,13 @@ def _upload(opt, G):
             opt.grad_buffers(b)[k].copy_(torch.from_numpy(g.view(np.int16)).cuda().view(torch.float16))
 
 
+@pytest.mark.parametrize("mode", ["inplace", "staged"])
 @pytest.mark.parametrize("max_norm", [None, 0.3])
-def test_zeroadam_inplace_mode(max_norm):
+def test_zeroadam_one_bank_modes(mode, max_norm):
     numels = [300_000, 77, 1_200_003, 5, 250_000]
     N, cap = 8, 1_000_000
     adam = workloads.AdamConfig(weight_decay=0.01)
-    L, opt, states = _opt_and_oracle(numels, N, cap, adam, "inplace", max_norm)
+    L, opt, states = _opt_and_oracle(numels, N, cap, adam, mode, max_norm)
     assert all(len(bank) == 1 for bank in opt.master)          # one bank: 12 Psi/N of optimizer state
     scale, good, t = 65536.0, 0, 0
     for step in range(1, 6):
@@ -227,7 +228,7 @@ def test_zeroadam_banks_mode_with_clipping():
         assert assert_u16_close(host_u16(p), states[b].params, "params") == 0
 
 
-@pytest.mark.parametrize("mode", ["banks", "inplace"])
+@pytest.mark.parametrize("mode", ["banks", "inplace", "staged"])
 def test_checkpoint_resume_bit_identical(mode):
     """Save after step 2, reload into a fresh optimizer: steps 3-5 (one with
     an injected overflow) are bit-identical to the uninterrupted run."""
@@ -286,7 +287,7 @@ def test_stats_pipeline(world, dtype, goff):
         to_dev_u16(g, TD[dtype], buf=c.g_dev[world - 1])
 
 
-@pytest.mark.parametrize("mode", ["banks", "inplace"])
+@pytest.mark.parametrize("mode", ["banks", "inplace", "staged"])
 def test_step_from_host_matches_device_step(mode):
     """The end-to-end entry (pinned host gradients, per-bucket copy stream)
     gives the same bits as writing the gradients on the device first."""

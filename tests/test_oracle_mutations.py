@@ -47,6 +47,7 @@ MUTANTS = [
     ("norm squares the scaled sum", "float g = s[j] * inv;\n        acc += (double)g * (double)g;",
      "float g = s[j];\n        acc += (double)g * (double)g;"),
     ("clip factor not clamped", "return coef < 1.0 ? (float)coef : 1.0f;", "return (float)coef;"),
+    ("reduced gradient not unscaled", "g[j] = s[j] * inv;", "g[j] = s[j];"),
 ]
 
 # cheap pins first; each entry is (label, callable)
@@ -61,6 +62,7 @@ PINS = [
     ("nan flag", R.test_nan_alone_sets_the_flag),
     ("flag f16", lambda: R.test_overflow_flag(oracle.F16)),
     ("sqnorm", R.test_grad_sqnorm_matches_fp64_sum),
+    ("unscale exact", lambda: R.test_unscale_by_power_of_two_is_exact(8, 65536.0)),
     ("gather offset", LY.test_allgather_with_offset_brute_force),
     ("adam constants", A.test_constants_are_rounded_from_double),
     ("adam step-1 closed form", lambda: A.test_step1_closed_form(0.0)),

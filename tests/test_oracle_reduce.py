@@ -90,3 +90,25 @@ def test_nan_alone_sets_the_flag():
     G[2][17] = 0xFC00                          # -inf: inf + (-inf) is NaN
     s = oracle.reduce(G)
     assert np.isnan(s[17]) and oracle.any_nonfinite(s) == 1
+
+
+@pytest.mark.parametrize("N,S", [(8, 65536.0), (16, 1024.0), (1, 1.0)])
+def test_unscale_by_power_of_two_is_exact(N, S):
+    # 1/(N*S) is a power of two: the unscaled gradient is s * 2^-k exactly
+    G = [workloads.grads(5_003, 40 + k, 1e-3, S) for k in range(N)]
+    s = oracle.reduce(G)
+    k = int(np.log2(N * S))
+    g = oracle.unscale(s, 2.0 ** -k)
+    assert np.array_equal(g, np.ldexp(s, -k).astype(np.float32))
+
+
+def test_unscale_is_the_correctly_rounded_product():
+    # inv = 1/(3 * 1000) is not a power of two; the product of two fp32
+    # values is exact in fp64 (48 significant bits), so the fp32 result must
+    # be that exact product rounded once to nearest
+    s = oracle.reduce([workloads.grads(20_011, 60 + k, 1e-3, 1000.0) for k in range(3)])
+    inv = np.float32(1.0 / 3000.0)
+    g = oracle.unscale(s, float(inv))
+    exact = s.astype(np.float64) * np.float64(inv)
+    assert np.array_equal(g, exact.astype(np.float32))
+    assert not np.array_equal(g, s)

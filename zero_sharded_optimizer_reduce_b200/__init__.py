@@ -104,6 +104,12 @@ def _load():
         vp, vp, vp, vp, vp, vp, vp, ctypes.c_int,
         ctypes.POINTER(AdamHParams), f32, vp, vp, vp, vp, vp, f32, vp]
     L.zero_reduce_scatter_adam_step_gated.restype = ctypes.c_int
+    L.zero_reduce_scatter_grads.argtypes = [ctypes.POINTER(vp), i32, i64, i32, ctypes.c_int, f32, f32, vp, vp, vp,
+                                            vp, vp]
+    L.zero_reduce_scatter_grads.restype = ctypes.c_int
+    L.zero_adam_step_reduced.argtypes = [vp, i64, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int,
+                                         ctypes.POINTER(AdamHParams), vp, vp, f32, vp]
+    L.zero_adam_step_reduced.restype = ctypes.c_int
     L.zero_ipc_export.argtypes = [vp, ctypes.POINTER(IpcHandle), ctypes.POINTER(i64)]
     L.zero_ipc_export.restype = ctypes.c_int
     L.zero_ipc_import.argtypes = [ctypes.POINTER(IpcHandle), i64, ctypes.POINTER(vp), ctypes.POINTER(vp)]
@@ -297,6 +303,26 @@ def zero_reduce_scatter_adam_step_gated(grad_bufs, padded_numel: int, partition:
         _ptr(master_in), _ptr(m_in), _ptr(v_in), _ptr(master_out), _ptr(m_out), _ptr(v_out),
         _ptr(param_out), _dtype_code(param_out), ctypes.byref(hp), float(loss_scale),
         _ptr(overflow_flag), _ptr(grad_sqnorm), _ptr(workspace), _ptr(gate), _ptr(clip_sqnorm),
+        float(max_norm), _stream(stream)))
+
+
+def zero_reduce_scatter_grads(grad_bufs, padded_numel: int, partition: int, loss_scale: float, reduced_out,
+                              overflow_flag, grad_sqnorm=None, workspace=None, grad_divisor: float = 0.0,
+                              stream=None) -> None:
+    """Staged reduce-scatter: reduced_out = fp32 unscaled rank-order sums, plus flag and norm."""
+    _check(lib.zero_reduce_scatter_grads(_ptrs(grad_bufs), len(grad_bufs), padded_numel, partition,
+                                         _dtype_code(grad_bufs[0]), float(loss_scale), float(grad_divisor),
+                                         _ptr(reduced_out), _ptr(overflow_flag), _ptr(grad_sqnorm),
+                                         _ptr(workspace), _stream(stream)))
+
+
+def zero_adam_step_reduced(reduced_grad, count: int, master_in, m_in, v_in, master_out, m_out, v_out, param_out,
+                           hp: AdamHParams, gate=None, clip_sqnorm=None, max_norm: float = 0.0,
+                           stream=None) -> None:
+    """Staged update: Adam on `count` elements from fp32 reduced gradients (gated, optionally clipped)."""
+    _check(lib.zero_adam_step_reduced(
+        _ptr(reduced_grad), count, _ptr(master_in), _ptr(m_in), _ptr(v_in), _ptr(master_out), _ptr(m_out),
+        _ptr(v_out), _ptr(param_out), _dtype_code(param_out), ctypes.byref(hp), _ptr(gate), _ptr(clip_sqnorm),
         float(max_norm), _stream(stream)))
 
 

@@ -21,8 +21,10 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libzero.so")
 
-SOURCES = ["step.cu", "step_static.cu", "stats.cu", "selftest.cu", "runner.cu", "copy.cu", "host.cpp", "ipc.cpp"]
-HEADERS = [os.path.join(CSRC, n) for n in ("common.h", "fused_step.cuh", "grad_stats.cuh", "step_launch.h")] + [os.path.join(INCLUDE, "zero.h")]
+SOURCES = ["step.cu", "step_static.cu", "stats.cu", "staged.cu", "selftest.cu", "runner.cu", "copy.cu", "host.cpp",
+           "ipc.cpp"]
+HEADERS = [os.path.join(CSRC, n) for n in ("common.h", "fused_step.cuh", "grad_stats.cuh", "staged.cuh",
+                                                        "step_launch.h")] + [os.path.join(INCLUDE, "zero.h")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -2,8 +2,10 @@
 // replicas, the overflow OR and (optionally) the squared norm of the
 // unscaled gradient, with no optimizer state read or written.  2N bytes per
 // element.  Used before an in-place update (exact skip with one bank of
-// states) and for global-norm clipping.  Device helpers come from
-// fused_step.cuh.
+// states) and for global-norm clipping.  With kWrite they are also the
+// staged reduce-scatter: each element's unscaled gradient g = s * inv is
+// stored to `reduced` as fp32 (2N + 4 bytes per element).  Device helpers
+// come from fused_step.cuh.
 #pragma once
 
 #include "fused_step.cuh"
@@ -20,10 +22,10 @@ __device__ __forceinline__ float replica_sum(const StepParams& p, int64_t e) {
     return s;
 }
 
-// Elements outside the vector (or tile) region, statistics only.
-template <typename GT>
-__device__ __forceinline__ void stats_scalar_elements(const StepParams& p, int64_t tid, int64_t nthreads, bool& bad,
-                                                      double& sq) {
+// Elements outside the vector (or tile) region.
+template <typename GT, bool kWrite>
+__device__ __forceinline__ void stats_scalar_elements(const StepParams& p, float* reduced, int64_t tid,
+                                                      int64_t nthreads, bool& bad, double& sq) {
     const float inv = p.c.inv;
     const int64_t vec_end = p.head + p.nvec * kVec;
     const int64_t nscalar = p.head + (p.count - vec_end);
@@ -31,10 +33,9 @@ __device__ __forceinline__ void stats_scalar_elements(const StepParams& p, int64
         const int64_t e = q < p.head ? q : vec_end + (q - p.head);
         const float s = replica_sum<GT>(p, e);
         bad |= !isfinite(s);
-        if (p.sqnorm) {
-            const float g = __fmul_rn(s, inv);
-            sq = fma(static_cast<double>(g), static_cast<double>(g), sq);
-        }
+        const float g = __fmul_rn(s, inv);
+        if constexpr (kWrite) reduced[e] = g;
+        if (p.sqnorm) sq = fma(static_cast<double>(g), static_cast<double>(g), sq);
     }
 }
 
@@ -43,8 +44,10 @@ __device__ __forceinline__ void stats_scalar_elements(const StepParams& p, int64
 // gradient g = s * inv, without reading or writing any optimizer state.
 // 2N bytes per element.  Lets a caller decide skip and clipping for a whole
 // step before any state is written (in-place update with an exact skip).
-template <typename GT>
-__global__ void __launch_bounds__(kThreads) grad_stats_kernel(const __grid_constant__ StepParams p) {
+// kWrite: also store g to reduced[e] (16-byte stores).
+template <typename GT, bool kWrite>
+__global__ void __launch_bounds__(kThreads) grad_stats_kernel(const __grid_constant__ StepParams p,
+                                                              float* __restrict__ reduced) {
     const int64_t tid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
     const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
     const int world = p.world;
@@ -74,25 +77,30 @@ __global__ void __launch_bounds__(kThreads) grad_stats_kernel(const __grid_const
             for (int b = 0; b < kBatch; ++b)
                 if (k0 + b < world) add8<GT>(r[b], s);
         }
+        float g[kVec];
 #pragma unroll
         for (int e = 0; e < kVec; ++e) {
             bad |= !isfinite(s[e]);
-            if (want_sq) {
-                const float g = __fmul_rn(s[e], inv);
-                sq = fma(static_cast<double>(g), static_cast<double>(g), sq);
-            }
+            g[e] = __fmul_rn(s[e], inv);
+            if (want_sq) sq = fma(static_cast<double>(g[e]), static_cast<double>(g[e]), sq);
+        }
+        if constexpr (kWrite) {
+            st_state16(reduced + e0, g[0], g[1], g[2], g[3]);
+            st_state16(reduced + e0 + 4, g[4], g[5], g[6], g[7]);
         }
     }
-    stats_scalar_elements<GT>(p, tid, nthreads, bad, sq);
+    stats_scalar_elements<GT, kWrite>(p, reduced, tid, nthreads, bad, sq);
     finish_block<kThreads>(p, bad, sq);
 }
 
 // Pipeline statistics kernel: the producer warp streams tiles of the N
 // gradient slices into two shared-memory stages with 1-D bulk copies (no
 // multicast, this CTA's own shared memory); 16 consumer warps sum each
-// 4-element chunk in rank order.  Waits bounded as in the step's pipeline.
-template <typename GT>
-__global__ void __launch_bounds__(kPipeThreads, 1) grad_stats_pipe_kernel(const __grid_constant__ StepParams p) {
+// 4-element chunk in rank order (kWrite: and store its 4 unscaled gradients
+// with one 16-byte store).  Waits bounded as in the step's pipeline.
+template <typename GT, bool kWrite>
+__global__ void __launch_bounds__(kPipeThreads, 1) grad_stats_pipe_kernel(const __grid_constant__ StepParams p,
+                                                                          float* __restrict__ reduced) {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t full[kPipeStages];
     __shared__ __align__(8) uint64_t empty[kPipeStages];
@@ -165,6 +173,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) grad_stats_pipe_kernel(const 
                 break;
             }
             const unsigned char* st = smem + static_cast<size_t>(s) * stage;
+            const int64_t base = p.head + tile * T;
             for (int ch = t; ch < T / 4; ch += C) {
                 const int j = 4 * ch;
                 const uint2 r0 = *reinterpret_cast<const uint2*>(st + 2 * j);
@@ -178,9 +187,10 @@ __global__ void __launch_bounds__(kPipeThreads, 1) grad_stats_pipe_kernel(const 
                     a3 = __fadd_rn(a3, Fmt<GT>::hi(r.y));
                 }
                 bad |= !isfinite(a0) | !isfinite(a1) | !isfinite(a2) | !isfinite(a3);
+                const float g0 = __fmul_rn(a0, inv), g1 = __fmul_rn(a1, inv);
+                const float g2 = __fmul_rn(a2, inv), g3 = __fmul_rn(a3, inv);
+                if constexpr (kWrite) st_state16(reduced + base + j, g0, g1, g2, g3);
                 if (want_sq) {
-                    const float g0 = __fmul_rn(a0, inv), g1 = __fmul_rn(a1, inv);
-                    const float g2 = __fmul_rn(a2, inv), g3 = __fmul_rn(a3, inv);
                     sq = fma(static_cast<double>(g0), static_cast<double>(g0), sq);
                     sq = fma(static_cast<double>(g1), static_cast<double>(g1), sq);
                     sq = fma(static_cast<double>(g2), static_cast<double>(g2), sq);
@@ -190,8 +200,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1) grad_stats_pipe_kernel(const 
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
         }
-        stats_scalar_elements<GT>(p, static_cast<int64_t>(blockIdx.x) * C + t, static_cast<int64_t>(gridDim.x) * C,
-                                  bad, sq);
+        stats_scalar_elements<GT, kWrite>(p, reduced, static_cast<int64_t>(blockIdx.x) * C + t,
+                                          static_cast<int64_t>(gridDim.x) * C, bad, sq);
     }
     finish_block<kPipeThreads>(p, bad, sq);
 }

@@ -1,0 +1,163 @@
+// The staged ZeRO-2 step: a reduce-scatter that stores each partition's
+// reduced gradients in fp32, then the Adam update from them.
+//
+// ZeRO explainer (azimuth.plus), "Stage 2 - Gradient Partitioning (P_os+g)":
+// the gradients are reduce-scattered so that each rank keeps only the
+// reduced gradients of its own partition, and updates that partition.  The
+// fused step never materialises them (2N + 26 bytes per element, but its
+// exact skip needs a second bank of states); the statistics route re-reads
+// the N replicas (4N + 26).  Staged, the reduce-scatter writes the reduced
+// gradients once (2N + 4) and the update reads them back (30): 2N + 34 bytes
+// per element with one bank of states plus 4 bytes per element of reduced
+// gradients, the exact skip taken by the update's device-side gate.
+#include "staged.cuh"
+#include "step_launch.h"
+
+namespace zero {
+namespace fused {
+namespace {
+
+inline KernelFn pick_reduced_kernel(zero_dtype_t pd) {
+    return pd == ZERO_F16 ? adam_reduced_kernel<__half> : adam_reduced_kernel<__nv_bfloat16>;
+}
+
+std::mutex g_red_mu;
+int g_red_blocks[64][2] = {};
+
+inline int reduced_grid_limit(zero_dtype_t pd, int* out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return fail(ZERO_ERR_CUDA, "cudaGetDevice failed");
+    std::lock_guard<std::mutex> lk(g_red_mu);
+    int& per_sm = g_red_blocks[dev][pd == ZERO_F16 ? 0 : 1];
+    static int sms[64] = {};
+    if (sms[dev] == 0 && cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return fail(ZERO_ERR_CUDA, "cannot query the SM count");
+    if (per_sm == 0) {
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pick_reduced_kernel(pd), kThreads, 0);
+        if (e != cudaSuccess || per_sm < 1) {
+            per_sm = 0;
+            return fail(ZERO_ERR_CUDA, "occupancy query failed: %s", cudaGetErrorString(e));
+        }
+    }
+    const int lim = sms[dev] * per_sm;
+    *out = lim < kMaxBlocks ? lim : kMaxBlocks;
+    return ZERO_OK;
+}
+
+// Validate an update-from-reduced call and build its parameters;
+// *work_out is the number of vector (or, with none, scalar) work items.
+inline int prepare_reduced(const char* fn, const float* reduced, int64_t count, const float* master_in,
+                           const float* m_in, const float* v_in, float* master_out, float* m_out, float* v_out,
+                           void* param_out, zero_dtype_t param_dtype, const zero_adam_hparams_t* hp,
+                           StepParams* prm_out, int64_t* work_out) {
+    if (!hp) return fail(ZERO_ERR_ARG, "%s: NULL hp", fn);
+    if (count < 0) return fail(ZERO_ERR_ARG, "%s: negative count", fn);
+    if (param_dtype != ZERO_F16 && param_dtype != ZERO_BF16)
+        return fail(ZERO_ERR_DTYPE, "%s: parameters must be ZERO_F16 or ZERO_BF16", fn);
+    if (int rc = check_hparams(fn, hp)) return rc;
+    if (count == 0) {
+        *work_out = 0;
+        return ZERO_OK;
+    }
+    const float* f_in[] = {master_in, m_in, v_in, reduced};
+    float* f_out[] = {master_out, m_out, v_out};
+    for (const float* a : f_in) {
+        if (!a) return fail(ZERO_ERR_ARG, "%s: NULL input array", fn);
+        if (!aligned(a, 4)) return fail(ZERO_ERR_ALIGN, "%s: fp32 input not 4-byte aligned", fn);
+    }
+    for (float* a : f_out) {
+        if (!a) return fail(ZERO_ERR_ARG, "%s: NULL output array", fn);
+        if (!aligned(a, 4)) return fail(ZERO_ERR_ALIGN, "%s: fp32 output not 4-byte aligned", fn);
+    }
+    if (!param_out) return fail(ZERO_ERR_ARG, "%s: NULL param_out", fn);
+    if (!aligned(param_out, 2)) return fail(ZERO_ERR_ALIGN, "%s: param_out not 2-byte aligned", fn);
+    // each output is its own input (in place) or overlaps nothing else
+    const int64_t fb = count * 4;
+    const void* outs[] = {master_out, m_out, v_out, param_out};
+    const int64_t out_bytes[] = {fb, fb, fb, count * 2};
+    for (int i = 0; i < 4; ++i) {
+        for (int j = i + 1; j < 4; ++j)
+            if (overlaps(outs[i], out_bytes[i], outs[j], out_bytes[j]))
+                return fail(ZERO_ERR_ARG, "%s: output arrays overlap", fn);
+        for (int j = 0; j < 4; ++j)
+            if (!(i == j && j < 3 && outs[i] == f_in[j]) && overlaps(outs[i], out_bytes[i], f_in[j], fb))
+                return fail(ZERO_ERR_ARG, "%s: an output overlaps an input it does not replace", fn);
+    }
+
+    StepParams prm{};
+    prm.world = 1;
+    prm.grads[0] = reduced;
+    prm.count = count;
+    prm.master_in = master_in;
+    prm.m_in = m_in;
+    prm.v_in = v_in;
+    prm.master_out = master_out;
+    prm.m_out = m_out;
+    prm.v_out = v_out;
+    prm.param_out = param_out;
+    prm.c = adam_consts(hp, 1.0f);
+    // the first element at which every array sits on a 16-byte boundary
+    int64_t h = -1;
+    for (int64_t c = 0; c < kVec && h < 0; ++c) {
+        bool good = ((reinterpret_cast<uintptr_t>(param_out) + 2 * c) % 16) == 0;
+        const void* f32s[] = {reduced, master_in, m_in, v_in, master_out, m_out, v_out};
+        for (const void* a : f32s) good = good && ((reinterpret_cast<uintptr_t>(a) + 4 * c) % 16) == 0;
+        if (good) h = c;
+    }
+    if (h < 0 || h >= count) {
+        prm.head = count;
+        prm.nvec = 0;
+    } else {
+        prm.head = h;
+        prm.nvec = (count - h) / kVec;
+    }
+    *prm_out = prm;
+    *work_out = prm.nvec > 0 ? prm.nvec : count;
+    return ZERO_OK;
+}
+
+}  // namespace
+}  // namespace fused
+}  // namespace zero
+
+using zero::fail;
+
+extern "C" int zero_reduce_scatter_grads(const void* const* grad_bufs, int32_t world, int64_t padded_numel,
+                                         int32_t partition, zero_dtype_t grad_dtype, float loss_scale,
+                                         float grad_divisor, float* reduced_out, int32_t* overflow_flag,
+                                         double* grad_sqnorm, void* workspace, zero_stream_t stream) {
+    using namespace zero::fused;
+    const char* fn = "zero_reduce_scatter_grads";
+    if (!reduced_out) return fail(ZERO_ERR_ARG, "%s: NULL reduced_out", fn);
+    StepParams prm{};
+    int64_t blocks = 0;
+    if (int rc = prepare_stats(fn, grad_bufs, world, padded_numel, partition, grad_dtype, loss_scale, grad_divisor,
+                               reduced_out, overflow_flag, grad_sqnorm, workspace, &prm, &blocks))
+        return rc;
+    return launch_stats(fn, prm, blocks, grad_dtype, reduced_out, stream);
+}
+
+extern "C" int zero_adam_step_reduced(const float* reduced_grad, int64_t count, const float* master_in,
+                                      const float* m_in, const float* v_in, float* master_out, float* m_out,
+                                      float* v_out, void* param_out, zero_dtype_t param_dtype,
+                                      const zero_adam_hparams_t* hp, const int32_t* gate, const double* clip_sqnorm,
+                                      float max_norm, zero_stream_t stream) {
+    using namespace zero::fused;
+    const char* fn = "zero_adam_step_reduced";
+    StepParams prm{};
+    int64_t work = 0;
+    if (int rc = prepare_reduced(fn, reduced_grad, count, master_in, m_in, v_in, master_out, m_out, v_out, param_out,
+                                 param_dtype, hp, &prm, &work))
+        return rc;
+    if (int rc = add_gate_and_clip(fn, &prm, gate, clip_sqnorm, max_norm)) return rc;
+    if (work == 0) return zero::ok();
+    int limit = 0;
+    if (int rc = reduced_grid_limit(param_dtype, &limit)) return rc;
+    int64_t blocks = (work + kThreads - 1) / kThreads;
+    if (blocks > limit) blocks = limit;
+    pick_reduced_kernel(param_dtype)<<<static_cast<unsigned int>(blocks), kThreads, 0,
+                                       reinterpret_cast<cudaStream_t>(stream)>>>(prm);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(ZERO_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
+    return zero::ok();
+}

@@ -21,9 +21,9 @@ extern "C" int zero_grad_stats(const void* const* grad_bufs, int32_t world, int6
     StepParams prm{};
     int64_t blocks = 0;
     if (int rc = prepare_stats(fn, grad_bufs, world, padded_numel, partition, grad_dtype, loss_scale, grad_divisor,
-                               overflow_flag, grad_sqnorm, workspace, &prm, &blocks))
+                               nullptr, overflow_flag, grad_sqnorm, workspace, &prm, &blocks))
         return rc;
-    return launch_stats(fn, prm, blocks, grad_dtype, stream);
+    return launch_stats(fn, prm, blocks, grad_dtype, nullptr, stream);
 }
 
 extern "C" int zero_reduce_scatter_adam_step_gated(

@@ -18,6 +18,7 @@ constexpr uint32_t kPipeSmemMax = 220u * 1024u;     // dynamic shared memory cap
 constexpr int kPipeMaxWorld = 20;                   // largest N measured to gain from the pipeline
 
 using KernelFn = void (*)(StepParams);
+using StatsKernelFn = void (*)(StepParams, float*);
 
 inline KernelFn pick_kernel(zero_dtype_t g, zero_dtype_t pd) {
     if (g == ZERO_F16 && pd == ZERO_F16) return fused_step_kernel<__half, __half>;
@@ -26,12 +27,17 @@ inline KernelFn pick_kernel(zero_dtype_t g, zero_dtype_t pd) {
     return fused_step_kernel<__nv_bfloat16, __nv_bfloat16>;
 }
 
-inline KernelFn pick_stats_kernel(zero_dtype_t g) {
-    return g == ZERO_F16 ? grad_stats_kernel<__half> : grad_stats_kernel<__nv_bfloat16>;
+// write: the staged reduce-scatter variant that also stores the unscaled
+// gradients
+inline StatsKernelFn pick_stats_kernel(zero_dtype_t g, bool write) {
+    if (write) return g == ZERO_F16 ? grad_stats_kernel<__half, true> : grad_stats_kernel<__nv_bfloat16, true>;
+    return g == ZERO_F16 ? grad_stats_kernel<__half, false> : grad_stats_kernel<__nv_bfloat16, false>;
 }
 
-inline KernelFn pick_stats_pipe_kernel(zero_dtype_t g) {
-    return g == ZERO_F16 ? grad_stats_pipe_kernel<__half> : grad_stats_pipe_kernel<__nv_bfloat16>;
+inline StatsKernelFn pick_stats_pipe_kernel(zero_dtype_t g, bool write) {
+    if (write)
+        return g == ZERO_F16 ? grad_stats_pipe_kernel<__half, true> : grad_stats_pipe_kernel<__nv_bfloat16, true>;
+    return g == ZERO_F16 ? grad_stats_pipe_kernel<__half, false> : grad_stats_pipe_kernel<__nv_bfloat16, false>;
 }
 
 inline KernelFn pick_pipe_kernel(zero_dtype_t g, zero_dtype_t pd) {
@@ -79,9 +85,9 @@ inline uint32_t pipe_smem_bytes(int world, int tile) {
 struct DeviceInfo {
     int sms = 0;
     int blocks_per_sm[4] = {0, 0, 0, 0};
-    int stats_blocks_per_sm[2] = {0, 0};
+    int stats_blocks_per_sm[4] = {0, 0, 0, 0};   // [dtype * 2 + write]
     bool pipe_ready[4] = {false, false, false, false};
-    bool stats_pipe_ready[2] = {false, false};
+    bool stats_pipe_ready[4] = {false, false, false, false};
 };
 
 std::mutex g_dev_mu;
@@ -116,14 +122,14 @@ inline int grid_limit(zero_dtype_t g, zero_dtype_t pd, int* out) {
     return ZERO_OK;
 }
 
-inline int stats_grid_limit(zero_dtype_t g, int* out) {
-    const int which = static_cast<int>(g);
+inline int stats_grid_limit(zero_dtype_t g, bool write, int* out) {
+    const int which = static_cast<int>(g) * 2 + (write ? 1 : 0);
     std::lock_guard<std::mutex> lk(g_dev_mu);
     DeviceInfo* d = nullptr;
     if (int rc = device_info(&d)) return rc;
     if (d->stats_blocks_per_sm[which] == 0) {
         int n = 0;
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, pick_stats_kernel(g), kThreads, 0);
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, pick_stats_kernel(g, write), kThreads, 0);
         if (e != cudaSuccess || n < 1) return fail(ZERO_ERR_CUDA, "occupancy query failed: %s", cudaGetErrorString(e));
         d->stats_blocks_per_sm[which] = n;
     }
@@ -165,6 +171,35 @@ inline int64_t common_phase(const StepParams& p) {
 }
 
 
+// Range checks of the Adam hyper-parameters shared by every update call.
+inline int check_hparams(const char* fn, const zero_adam_hparams_t* hp) {
+    if (!(hp->step >= 1)) return fail(ZERO_ERR_ARG, "%s: hp->step must be >= 1", fn);
+    if (!std::isfinite(hp->lr) || !std::isfinite(hp->eps) || !std::isfinite(hp->weight_decay) ||
+        !(hp->beta1 >= 0.0f && hp->beta1 < 1.0f) || !(hp->beta2 >= 0.0f && hp->beta2 < 1.0f) ||
+        !(hp->grad_divisor >= 0.0f) || !std::isfinite(hp->grad_divisor))
+        return fail(ZERO_ERR_ARG, "%s: hyper-parameters out of range", fn);
+    return ZERO_OK;
+}
+
+// The update's constants for step hp->step: each computed in double and
+// rounded once to float; `inv` multiplies the incoming gradient.
+inline Consts adam_consts(const zero_adam_hparams_t* hp, float inv) {
+    const double t = static_cast<double>(hp->step);
+    Consts c{};
+    c.lr = hp->lr;
+    c.b1 = hp->beta1;
+    c.b2 = hp->beta2;
+    c.eps = hp->eps;
+    c.inv = inv;
+    c.omb1 = static_cast<float>(1.0 - static_cast<double>(hp->beta1));
+    c.omb2 = static_cast<float>(1.0 - static_cast<double>(hp->beta2));
+    c.rbc1 = static_cast<float>(1.0 / (1.0 - std::pow(static_cast<double>(hp->beta1), t)));
+    c.rsbc2 = static_cast<float>(1.0 / std::sqrt(1.0 - std::pow(static_cast<double>(hp->beta2), t)));
+    c.decay = static_cast<float>(1.0 - static_cast<double>(hp->lr) * static_cast<double>(hp->weight_decay));
+    c.clip = 1.0f;
+    return c;
+}
+
 // Validate the arguments of a fused-step call and build its kernel
 // parameters and grid size.  `workspace` is the scratch used for the
 // gradient norm (ticket + per-block partials).  On success *blocks_out is the
@@ -185,11 +220,7 @@ inline int prepare_step(const char* fn, const void* const* grad_bufs, int32_t wo
         return fail(ZERO_ERR_RANGE, "%s: partition %d outside 0..%d", fn, partition, world - 1);
     if ((grad_dtype != ZERO_F16 && grad_dtype != ZERO_BF16) || (param_dtype != ZERO_F16 && param_dtype != ZERO_BF16))
         return fail(ZERO_ERR_DTYPE, "%s: gradients and parameters must be ZERO_F16 or ZERO_BF16", fn);
-    if (!(hp->step >= 1)) return fail(ZERO_ERR_ARG, "%s: hp->step must be >= 1", fn);
-    if (!std::isfinite(hp->lr) || !std::isfinite(hp->eps) || !std::isfinite(hp->weight_decay) ||
-        !(hp->beta1 >= 0.0f && hp->beta1 < 1.0f) || !(hp->beta2 >= 0.0f && hp->beta2 < 1.0f) ||
-        !(hp->grad_divisor >= 0.0f) || !std::isfinite(hp->grad_divisor))
-        return fail(ZERO_ERR_ARG, "%s: hyper-parameters out of range", fn);
+    if (int rc = check_hparams(fn, hp)) return rc;
     if (!(loss_scale > 0.0f) || !std::isfinite(loss_scale))
         return fail(ZERO_ERR_ARG, "%s: loss_scale must be positive and finite", fn);
     if (grad_sqnorm && !workspace) return fail(ZERO_ERR_ARG, "%s: grad_sqnorm needs a workspace", fn);
@@ -251,20 +282,8 @@ inline int prepare_step(const char* fn, const void* const* grad_bufs, int32_t wo
         prm.ticket = static_cast<unsigned int*>(workspace);
         prm.partials = reinterpret_cast<double*>(static_cast<char*>(workspace) + kWsPartialsOffset);
     }
-    // constants: double, rounded once to float
     const double divisor = hp->grad_divisor > 0.0f ? static_cast<double>(hp->grad_divisor) : static_cast<double>(world);
-    const double t = static_cast<double>(hp->step);
-    prm.c.lr = hp->lr;
-    prm.c.b1 = hp->beta1;
-    prm.c.b2 = hp->beta2;
-    prm.c.eps = hp->eps;
-    prm.c.inv = static_cast<float>(1.0 / (divisor * static_cast<double>(loss_scale)));
-    prm.c.omb1 = static_cast<float>(1.0 - static_cast<double>(hp->beta1));
-    prm.c.omb2 = static_cast<float>(1.0 - static_cast<double>(hp->beta2));
-    prm.c.rbc1 = static_cast<float>(1.0 / (1.0 - std::pow(static_cast<double>(hp->beta1), t)));
-    prm.c.rsbc2 = static_cast<float>(1.0 / std::sqrt(1.0 - std::pow(static_cast<double>(hp->beta2), t)));
-    prm.c.decay = static_cast<float>(1.0 - static_cast<double>(hp->lr) * static_cast<double>(hp->weight_decay));
-    prm.c.clip = 1.0f;
+    prm.c = adam_consts(hp, static_cast<float>(1.0 / (divisor * static_cast<double>(loss_scale))));
     prm.gate = nullptr;
     prm.clip_sqnorm = nullptr;
     prm.max_norm = 0.0;
@@ -307,13 +326,13 @@ inline int prepare_step(const char* fn, const void* const* grad_bufs, int32_t wo
 }
 
 // SM count, and the statistics pipeline kernel's shared-memory limit.
-inline int stats_pipe_setup(zero_dtype_t g, int* sms) {
-    const int which = static_cast<int>(g);
+inline int stats_pipe_setup(zero_dtype_t g, bool write, int* sms) {
+    const int which = static_cast<int>(g) * 2 + (write ? 1 : 0);
     std::lock_guard<std::mutex> lk(g_dev_mu);
     DeviceInfo* d = nullptr;
     if (int rc = device_info(&d)) return rc;
     if (!d->stats_pipe_ready[which]) {
-        cudaError_t e = cudaFuncSetAttribute(pick_stats_pipe_kernel(g), cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(pick_stats_pipe_kernel(g, write), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(kPipeSmemMax));
         if (e != cudaSuccess) return fail(ZERO_ERR_CUDA, "cannot raise the shared-memory limit: %s", cudaGetErrorString(e));
         d->stats_pipe_ready[which] = true;
@@ -326,8 +345,8 @@ inline int stats_pipe_setup(zero_dtype_t g, int* sms) {
 // pointers stay NULL: the statistics kernel reads gradients only).
 inline int prepare_stats(const char* fn, const void* const* grad_bufs, int32_t world, int64_t padded_numel,
                          int32_t partition, zero_dtype_t grad_dtype, float loss_scale, float grad_divisor,
-                         int32_t* overflow_flag, double* grad_sqnorm, void* workspace, StepParams* prm_out,
-                         int64_t* blocks_out) {
+                         const float* reduced, int32_t* overflow_flag, double* grad_sqnorm, void* workspace,
+                         StepParams* prm_out, int64_t* blocks_out) {
     if (!grad_bufs || !overflow_flag) return fail(ZERO_ERR_ARG, "%s: NULL grad_bufs or overflow_flag", fn);
     if (world < 1 || world > ZERO_MAX_WORLD)
         return fail(ZERO_ERR_ARG, "%s: world %d outside 1..%d", fn, world, ZERO_MAX_WORLD);
@@ -353,6 +372,12 @@ inline int prepare_stats(const char* fn, const void* const* grad_bufs, int32_t w
     const int64_t P = padded_numel / world;
     const int64_t begin = partition == ZERO_ALL_PARTITIONS ? 0 : static_cast<int64_t>(partition) * P;
     const int64_t count = partition == ZERO_ALL_PARTITIONS ? padded_numel : P;
+    if (reduced) {
+        if (!aligned(reduced, 4)) return fail(ZERO_ERR_ALIGN, "%s: reduced_out not 4-byte aligned", fn);
+        for (int k = 0; k < world; ++k)
+            if (overlaps(reduced, count * 4, grad_bufs[k], padded_numel * 2))
+                return fail(ZERO_ERR_ARG, "%s: reduced_out overlaps grad_bufs[%d]", fn, k);
+    }
     if (count == 0) {
         *blocks_out = 0;
         return ZERO_OK;
@@ -370,10 +395,11 @@ inline int prepare_stats(const char* fn, const void* const* grad_bufs, int32_t w
     const double divisor = grad_divisor > 0.0f ? static_cast<double>(grad_divisor) : static_cast<double>(world);
     prm.c.inv = static_cast<float>(1.0 / (divisor * static_cast<double>(loss_scale)));
     prm.c.clip = 1.0f;
-    // gradients only: the first element at which every replica is 16-byte aligned
+    // the first element at which every replica (and the reduced output) is
+    // 16-byte aligned
     int64_t h = -1;
     for (int64_t c = 0; c < kVec && h < 0; ++c) {
-        bool good = true;
+        bool good = !reduced || ((reinterpret_cast<uintptr_t>(reduced) + 4 * c) % 16) == 0;
         for (int k = 0; k < world && good; ++k)
             good = ((reinterpret_cast<uintptr_t>(prm.grads[k]) + 2 * c) % 16) == 0;
         if (good) h = c;
@@ -390,7 +416,7 @@ inline int prepare_stats(const char* fn, const void* const* grad_bufs, int32_t w
     const int tile = h >= 0 ? stats_pipe_tile(world) : 0;
     if (tile > 0) {
         int sms = 0;
-        if (int rc = stats_pipe_setup(grad_dtype, &sms)) return rc;
+        if (int rc = stats_pipe_setup(grad_dtype, reduced != nullptr, &sms)) return rc;
         const int64_t ntiles = (count - h) / tile;
         if (ntiles >= 2 * static_cast<int64_t>(sms)) {
             prm.tile = tile;
@@ -400,7 +426,7 @@ inline int prepare_stats(const char* fn, const void* const* grad_bufs, int32_t w
     }
     if (prm.tile == 0) {
         int limit = 0;
-        if (int rc = stats_grid_limit(grad_dtype, &limit)) return rc;
+        if (int rc = stats_grid_limit(grad_dtype, reduced != nullptr, &limit)) return rc;
         const int64_t work = prm.nvec > 0 ? prm.nvec : count;
         blocks = (work + kThreads - 1) / kThreads;
         if (blocks > limit) blocks = limit;
@@ -411,15 +437,18 @@ inline int prepare_stats(const char* fn, const void* const* grad_bufs, int32_t w
     return ZERO_OK;
 }
 
+// Enqueue the statistics kernel prepared by prepare_stats; `reduced` is the
+// same pointer prepare_stats saw (NULL: statistics only).
 inline int launch_stats(const char* fn, const StepParams& prm, int64_t blocks, zero_dtype_t grad_dtype,
-                        zero_stream_t stream) {
+                        float* reduced, zero_stream_t stream) {
     if (blocks == 0) return ok();
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const bool write = reduced != nullptr;
     if (prm.tile > 0) {
-        pick_stats_pipe_kernel(grad_dtype)<<<static_cast<unsigned int>(blocks), kPipeThreads,
-                                             stats_pipe_smem_bytes(prm.world, prm.tile), s>>>(prm);
+        pick_stats_pipe_kernel(grad_dtype, write)<<<static_cast<unsigned int>(blocks), kPipeThreads,
+                                                    stats_pipe_smem_bytes(prm.world, prm.tile), s>>>(prm, reduced);
     } else {
-        pick_stats_kernel(grad_dtype)<<<static_cast<unsigned int>(blocks), kThreads, 0, s>>>(prm);
+        pick_stats_kernel(grad_dtype, write)<<<static_cast<unsigned int>(blocks), kThreads, 0, s>>>(prm, reduced);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(ZERO_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));

@@ -14,8 +14,14 @@ bucket.  Two ways to run a step, both with an exact skip on overflow:
     overflow flag, squared norm) and then the update in place, gated on the
     device by that flag: one bank, the pages' 12 Psi/N, for 4N + 26 bytes per
     element.
+  mode="staged": the reduce-scatter stores every bucket's reduced fp32
+    gradients (with the flag and norm), then the in-place update reads them,
+    gated by that flag: one bank plus 4 bytes per element of reduced
+    gradients, for 2N + 34 bytes per element (ZeRO explainer, "Stage 2 -
+    Gradient Partitioning": each rank keeps the reduced gradients of its own
+    partition).
 
-max_grad_norm (either mode) clips the unscaled gradients to that global
+max_grad_norm (any mode) clips the unscaled gradients to that global
 norm, with the coefficient computed on the device from the statistics pass
 (banks mode then also takes the two-pass route).
 
@@ -28,9 +34,9 @@ from __future__ import annotations
 
 import torch
 
-from . import (ZERO_ALL_PARTITIONS, Runner, hparams, zero_flatten_bucket, zero_grad_stats, zero_loss_scale_update,
-               zero_partition_layout, zero_reduce_scatter_adam_step, zero_reduce_scatter_adam_step_gated,
-               zero_step_workspace_bytes)
+from . import (ZERO_ALL_PARTITIONS, Runner, hparams, zero_adam_step_reduced, zero_flatten_bucket, zero_grad_stats,
+               zero_loss_scale_update, zero_partition_layout, zero_reduce_scatter_adam_step,
+               zero_reduce_scatter_adam_step_gated, zero_reduce_scatter_grads, zero_step_workspace_bytes)
 
 
 class ZeroAdam:
@@ -40,12 +46,12 @@ class ZeroAdam:
                  growth_interval: int = 1000, min_scale: float = 1.0, grad_divisor: float = 0.0,
                  track_grad_norm: bool = False, mode: str = "banks", max_grad_norm: float | None = None,
                  device="cuda"):
-        if mode not in ("banks", "inplace"):
-            raise ValueError("mode must be 'banks' or 'inplace'")
+        if mode not in ("banks", "inplace", "staged"):
+            raise ValueError("mode must be 'banks', 'inplace' or 'staged'")
         if max_grad_norm is not None and not max_grad_norm > 0:
             raise ValueError("max_grad_norm must be positive")
         self.mode, self.max_grad_norm = mode, max_grad_norm
-        self.two_pass = mode == "inplace" or max_grad_norm is not None
+        self.two_pass = mode != "banks" or max_grad_norm is not None
         self.layout = zero_partition_layout(list(numels), world, bucket_elems, align_elems)
         self.world = world
         self.device = torch.device(device)
@@ -57,7 +63,7 @@ class ZeroAdam:
         self.cur = 0
         L, dev = self.layout, self.device
         f32 = dict(dtype=torch.float32, device=dev)
-        nbank = 1 if mode == "inplace" else 2
+        nbank = 2 if mode == "banks" else 1
         self.master = [[torch.zeros(L.bucket_padded[b], **f32) for _ in range(nbank)] for b in range(L.n_buckets)]
         self.m = [[torch.zeros(L.bucket_padded[b], **f32) for _ in range(nbank)] for b in range(L.n_buckets)]
         self.v = [[torch.zeros(L.bucket_padded[b], **f32) for _ in range(nbank)] for b in range(L.n_buckets)]
@@ -65,6 +71,9 @@ class ZeroAdam:
                             for b in range(L.n_buckets)]
         self.grads = [[torch.zeros(L.bucket_padded[b], dtype=grad_dtype, device=dev) for _ in range(world)]
                       for b in range(L.n_buckets)]
+        # staged mode: every rank's reduced fp32 gradient partition, per bucket
+        self.reduced = ([torch.zeros(L.bucket_padded[b], **f32) for b in range(L.n_buckets)]
+                        if mode == "staged" else None)
         # flags[0]: the step's overflow flag (read by the host, the gate of
         # the two-pass update); flags[1]: the gated update's own flag
         self.flags = torch.zeros(2, dtype=torch.int32, device=dev)
@@ -158,19 +167,33 @@ class ZeroAdam:
                 on_launch(b, "after")
 
     def _launch_two_pass(self, hp, on_launch, before_bucket=None) -> None:
-        """Statistics over every bucket, then the gated (and clipped) update."""
+        """Statistics (or the staged reduce-scatter) over every bucket, then
+        the gated (and clipped) update."""
         L = self.layout
         for b in range(L.n_buckets):
             if before_bucket is not None:
                 before_bucket(b)
-            zero_grad_stats(self.grads[b], L.bucket_padded[b], ZERO_ALL_PARTITIONS, self.scale, self.flag,
-                            self.sqnorm, self.workspace, self.grad_divisor)
+            if self.mode == "staged":
+                zero_reduce_scatter_grads(self.grads[b], L.bucket_padded[b], ZERO_ALL_PARTITIONS, self.scale,
+                                          self.reduced[b], self.flag, self.sqnorm, self.workspace,
+                                          self.grad_divisor)
+            else:
+                zero_grad_stats(self.grads[b], L.bucket_padded[b], ZERO_ALL_PARTITIONS, self.scale, self.flag,
+                                self.sqnorm, self.workspace, self.grad_divisor)
         c = self.cur
-        n = c if self.mode == "inplace" else c ^ 1
+        n = c ^ 1 if self.mode == "banks" else c
         clip = self.sqnorm if self.max_grad_norm is not None else None
         for b in range(L.n_buckets):
             if on_launch is not None:
                 on_launch(b, "before")
+            if self.mode == "staged":
+                zero_adam_step_reduced(
+                    self.reduced[b], L.bucket_padded[b], self.master[b][c], self.m[b][c], self.v[b][c],
+                    self.master[b][n], self.m[b][n], self.v[b][n], self.params_bank[b][n],
+                    hp, gate=self.flag, clip_sqnorm=clip, max_norm=self.max_grad_norm or 0.0)
+                if on_launch is not None:
+                    on_launch(b, "after")
+                continue
             zero_reduce_scatter_adam_step_gated(
                 self.grads[b], L.bucket_padded[b], ZERO_ALL_PARTITIONS,
                 self.master[b][c], self.m[b][c], self.v[b][c],
