@@ -332,18 +332,22 @@ int zero_reduce_scatter_grads(const void* const* grad_bufs, int32_t world, int64
  *               zero_reduce_scatter_adam_step, `count` elements each
  *               (hp->grad_divisor is not used: the gradients are already
  *               unscaled); in place when each *_out equals its *_in
+ * status        device int32, required: bit 1 (value 2) is OR-ed in when
+ *               the kernel's copy pipeline gave up waiting (then the
+ *               outputs are incomplete; see zero_reduce_scatter_adam_step);
+ *               otherwise untouched.  Must not be `gate`.
  * gate, clip_sqnorm, max_norm: as for zero_reduce_scatter_adam_step_gated
  *               (pass the flag and the norm of the step's
  *               zero_reduce_scatter_grads calls: an overflowing step then
  *               writes nothing)
- * No flag or norm is produced.
+ * No overflow flag or norm is produced (the reduce-scatter made them).
  * Errors: ZERO_ERR_ARG, ZERO_ERR_DTYPE, ZERO_ERR_ALIGN, ZERO_ERR_CUDA.
  */
 int zero_adam_step_reduced(const float* reduced_grad, int64_t count,
                            const float* master_in, const float* m_in, const float* v_in,
                            float* master_out, float* m_out, float* v_out,
                            void* param_out, zero_dtype_t param_dtype,
-                           const zero_adam_hparams_t* hp,
+                           const zero_adam_hparams_t* hp, int32_t* status,
                            const int32_t* gate, const double* clip_sqnorm, float max_norm,
                            zero_stream_t stream);
 

@@ -159,8 +159,8 @@ def _reduced_call(**kw):
     hp = kw.get("hp", Z.hparams())
     return Z.lib.zero_adam_step_reduced(
         kw.get("red", base + 0x100_0000 * 12), kw.get("n", 64), f(1), f(2), f(3), f(4), f(5), f(6), f(7),
-        kw.get("pd", 0), None if hp is None else ctypes.byref(hp), kw.get("gate", None), kw.get("clip", None),
-        kw.get("max_norm", 0.0), None)
+        kw.get("pd", 0), None if hp is None else ctypes.byref(hp), kw.get("status", base + 0x100_0000 * 13),
+        kw.get("gate", None), kw.get("clip", None), kw.get("max_norm", 0.0), None)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -177,6 +177,9 @@ def _reduced_call(**kw):
     (dict(p5=0x7100_0000), -1),                     # m_out is master_in
     (dict(gate=0x7D00_0002), -2),                   # misaligned gate
     (dict(clip=0x7E00_0000, max_norm=0.0), -1),     # clipping without a positive max_norm
+    (dict(status=0), -1),                           # NULL status
+    (dict(status=0x7D00_0001), -2),                 # misaligned status
+    (dict(gate=0x7D00_0000, status=0x7D00_0000), -1),   # gate is the status word
 ])
 def test_reduced_update_rejects_bad_arguments(kw, code):
     assert _reduced_call(**kw) == code

@@ -7,7 +7,8 @@ update from it must equal the oracle's step on the same inputs bit for bit,
 in and out of place, gated and clipped.  Sizes cover the register and the
 pipeline statistics kernels (N <= 20 and enough tiles), ragged tails,
 single partitions, bf16, a reduced buffer off the gradients' 16-byte phase
-(scalar path) and N up to 64.
+(scalar path), N up to 64, and sizes that take the update's pipeline
+kernel (at least two 6144-element tiles per SM).
 """
 import numpy as np
 import pytest
@@ -29,7 +30,7 @@ class Staged(Case):
     def __init__(self, *a, roff=0, **k):
         super().__init__(*a, norm=True, **k)
         self.red = Guarded(self.n, torch.float32, roff)
-        self.divisor = 0.0
+        self.status = torch.zeros(1, dtype=torch.int32, device="cuda")
 
     def reduce_scatter(self, divisor=0.0):
         Z.zero_reduce_scatter_grads([g.t for g in self.g_dev], self.padded, self.partition, self.scale,
@@ -40,8 +41,10 @@ class Staged(Case):
 
     def update(self, adam, t=1, gate=None, clip_sqnorm=None, max_norm=0.0):
         Z.zero_adam_step_reduced(self.red.t, self.n, *[b.t for b in self.in_dev], *[b.t for b in self.out_dev],
-                                 self.p_dev.t, _hp(adam, t), gate=gate, clip_sqnorm=clip_sqnorm, max_norm=max_norm)
+                                 self.p_dev.t, _hp(adam, t), self.status, gate=gate, clip_sqnorm=clip_sqnorm,
+                                 max_norm=max_norm)
         torch.cuda.synchronize()
+        assert int(self.status.item()) == 0
         for b in self.in_dev + list(self.out_dev) + [self.p_dev, self.red]:
             b.check()
 
@@ -68,6 +71,10 @@ CASES = [
     (4, 4 * 20_011, oracle.F16, -1, 3, 0),
     (4, 4 * 20_011, oracle.F16, -1, 0, 1),
     (64, 64 * 4099, oracle.F16, -1, 0, 0),
+    # >= 2 x 148 update tiles of 6144: the update's pipeline kernel
+    (4, 4 * 600_007, oracle.F16, -1, 0, 0),
+    (2, 2 * 1_000_003, oracle.BF16, -1, 0, 0),
+    (2, 2 * 1_900_003, oracle.F16, 1, 0, 0),
 ]
 
 
@@ -115,7 +122,7 @@ def test_staged_step_equals_oracle_step(world, padded, gd, part, goff, roff, inp
 def test_staged_update_from_oracle_reduced_input():
     """The update alone, fed the oracle's reduced gradients (uploaded, not
     produced by the GPU reduce-scatter), against the oracle's update."""
-    world, padded = 4, 4 * 300_007
+    world, padded = 4, 4 * 600_007
     c = Staged(padded, world, seed=560, scale=4096.0, pdtype=oracle.BF16)
     s, inv, g = c.oracle_reduced()
     to_dev_f32(g, buf=c.red)
@@ -126,7 +133,7 @@ def test_staged_update_from_oracle_reduced_input():
 
 
 def test_staged_gate_writes_nothing():
-    world, padded = 8, 8 * 100_003
+    world, padded = 8, 8 * 250_003
     c = Staged(padded, world, seed=570, scale=65536.0, inplace=True)
     workloads.inject(c.G[0], np.array([5]), np.array([False]))
     to_dev_u16(c.G[0], torch.float16, buf=c.g_dev[0])
@@ -140,7 +147,7 @@ def test_staged_gate_writes_nothing():
 
 
 def test_staged_clip_matches_oracle():
-    world, padded = 8, 8 * 200_003
+    world, padded = 8, 8 * 250_003
     c = Staged(padded, world, seed=580, scale=65536.0)
     c.reduce_scatter()
     s, inv, _ = c.oracle_reduced()

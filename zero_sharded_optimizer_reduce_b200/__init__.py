@@ -108,7 +108,7 @@ def _load():
                                             vp, vp]
     L.zero_reduce_scatter_grads.restype = ctypes.c_int
     L.zero_adam_step_reduced.argtypes = [vp, i64, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int,
-                                         ctypes.POINTER(AdamHParams), vp, vp, f32, vp]
+                                         ctypes.POINTER(AdamHParams), vp, vp, vp, f32, vp]
     L.zero_adam_step_reduced.restype = ctypes.c_int
     L.zero_ipc_export.argtypes = [vp, ctypes.POINTER(IpcHandle), ctypes.POINTER(i64)]
     L.zero_ipc_export.restype = ctypes.c_int
@@ -317,13 +317,14 @@ def zero_reduce_scatter_grads(grad_bufs, padded_numel: int, partition: int, loss
 
 
 def zero_adam_step_reduced(reduced_grad, count: int, master_in, m_in, v_in, master_out, m_out, v_out, param_out,
-                           hp: AdamHParams, gate=None, clip_sqnorm=None, max_norm: float = 0.0,
+                           hp: AdamHParams, status, gate=None, clip_sqnorm=None, max_norm: float = 0.0,
                            stream=None) -> None:
-    """Staged update: Adam on `count` elements from fp32 reduced gradients (gated, optionally clipped)."""
+    """Staged update: Adam on `count` elements from fp32 reduced gradients (gated, optionally clipped);
+    `status` (device int32) receives bit 1 if the kernel's copy pipeline timed out."""
     _check(lib.zero_adam_step_reduced(
         _ptr(reduced_grad), count, _ptr(master_in), _ptr(m_in), _ptr(v_in), _ptr(master_out), _ptr(m_out),
-        _ptr(v_out), _ptr(param_out), _dtype_code(param_out), ctypes.byref(hp), _ptr(gate), _ptr(clip_sqnorm),
-        float(max_norm), _stream(stream)))
+        _ptr(v_out), _ptr(param_out), _dtype_code(param_out), ctypes.byref(hp), _ptr(status), _ptr(gate),
+        _ptr(clip_sqnorm), float(max_norm), _stream(stream)))
 
 
 def zero_allgather_params(shards, shard_offset: int, part_numel: int, dst, stream=None) -> None:

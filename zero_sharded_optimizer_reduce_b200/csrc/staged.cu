@@ -17,30 +17,57 @@ namespace zero {
 namespace fused {
 namespace {
 
+// Tile of the pipeline kernel: 4 fp32 arrays x 4096 elements per stage
+// (64 KB), 2 rounds of one 4-element chunk per consumer thread.  Measured on
+// B200 (GPT-2 1.5B buckets): 6305 GB/s; 6144-element tiles 6092 GB/s.
+constexpr int kReducedTile = 4096;
+
+inline uint32_t reduced_pipe_smem_bytes(int tile) {
+    return static_cast<uint32_t>(kReducedStages) * 16u * static_cast<uint32_t>(tile);
+}
+
 inline KernelFn pick_reduced_kernel(zero_dtype_t pd) {
     return pd == ZERO_F16 ? adam_reduced_kernel<__half> : adam_reduced_kernel<__nv_bfloat16>;
 }
 
-std::mutex g_red_mu;
-int g_red_blocks[64][2] = {};
+inline KernelFn pick_reduced_pipe_kernel(zero_dtype_t pd) {
+    return pd == ZERO_F16 ? adam_reduced_pipe_kernel<__half> : adam_reduced_pipe_kernel<__nv_bfloat16>;
+}
 
-inline int reduced_grid_limit(zero_dtype_t pd, int* out) {
+struct ReducedDevice {
+    int sms = 0;
+    int blocks_per_sm[2] = {0, 0};
+    bool pipe_ready[2] = {false, false};
+};
+
+std::mutex g_red_mu;
+ReducedDevice g_red[64];
+
+// SM count, resident blocks of the register kernel, and the pipeline
+// kernel's shared-memory limit, queried or set once per device and dtype.
+inline int reduced_device(zero_dtype_t pd, ReducedDevice** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return fail(ZERO_ERR_CUDA, "cudaGetDevice failed");
     std::lock_guard<std::mutex> lk(g_red_mu);
-    int& per_sm = g_red_blocks[dev][pd == ZERO_F16 ? 0 : 1];
-    static int sms[64] = {};
-    if (sms[dev] == 0 && cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    ReducedDevice& d = g_red[dev];
+    const int w = pd == ZERO_F16 ? 0 : 1;
+    if (d.sms == 0 && cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        d.sms = 0;
         return fail(ZERO_ERR_CUDA, "cannot query the SM count");
-    if (per_sm == 0) {
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pick_reduced_kernel(pd), kThreads, 0);
-        if (e != cudaSuccess || per_sm < 1) {
-            per_sm = 0;
-            return fail(ZERO_ERR_CUDA, "occupancy query failed: %s", cudaGetErrorString(e));
-        }
     }
-    const int lim = sms[dev] * per_sm;
-    *out = lim < kMaxBlocks ? lim : kMaxBlocks;
+    if (d.blocks_per_sm[w] == 0) {
+        int n = 0;
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, pick_reduced_kernel(pd), kThreads, 0);
+        if (e != cudaSuccess || n < 1) return fail(ZERO_ERR_CUDA, "occupancy query failed: %s", cudaGetErrorString(e));
+        d.blocks_per_sm[w] = n;
+    }
+    if (!d.pipe_ready[w]) {
+        cudaError_t e = cudaFuncSetAttribute(pick_reduced_pipe_kernel(pd), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(reduced_pipe_smem_bytes(kReducedTile)));
+        if (e != cudaSuccess) return fail(ZERO_ERR_CUDA, "cannot raise the shared-memory limit: %s", cudaGetErrorString(e));
+        d.pipe_ready[w] = true;
+    }
+    *out = &d;
     return ZERO_OK;
 }
 
@@ -111,6 +138,7 @@ inline int prepare_reduced(const char* fn, const float* reduced, int64_t count, 
         prm.head = h;
         prm.nvec = (count - h) / kVec;
     }
+    prm.tile = 0;
     *prm_out = prm;
     *work_out = prm.nvec > 0 ? prm.nvec : count;
     return ZERO_OK;
@@ -140,23 +168,38 @@ extern "C" int zero_reduce_scatter_grads(const void* const* grad_bufs, int32_t w
 extern "C" int zero_adam_step_reduced(const float* reduced_grad, int64_t count, const float* master_in,
                                       const float* m_in, const float* v_in, float* master_out, float* m_out,
                                       float* v_out, void* param_out, zero_dtype_t param_dtype,
-                                      const zero_adam_hparams_t* hp, const int32_t* gate, const double* clip_sqnorm,
-                                      float max_norm, zero_stream_t stream) {
+                                      const zero_adam_hparams_t* hp, int32_t* status, const int32_t* gate,
+                                      const double* clip_sqnorm, float max_norm, zero_stream_t stream) {
     using namespace zero::fused;
     const char* fn = "zero_adam_step_reduced";
+    if (!status) return fail(ZERO_ERR_ARG, "%s: NULL status", fn);
+    if (!zero::aligned(status, 4)) return fail(ZERO_ERR_ALIGN, "%s: status misaligned", fn);
     StepParams prm{};
     int64_t work = 0;
     if (int rc = prepare_reduced(fn, reduced_grad, count, master_in, m_in, v_in, master_out, m_out, v_out, param_out,
                                  param_dtype, hp, &prm, &work))
         return rc;
+    prm.overflow = status;
     if (int rc = add_gate_and_clip(fn, &prm, gate, clip_sqnorm, max_norm)) return rc;
     if (work == 0) return zero::ok();
-    int limit = 0;
-    if (int rc = reduced_grid_limit(param_dtype, &limit)) return rc;
-    int64_t blocks = (work + kThreads - 1) / kThreads;
-    if (blocks > limit) blocks = limit;
-    pick_reduced_kernel(param_dtype)<<<static_cast<unsigned int>(blocks), kThreads, 0,
-                                       reinterpret_cast<cudaStream_t>(stream)>>>(prm);
+    ReducedDevice* d = nullptr;
+    if (int rc = reduced_device(param_dtype, &d)) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t ntiles = prm.nvec > 0 ? (count - prm.head) / kReducedTile : 0;
+    if (ntiles >= 2 * static_cast<int64_t>(d->sms)) {
+        // the pipeline kernel takes the whole tiles; the rest goes through
+        // its scalar path
+        prm.tile = kReducedTile;
+        prm.nvec = ntiles * kReducedTile / kVec;
+        pick_reduced_pipe_kernel(param_dtype)<<<static_cast<unsigned int>(d->sms), kPipeThreads,
+                                                reduced_pipe_smem_bytes(kReducedTile), s>>>(prm);
+    } else {
+        const int64_t limit = static_cast<int64_t>(d->sms) * d->blocks_per_sm[param_dtype == ZERO_F16 ? 0 : 1];
+        int64_t blocks = (work + kThreads - 1) / kThreads;
+        if (blocks > limit) blocks = limit;
+        if (blocks > kMaxBlocks) blocks = kMaxBlocks;
+        pick_reduced_kernel(param_dtype)<<<static_cast<unsigned int>(blocks), kThreads, 0, s>>>(prm);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(ZERO_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
     return zero::ok();

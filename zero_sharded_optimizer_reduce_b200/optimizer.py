@@ -190,7 +190,7 @@ class ZeroAdam:
                 zero_adam_step_reduced(
                     self.reduced[b], L.bucket_padded[b], self.master[b][c], self.m[b][c], self.v[b][c],
                     self.master[b][n], self.m[b][n], self.v[b][n], self.params_bank[b][n],
-                    hp, gate=self.flag, clip_sqnorm=clip, max_norm=self.max_grad_norm or 0.0)
+                    hp, self.flags[1:2], gate=self.flag, clip_sqnorm=clip, max_norm=self.max_grad_norm or 0.0)
                 if on_launch is not None:
                     on_launch(b, "after")
                 continue
