@@ -136,29 +136,36 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def source_digest() -> str:
-    """Hash of the step kernels' source, comments and whitespace removed, so
-    that the recorded ncu traffic is dropped only when the code changes."""
+def source_digest(files=("fused_step.cuh",)) -> str:
+    """Hash of kernel sources, comments and whitespace removed, so that the
+    recorded ncu traffic is dropped only when the code changes."""
     import re
-    p = os.path.join(ROOT, "zero_sharded_optimizer_reduce_b200", "csrc", "fused_step.cuh")
-    with open(p) as f:
-        text = f.read()
+    text = ""
+    for name in files:
+        with open(os.path.join(ROOT, "zero_sharded_optimizer_reduce_b200", "csrc", name)) as f:
+            text += f.read()
     text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
     text = re.sub(r"//[^\n]*", " ", text)
     text = " ".join(text.split())
     return hashlib.sha256(text.encode()).hexdigest()[:16]
 
 
-def profiled_traffic(elems_per_launch: float):
-    """DRAM bytes per launch of the fused kernel from the committed ncu summary,
-    if it was taken on the current kernel source; else None."""
-    p = os.path.join(ROOT, "profiles", "fused_step_traffic.json")
+# timed kernel -> (committed ncu traffic record, the sources it was taken on)
+TRAFFIC_RECORDS = {"fused": ("fused_step_traffic.json", ("fused_step.cuh",)),
+                   "staged": ("adam_reduced_traffic.json", ("fused_step.cuh", "staged.cuh"))}
+
+
+def profiled_traffic(elems_per_launch: float, kernel: str = "fused"):
+    """DRAM bytes per launch of the timed kernel from the committed ncu
+    summary, if it was taken on the current kernel source; else None."""
+    name, files = TRAFFIC_RECORDS[kernel]
+    p = os.path.join(ROOT, "profiles", name)
     try:
         with open(p) as f:
             d = json.load(f)
     except Exception:
         return None
-    if d.get("kernel_source_sha256_16") != source_digest():
+    if d.get("kernel_source_sha256_16") != source_digest(files):
         return None
     return float(d["dram_bytes_per_elem"]) * elems_per_launch
 
@@ -362,7 +369,8 @@ def run_gpu(args):
     kern_s = sum(launch_ms) * 1e-3
     achieved = kern_bytes / kern_s / 1e9
     avg_elems = sum(launch_elems) / len(launch_elems)
-    traffic = profiled_traffic(avg_elems) if args.mode == "banks" else None
+    traffic = (profiled_traffic(avg_elems, "staged") if args.mode == "staged" else
+               profiled_traffic(avg_elems) if args.mode == "banks" else None)
 
     # ---- end to end through the public API: host gradients in, flag out
     e2e = None
@@ -470,16 +478,18 @@ def run_sweep(args):
 
 def run_stage3(args):
     """Layer-wise ZeRO-3 step on the 6.7B GPT shape (32 layers + embedding
-    unit, N = 8): two gathers per unit plus the per-unit statistics and gated
-    in-place update, timed with and without gather prefetch.  One JSON line."""
+    unit, N = 8): two gathers per unit plus the per-unit staged reduce-scatter
+    and gated in-place update, timed with and without gather prefetch, and
+    with the statistics-pass update for comparison.  One JSON line."""
     import torch
     import zero_sharded_optimizer_reduce_b200 as Z
     torch.cuda.set_device(0)
     w = workloads.gpt_6p7b_layerwise()
     out = {}
-    for prefetch in (False, True):
+    for prefetch, update in ((False, "staged"), (True, "stats"), (True, "staged")):
         s3 = Z.ZeroStage3(w.numels, w.world, lr=w.adam.lr, betas=(w.adam.beta1, w.adam.beta2), eps=w.adam.eps,
-                          weight_decay=w.adam.weight_decay, loss_scale=w.loss_scale, prefetch=prefetch)
+                          weight_decay=w.adam.weight_decay, loss_scale=w.loss_scale, prefetch=prefetch,
+                          update=update)
         gen = torch.Generator(device="cuda")
         for u in range(s3.U):
             gen.manual_seed(4000 + u)
@@ -498,8 +508,8 @@ def run_stage3(args):
             s3.step()
         e1.record()
         torch.cuda.synchronize()
-        out[prefetch] = e0.elapsed_time(e1) / args.steps
-        if prefetch:
+        out[(prefetch, update)] = e0.elapsed_time(e1) / args.steps
+        if prefetch and update == "staged":
             # the all-gather alone: unit 0 from the 8 shards into a layer buffer
             for _ in range(3):
                 s3.unit_params(0, s3.layer[0][:s3.layout.bucket_padded[0]])
@@ -515,14 +525,20 @@ def run_stage3(args):
         torch.cuda.empty_cache()
     psi = sum(Z.zero_partition_layout(w.numels, w.world, 1, 8).bucket_padded)
     N = w.world
-    step_bytes = psi * (8 + 4 * N + 26)      # 2 gathers x (2 read + 2 write) + statistics + update
+    bpe = 8 + 2 * N + 34          # 2 gathers x (2 read + 2 write) + reduce-scatter to fp32 + update
+    bpe_stats = 8 + 4 * N + 26    # 2 gathers + statistics pass + fused gated update
+    best = out[(True, "staged")]
     peak, peak_kind = peaks()
-    line = {"metric": "ZeRO-3 layer-wise step (gathers + statistics + gated in-place update)", "unit": "Gparams/s",
-            "value": psi / (out[True] * 1e-3) / 1e9, "ms_per_step": out[True], "ms_per_step_no_prefetch": out[False],
-            "prefetch_gain": out[False] / out[True] - 1.0, "steps": args.steps, "warmup": args.warmup,
+    line = {"metric": "ZeRO-3 layer-wise step (gathers + staged reduce-scatter + gated in-place update)",
+            "unit": "Gparams/s", "value": psi / (best * 1e-3) / 1e9, "ms_per_step": best,
+            "ms_per_step_no_prefetch": out[(False, "staged")],
+            "prefetch_gain": out[(False, "staged")] / best - 1.0, "steps": args.steps, "warmup": args.warmup,
             "config": {"workload": w.name, "psi_padded": psi, "world": N, "units": len(w.numels)},
-            "hbm_gbs": step_bytes / (out[True] * 1e-3) / 1e9, "bytes_per_elem": 8 + 4 * N + 26,
-            "frac_measured": step_bytes / (out[True] * 1e-3) / 1e9 / peak, "peak_kind": peak_kind,
+            "hbm_gbs": psi * bpe / (best * 1e-3) / 1e9, "bytes_per_elem": bpe,
+            "frac_measured": psi * bpe / (best * 1e-3) / 1e9 / peak, "peak_kind": peak_kind,
+            "stats_update": {"ms_per_step": out[(True, "stats")], "bytes_per_elem": bpe_stats,
+                             "value": psi / (out[(True, "stats")] * 1e-3) / 1e9,
+                             "frac_measured": psi * bpe_stats / (out[(True, "stats")] * 1e-3) / 1e9 / peak},
             "allgather": {"elements": gather_elems, "ms": gather_ms, "bytes_per_elem": 4,
                           "gbs": gather_elems * 4 / (gather_ms * 1e-3) / 1e9,
                           "frac_measured": gather_elems * 4 / (gather_ms * 1e-3) / 1e9 / peak,

@@ -1,6 +1,8 @@
 """ZeroStage3 (layer-wise ZeRO-3 with gather prefetch) against the oracle.
 
-Per unit the update is the Stage-2 update of that unit's partitions, so the
+Per unit the update is the Stage-2 update of that unit's partitions (staged
+reduce-scatter + update from the reduced gradients, or statistics pass +
+fused gated update), so the
 oracle runs flat_step per unit; the parameters read back through the
 all-gather of the shards must equal the oracle's bit for bit.  Prefetch on
 and off give identical bits.  An overflow injected into one unit skips that
@@ -32,10 +34,10 @@ def _unit_grads(L, u, step, scale, inject=False):
     return out
 
 
-def _run(prefetch, inject_unit=None):
+def _run(prefetch, inject_unit=None, update="staged"):
     adam = workloads.AdamConfig(weight_decay=0.01)
     s3 = Z.ZeroStage3(UNITS, N, lr=adam.lr, betas=(adam.beta1, adam.beta2), eps=adam.eps,
-                      weight_decay=adam.weight_decay, loss_scale=65536.0, prefetch=prefetch)
+                      weight_decay=adam.weight_decay, loss_scale=65536.0, prefetch=prefetch, update=update)
     L = oracle.partition_layout(UNITS, N, 1, 8)
     init = [np.concatenate([workloads.master(n, 950 + u), np.zeros(L.bucket_padded[u] - n, np.float32)])
             for u, n in enumerate(UNITS)]
@@ -55,10 +57,11 @@ def _run(prefetch, inject_unit=None):
     return s3, L, init, results, params, states
 
 
+@pytest.mark.parametrize("update", ["staged", "stats"])
 @pytest.mark.parametrize("inject_unit", [None, 1])
-def test_stage3_matches_oracle_and_prefetch_is_exact(inject_unit):
-    s3a, L, init, res_a, par_a, st_a = _run(True, inject_unit)
-    s3b, _, _, res_b, par_b, st_b = _run(False, inject_unit)
+def test_stage3_matches_oracle_and_prefetch_is_exact(inject_unit, update):
+    s3a, L, init, res_a, par_a, st_a = _run(True, inject_unit, update)
+    s3b, _, _, res_b, par_b, st_b = _run(False, inject_unit, update)
     assert res_a == res_b
     for x, y in zip(par_a, par_b):
         assert np.array_equal(x, y)

@@ -12,9 +12,13 @@ Simulation on one GPU, per unit u (a transformer layer or the embedding):
   - fp32 master / m / v per unit in flat (rank-major) order, one bank;
   - N replica gradient buffers, reused by every unit; `grad_fill(u, bufs)`
     stands for the backward pass that produces unit u's gradients;
-  - the update of unit u: a statistics pass over the unit (overflow flag),
-    then one gated call per rank r updating slice r in place and writing the
-    new parameters into shard r's slot of unit u.
+  - the update of unit u, update="staged" (default): the reduce-scatter of
+    the unit stores every rank's reduced fp32 gradients (and the unit's
+    overflow flag) in a reused buffer, then one gated call per rank r updates
+    slice r in place from them and writes the new parameters into shard r's
+    slot of unit u: 2N + 34 bytes per element.  update="stats": a
+    statistics pass over the unit, then one gated fused call per rank that
+    re-reads the N replicas: 4N + 26 bytes per element.
 Step: forward gathers u = 0 .. U-1, then for u = U-1 .. 0: gather, gradients,
 update.  With prefetch, the gather of the next unit runs on a side stream
 into the other layer buffer while the current unit's work runs; events order
@@ -30,15 +34,18 @@ from __future__ import annotations
 
 import torch
 
-from . import (hparams, zero_allgather_params, zero_grad_stats, zero_loss_scale_update, zero_partition_layout,
-               zero_reduce_scatter_adam_step_gated)
+from . import (hparams, zero_adam_step_reduced, zero_allgather_params, zero_grad_stats, zero_loss_scale_update,
+               zero_partition_layout, zero_reduce_scatter_adam_step_gated, zero_reduce_scatter_grads)
 
 
 class ZeroStage3:
     def __init__(self, unit_numels, world: int, *, align_elems: int = 8, lr: float = 1e-3, betas=(0.9, 0.999),
                  eps: float = 1e-8, weight_decay: float = 0.0, grad_dtype=torch.float16,
                  param_dtype=torch.float16, loss_scale: float = 65536.0, growth_interval: int = 1000,
-                 min_scale: float = 1.0, prefetch: bool = True, device="cuda"):
+                 min_scale: float = 1.0, prefetch: bool = True, update: str = "staged", device="cuda"):
+        if update not in ("staged", "stats"):
+            raise ValueError("update must be 'staged' or 'stats'")
+        self.update_mode = update
         self.world = world
         self.layout = L = zero_partition_layout(list(unit_numels), world, 1, align_elems)   # one unit per bucket
         self.U = L.n_buckets
@@ -59,6 +66,7 @@ class ZeroStage3:
         self.v = [torch.zeros(L.bucket_padded[u], **f32) for u in range(self.U)]
         mx = max(L.bucket_padded)
         self.grads = [torch.zeros(mx, dtype=grad_dtype, device=dev) for _ in range(world)]
+        self.reduced = torch.zeros(mx, **f32) if update == "staged" else None
         self.layer = [torch.zeros(mx, dtype=param_dtype, device=dev) for _ in range(2)]
         self.unit_flags = torch.zeros(self.U, dtype=torch.int32, device=dev)
         self.step_flag = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -99,6 +107,16 @@ class ZeroStage3:
         pad = L.bucket_padded[u]
         g = [x[:pad] for x in self.grads]
         flag = self.unit_flags[u:u + 1]
+        if self.update_mode == "staged":
+            red = self.reduced[:pad]
+            zero_reduce_scatter_grads(g, pad, -1, self.scale, red, flag)
+            for r in range(self.world):
+                sl = slice(r * P, (r + 1) * P)
+                zero_adam_step_reduced(red[sl], P, self.master[u][sl], self.m[u][sl], self.v[u][sl],
+                                       self.master[u][sl], self.m[u][sl], self.v[u][sl],
+                                       self.shards[r][self.shard_off[u]:self.shard_off[u] + P],
+                                       hp, self.step_flag, gate=flag)
+            return
         zero_grad_stats(g, pad, -1, self.scale, flag)
         for r in range(self.world):
             sl = slice(r * P, (r + 1) * P)
