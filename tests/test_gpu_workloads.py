@@ -80,18 +80,20 @@ def _u16(t):
 
 
 @pytest.mark.skipif(not torch.cuda.is_available() or _free_gb() < 80, reason="needs ~70 GB of HBM")
-def test_gpt2_1p5b_windows_five_steps():
+@pytest.mark.parametrize("mode", ["banks", "staged"])
+def test_gpt2_1p5b_windows_five_steps(mode):
     w = workloads.gpt2_1p5b()
     opt = Z.ZeroAdam(w.numels, w.world, w.bucket_elems, lr=w.adam.lr, betas=(w.adam.beta1, w.adam.beta2),
-                     eps=w.adam.eps, weight_decay=w.adam.weight_decay, loss_scale=w.loss_scale)
+                     eps=w.adam.eps, weight_decay=w.adam.weight_decay, loss_scale=w.loss_scale, mode=mode)
     L = opt.layout
     wins, refs = [], []
     for b in range(L.n_buckets):
         _device_master(opt.master[b][0], 700 + b)
         opt.master[b][0][L.bucket_numel[b]:].zero_()
         opt.params_bank[b][0].copy_(opt.master[b][0])
-        opt.master[b][1].copy_(opt.master[b][0])
-        opt.params_bank[b][1].copy_(opt.params_bank[b][0])
+        for extra in range(1, len(opt.master[b])):
+            opt.master[b][extra].copy_(opt.master[b][0])
+            opt.params_bank[b][extra].copy_(opt.params_bank[b][0])
         wb = _windows(L.bucket_padded[b], w.world, n_random=16, seed=b)
         wins.append(wb)
         # the oracle's state on the windows, from the device's initial values
@@ -122,18 +124,20 @@ def test_gpt2_1p5b_windows_five_steps():
 
 
 @pytest.mark.skipif(not torch.cuda.is_available() or _free_gb() < 12, reason="needs ~8 GB of HBM")
-def test_overflow_workload_full_arrays():
+@pytest.mark.parametrize("mode", ["banks", "staged", "inplace"])
+def test_overflow_workload_full_arrays(mode):
     w = workloads.overflow_flat()
     (psi,) = w.numels
     N = w.world
     opt = Z.ZeroAdam([psi], N, lr=w.adam.lr, betas=(w.adam.beta1, w.adam.beta2), eps=w.adam.eps,
-                     weight_decay=w.adam.weight_decay, loss_scale=w.loss_scale, track_grad_norm=True)
+                     weight_decay=w.adam.weight_decay, loss_scale=w.loss_scale, track_grad_norm=True, mode=mode)
     padded = opt.layout.bucket_padded[0]
     assert padded == psi
     _device_master(opt.master[0][0], 900)
     opt.params_bank[0][0].copy_(opt.master[0][0])
-    opt.master[0][1].copy_(opt.master[0][0])
-    opt.params_bank[0][1].copy_(opt.params_bank[0][0])
+    for extra in range(1, len(opt.master[0])):
+        opt.master[0][extra].copy_(opt.master[0][0])
+        opt.params_bank[0][extra].copy_(opt.params_bank[0][0])
     ref = oracle.FlatState(host_f32(opt.master[0][0]).copy(), np.zeros(psi, np.float32),
                            np.zeros(psi, np.float32), _u16(opt.params_bank[0][0]).copy())
     scaler = oracle.Scaler(w.loss_scale)

@@ -1,6 +1,7 @@
 """Property-based tests (hypothesis, derandomized): random layouts through
 the C ABI against the oracle on the CPU, and random small configurations of
-the fused step on the GPU against the oracle, bit for bit."""
+the fused step and of the staged step (reduce-scatter to fp32, then the
+update from it) on the GPU against the oracle, bit for bit."""
 import numpy as np
 import pytest
 from hypothesis import given, settings
@@ -41,3 +42,31 @@ def test_step_matches_oracle(world, per_rank, dtypes, offs, part, inplace, wd, t
     c.run(adam, t=t)
     assert int(c.flag.item()) == ovf == 0
     assert c.compare(ref) == [0, 0, 0, 0]
+
+
+@pytest.mark.gpu
+@settings(max_examples=30, deadline=None, derandomize=True)
+@given(world=st.integers(1, 17), per_rank=st.integers(1, 5000),
+       dtypes=st.sampled_from([(oracle.F16, oracle.F16), (oracle.BF16, oracle.BF16), (oracle.F16, oracle.BF16)]),
+       offs=st.tuples(st.integers(0, 7), st.integers(0, 7), st.integers(0, 7), st.integers(0, 7)),
+       part=st.integers(-1, 16), inplace=st.booleans(), wd=st.sampled_from([0.0, 0.01]),
+       t=st.integers(1, 50), seed=st.integers(0, 10_000))
+def test_staged_step_matches_oracle(world, per_rank, dtypes, offs, part, inplace, wd, t, seed):
+    from test_gpu_staged import Staged
+    gd, pd = dtypes
+    partition = part if part < world else -1
+    c = Staged(world * per_rank, world, gdtype=gd, pdtype=pd, seed=seed, partition=partition, goff=offs[0],
+               soff=offs[1], poff=offs[2], roff=offs[3], inplace=inplace, scale=1024.0)
+    adam = workloads.AdamConfig(weight_decay=wd)
+    ref, ovf, _ = c.expect(adam, t=t)
+    c.reduce_scatter()
+    s, inv, g = c.oracle_reduced()
+    assert np.array_equal(host_reduced(c), g.view(np.uint32))
+    c.update(adam, t=t, gate=c.flag)
+    assert int(c.flag.item()) == ovf == 0
+    assert c.compare(ref) == [0, 0, 0, 0]
+
+
+def host_reduced(c):
+    from _gpu import host_f32
+    return host_f32(c.red.t).view(np.uint32)
