@@ -11,7 +11,9 @@ another rank).  Rank k writes replica k's gradients; the fused kernel of rank
 r reads slice r of every peer's buffer in rank order.  After every step each
 rank's partition of the fp32 states and its full gathered parameter buffer
 must equal the oracle's Stage 2 bit for bit, including a step where one rank
-injects inf / NaN and every rank skips.
+injects inf / NaN and every rank skips.  Both the fused route (two banks) and
+the staged route (one bank plus the reduced gradients; the update runs only
+after the group's verdict) are run.
 """
 import os
 import socket
@@ -55,7 +57,7 @@ def _initial(L):
     return [oracle.flatten_bucket(L, b, tensors, np.float32) for b in range(L.n_buckets)]
 
 
-def _rank_main(rank, world, align, port, outdir):
+def _rank_main(rank, world, align, port, outdir, mode="banks"):
     import sys
     sys.path.insert(0, ROOT)
     import datetime
@@ -67,7 +69,7 @@ def _rank_main(rank, world, align, port, outdir):
     try:
         adam = workloads.AdamConfig(weight_decay=0.01)
         opt = Z.DistributedZeroAdam(NUMELS, CAP, align, lr=adam.lr, betas=(adam.beta1, adam.beta2), eps=adam.eps,
-                                    weight_decay=adam.weight_decay, loss_scale=65536.0)
+                                    weight_decay=adam.weight_decay, loss_scale=65536.0, mode=mode)
         L = oracle.partition_layout(NUMELS, world, CAP, align)
         init = _initial(L)
         opt.load([torch.from_numpy(x).cuda() for x in init],
@@ -96,11 +98,12 @@ def _rank_main(rank, world, align, port, outdir):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,align", [(2, 8), (3, 1)])
-def test_multiprocess_zero2_matches_oracle(world, align, tmp_path):
+@pytest.mark.parametrize("world,align,mode", [(2, 8, "banks"), (3, 1, "banks"), (2, 8, "staged"), (3, 1, "staged")])
+def test_multiprocess_zero2_matches_oracle(world, align, mode, tmp_path):
     port = _free_port()
     ctx = mp.get_context("spawn")
-    procs = [ctx.Process(target=_rank_main, args=(r, world, align, port, str(tmp_path))) for r in range(world)]
+    procs = [ctx.Process(target=_rank_main, args=(r, world, align, port, str(tmp_path), mode))
+             for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:

@@ -16,6 +16,8 @@ benchmark times (every rank's partition in one launch per bucket).
   parameters into its own shard; windows against the oracle, whole gathered
   units bit-exact.
 - Flat bandwidth-sweep points: windows.
+- The staged route on a bucket past 2^31 elements (64-bit indexing) and on a
+  bf16 N = 16 point: windows of the reduced gradients, states, parameters.
 """
 import numpy as np
 import pytest
@@ -283,4 +285,47 @@ def test_sweep_points_windows(psi, world, dtype):
         assert assert_f32_close(host_f32(st_out["p"][lo:hi]), ref.master, "master") == 0
         assert assert_f32_close(host_f32(st_out["m"][lo:hi]), ref.m, "m") == 0
         assert assert_f32_close(host_f32(st_out["v"][lo:hi]), ref.v, "v") == 0
+        assert assert_u16_close(_u16(params[lo:hi]), ref.params, "params") == 0
+
+
+@pytest.mark.parametrize("psi,world,dtype", [((2 << 30) + 4 * 1001, 4, oracle.F16), (256 << 20, 16, oracle.BF16)])
+def test_staged_windows_beyond_int32(psi, world, dtype):
+    """The staged route (reduce-scatter to fp32, then the in-place update from
+    it) on a bucket of more than 2^31 elements, as one all-partition call of
+    each: windows of the reduced gradients, states and parameters against the
+    oracle, including the windows past element 2^31 and the ragged end."""
+    need = psi * (2 * world + 22) / 1e9 + 2
+    if _free_gb() < need:
+        pytest.skip(f"needs {need:.0f} GB of HBM")
+    tdt = TD[dtype]
+    grads = [torch.empty(psi, dtype=tdt, device="cuda") for _ in range(world)]
+    for k in range(world):
+        _device_grads(grads[k], 6000 + k, 1e-3, 65536.0)
+    st = {nm: torch.empty(psi, dtype=torch.float32, device="cuda") for nm in ("p", "m", "v")}
+    _device_master(st["p"], 78)
+    st["m"].zero_()
+    st["v"].zero_()
+    wins = _windows(psi, world, n_random=8, seed=psi + world) + [(2 ** 31 - 8, 2 ** 31 + 8)] * (psi > 2 ** 31)
+    wins = sorted(set(wins))
+    start = [host_f32(st["p"][lo:hi]).copy() for lo, hi in wins]
+    reduced = torch.empty(psi, dtype=torch.float32, device="cuda")
+    params = torch.empty(psi, dtype=tdt, device="cuda")
+    flags = torch.zeros(2, dtype=torch.int32, device="cuda")
+    adam = workloads.AdamConfig(weight_decay=0.01)
+    hp = Z.hparams(adam.lr, adam.beta1, adam.beta2, adam.eps, adam.weight_decay, 1)
+    Z.zero_reduce_scatter_grads(grads, psi, Z.ZERO_ALL_PARTITIONS, 65536.0, reduced, flags[0:1])
+    Z.zero_adam_step_reduced(reduced, psi, st["p"], st["m"], st["v"], st["p"], st["m"], st["v"], params, hp,
+                             flags[1:2], gate=flags[0:1])
+    torch.cuda.synchronize()
+    assert flags.cpu().tolist() == [0, 0]
+    inv = oracle.adam_constants(adam, 1, float(world), 65536.0)[4]
+    for (lo, hi), p0 in zip(wins, start):
+        G = [_u16(g[lo:hi]) for g in grads]
+        s = oracle.reduce(G, dtype)
+        assert np.array_equal(host_f32(reduced[lo:hi]).view(np.uint32), oracle.unscale(s, inv).view(np.uint32))
+        ref = oracle.initial_state(p0, dtype)
+        oracle.flat_step(G, ref, adam, 1, 65536.0, float(world), dtype, dtype)
+        assert assert_f32_close(host_f32(st["p"][lo:hi]), ref.master, "master") == 0
+        assert assert_f32_close(host_f32(st["m"][lo:hi]), ref.m, "m") == 0
+        assert assert_f32_close(host_f32(st["v"][lo:hi]), ref.v, "v") == 0
         assert assert_u16_close(_u16(params[lo:hi]), ref.params, "params") == 0

@@ -20,6 +20,13 @@ A step (ZeRO explainer, "Stage 2 - Gradient Partitioning (P_os+g)"):
      their parameter buffers (the all-gather, again through the mappings);
   5. host barrier: nobody overwrites a buffer a peer is still reading.
 
+mode="staged" keeps one bank of partition states (the pages' 12 Psi / N
+bytes) plus the partition's reduced fp32 gradients (4 Psi / N): step 2 is
+the staged reduce-scatter (the same peer reads, storing the reduced
+gradients and the flag), the flags are OR-ed over the group, and only when
+no rank overflowed does every rank run the update from its reduced
+gradients in place, writing its slot of the parameter buffer directly.
+
 No kernel waits on another rank: all cross-rank ordering is host barriers,
 so the ranks may also share one GPU (each with its own context).  This class
 sequences library calls; all arithmetic runs in libzero's kernels.
@@ -29,9 +36,9 @@ from __future__ import annotations
 import torch
 import torch.distributed as dist
 
-from . import (DevicePtr, hparams, zero_allgather_params, zero_ipc_close,
+from . import (DevicePtr, hparams, zero_adam_step_reduced, zero_allgather_params, zero_ipc_close,
                zero_ipc_export, zero_ipc_import, zero_loss_scale_update, zero_partition_layout,
-               zero_reduce_scatter_adam_step)
+               zero_reduce_scatter_adam_step, zero_reduce_scatter_grads)
 
 
 class DistributedZeroAdam:
@@ -39,7 +46,10 @@ class DistributedZeroAdam:
                  betas=(0.9, 0.999),
                  eps: float = 1e-8, weight_decay: float = 0.0, grad_dtype=torch.float16,
                  param_dtype=torch.float16, loss_scale: float = 65536.0, growth_interval: int = 1000,
-                 min_scale: float = 1.0, device="cuda"):
+                 min_scale: float = 1.0, mode: str = "banks", device="cuda"):
+        if mode not in ("banks", "staged"):
+            raise ValueError("mode must be 'banks' or 'staged'")
+        self.mode = mode
         self.group = group
         self.rank = dist.get_rank(group)
         self.world = dist.get_world_size(group)
@@ -56,12 +66,17 @@ class DistributedZeroAdam:
         f32 = dict(dtype=torch.float32, device=dev)
         self.grads = [torch.zeros(L.bucket_padded[b], dtype=grad_dtype, device=dev) for b in range(L.n_buckets)]
         self.params = [torch.zeros(L.bucket_padded[b], dtype=param_dtype, device=dev) for b in range(L.n_buckets)]
-        self.master = [[torch.zeros(L.part(b), **f32) for _ in range(2)] for b in range(L.n_buckets)]
-        self.m = [[torch.zeros(L.part(b), **f32) for _ in range(2)] for b in range(L.n_buckets)]
-        self.v = [[torch.zeros(L.part(b), **f32) for _ in range(2)] for b in range(L.n_buckets)]
-        # spare parameter slot: the update of a step that may still be skipped
-        self.param_spare = [torch.zeros(L.part(b), dtype=param_dtype, device=dev) for b in range(L.n_buckets)]
-        self.flag = torch.zeros(1, dtype=torch.int32, device=dev)
+        nbank = 2 if mode == "banks" else 1
+        self.master = [[torch.zeros(L.part(b), **f32) for _ in range(nbank)] for b in range(L.n_buckets)]
+        self.m = [[torch.zeros(L.part(b), **f32) for _ in range(nbank)] for b in range(L.n_buckets)]
+        self.v = [[torch.zeros(L.part(b), **f32) for _ in range(nbank)] for b in range(L.n_buckets)]
+        if mode == "banks":
+            # spare parameter slot: the update of a step that may still be skipped
+            self.param_spare = [torch.zeros(L.part(b), dtype=param_dtype, device=dev) for b in range(L.n_buckets)]
+        else:
+            self.reduced = [torch.zeros(L.part(b), **f32) for b in range(L.n_buckets)]
+        self.flags = torch.zeros(2, dtype=torch.int32, device=dev)    # [step flag, update status]
+        self.flag = self.flags[0:1]
         self._map_peers()
 
     # ------------------------------------------------------------------ IPC
@@ -102,7 +117,7 @@ class DistributedZeroAdam:
         for b in range(self.layout.n_buckets):
             P = self.layout.part(b)
             own = slice(self.rank * P, (self.rank + 1) * P)
-            for bank in range(2):
+            for bank in range(len(self.master[b])):
                 self.master[b][bank].copy_(master_flat[b][own])
                 self.m[b][bank].zero_()
                 self.v[b][bank].zero_()
@@ -126,20 +141,35 @@ class DistributedZeroAdam:
         L, r = self.layout, self.rank
         torch.cuda.synchronize()
         dist.barrier(group=self.group)                  # every rank's gradients are written
-        self.flag.zero_()
+        self.flags.zero_()
         hp = hparams(self.lr, self.betas[0], self.betas[1], self.eps, self.weight_decay, self.t + 1)
-        c, n = self.cur, self.cur ^ 1
-        for b in range(L.n_buckets):
-            zero_reduce_scatter_adam_step(
-                self.peer_grads[b], L.bucket_padded[b], r,
-                self.master[b][c], self.m[b][c], self.v[b][c],
-                self.master[b][n], self.m[b][n], self.v[b][n], self.param_spare[b],
-                hp, self.scale, self.flag)
+        if self.mode == "staged":
+            for b in range(L.n_buckets):
+                zero_reduce_scatter_grads(self.peer_grads[b], L.bucket_padded[b], r, self.scale, self.reduced[b],
+                                          self.flag)
+        else:
+            c, n = self.cur, self.cur ^ 1
+            for b in range(L.n_buckets):
+                zero_reduce_scatter_adam_step(
+                    self.peer_grads[b], L.bucket_padded[b], r,
+                    self.master[b][c], self.m[b][c], self.v[b][c],
+                    self.master[b][n], self.m[b][n], self.v[b][n], self.param_spare[b],
+                    hp, self.scale, self.flag)
         ovf = self._or_over_ranks(int(self.flag.item()))     # synchronizes this rank's stream
         if ovf & 2:
             raise RuntimeError("fused step kernel timed out waiting on its copy pipeline; step not committed")
         applied = ovf == 0
-        if applied:
+        if applied and self.mode == "staged":
+            # every rank knows the verdict of the whole group: update in place
+            for b in range(L.n_buckets):
+                P = L.part(b)
+                st = (self.master[b][0], self.m[b][0], self.v[b][0])
+                zero_adam_step_reduced(self.reduced[b], P, *st, *st, self.params[b][r * P:(r + 1) * P], hp,
+                                       self.flags[1:2])
+            if int(self.flags[1].item()) & 2:
+                raise RuntimeError("staged update timed out waiting on its copy pipeline; states incomplete")
+            self.t += 1
+        elif applied:
             for b in range(L.n_buckets):
                 P = L.part(b)
                 zero_allgather_params([self.param_spare[b]], 0, P, self.params[b][r * P:(r + 1) * P])
