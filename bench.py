@@ -551,13 +551,17 @@ def run_e2e(opt, args, stream, barrier, world_gpus):
     """Same step through ZeroAdam.step_from_host: every step copies the N
     replicas' gradients from pinned host memory and reads the flag back."""
     import torch
+    short = 0.0
     try:
         import psutil
         need = sum(g.numel() * g.element_size() for per in opt.grads for g in per)
         if psutil.virtual_memory().available < 1.5 * need * max(1, world_gpus):
-            return {"value": None, "unit": UNIT, "skipped": "not enough host memory for pinned gradients"}
+            short = 1.0
     except Exception:
         pass
+    # every rank takes the same branch (the timed part below has collectives)
+    if max_over_ranks(short, "cuda") > 0:
+        return {"value": None, "unit": UNIT, "skipped": "not enough host memory for pinned gradients"}
     host = [[torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in per] for per in opt.grads]
     for b, per in enumerate(opt.grads):
         for k, g in enumerate(per):
