@@ -13,6 +13,7 @@ import subprocess
 
 import numpy as np
 import pytest
+import torch
 
 import oracle
 import workloads
@@ -269,3 +270,73 @@ def test_header_is_plain_c_and_links(tmp_path):
     lines = out.stdout.splitlines()
     assert lines[0] == "3 8 8"          # buckets [5], [7], [11] padded to multiples of 4
     assert lines[1].startswith("invalid argument|zero_reduce_scatter_adam_step")
+
+
+class _FakeCuda:
+    """Stands in for a CUDA tensor in the binding's checks (nothing is launched:
+    every case below fails before the C call)."""
+
+    def __init__(self, n, dtype, cuda=True, contiguous=True, ptr=0x7000_0000):
+        self.n, self.dtype, self.is_cuda, self._contig, self.ptr = n, dtype, cuda, contiguous, ptr
+
+    def numel(self):
+        return self.n
+
+    def element_size(self):
+        return torch.empty((), dtype=self.dtype).element_size()
+
+    def is_contiguous(self):
+        return self._contig
+
+    def data_ptr(self):
+        return self.ptr
+
+
+def _fake_step(**over):
+    f32, f16 = torch.float32, torch.float16
+    n, world = 64, 2
+    args = dict(grad_bufs=[_FakeCuda(n, f16), _FakeCuda(n, f16)], padded_numel=n, partition=-1,
+                master_in=_FakeCuda(n, f32), m_in=_FakeCuda(n, f32), v_in=_FakeCuda(n, f32),
+                master_out=_FakeCuda(n, f32), m_out=_FakeCuda(n, f32), v_out=_FakeCuda(n, f32),
+                param_out=_FakeCuda(n, f16), hp=Z.hparams(), loss_scale=1024.0,
+                overflow_flag=_FakeCuda(1, torch.int32))
+    args.update(over)
+    Z.zero_reduce_scatter_adam_step(**args, stream=0)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(master_in=_FakeCuda(64, torch.float32, cuda=False)), -1),         # host tensor
+    (dict(m_out=_FakeCuda(64, torch.float32, contiguous=False)), -1),       # strided view
+    (dict(v_in=_FakeCuda(64, torch.float16)), -3),                           # wrong dtype
+    (dict(master_out=_FakeCuda(63, torch.float32)), -4),                     # too small
+    (dict(param_out=_FakeCuda(10, torch.float16)), -4),
+    (dict(grad_bufs=[_FakeCuda(64, torch.float16), _FakeCuda(32, torch.float16)]), -4),
+    (dict(overflow_flag=_FakeCuda(1, torch.float32)), -3),
+    (dict(overflow_flag=_FakeCuda(1, torch.int32, cuda=False)), -1),
+])
+def test_binding_checks_tensors_before_the_call(over, code):
+    with pytest.raises(Z.ZeroError) as e:
+        _fake_step(**over)
+    assert e.value.code == code
+
+
+def test_binding_partition_sizes_and_staged_checks():
+    f32 = torch.float32
+    # one partition needs only P = 32 elements of state
+    small = {k: _FakeCuda(31, f32) for k in ("master_in",)}
+    with pytest.raises(Z.ZeroError) as e:
+        _fake_step(partition=1, **small)
+    assert e.value.code == -4
+    # staged update: the reduced gradient must be fp32 and large enough
+    st = [_FakeCuda(64, f32) for _ in range(6)]
+    with pytest.raises(Z.ZeroError) as e:
+        Z.zero_adam_step_reduced(_FakeCuda(63, f32), 64, *st, _FakeCuda(64, torch.float16), Z.hparams(),
+                                 _FakeCuda(1, torch.int32), stream=0)
+    assert e.value.code == -4
+    with pytest.raises(Z.ZeroError) as e:
+        Z.zero_reduce_scatter_grads([_FakeCuda(64, torch.float16)] * 2, 64, -1, 1.0, _FakeCuda(64, torch.float16),
+                                    _FakeCuda(1, torch.int32), stream=0)
+    assert e.value.code == -3
+    with pytest.raises(Z.ZeroError) as e:           # gather source shorter than offset + part
+        Z.zero_allgather_params([_FakeCuda(100, torch.float16)] * 2, 60, 50, _FakeCuda(100, torch.float16), stream=0)
+    assert e.value.code == -4

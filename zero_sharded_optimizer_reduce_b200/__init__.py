@@ -7,6 +7,12 @@ streams default to torch's current stream.
 
 The library is loaded from this package directory.  If it is missing, import
 fails with an error that says how to build it: there is no fallback.
+
+The C calls see bare pointers and cannot check sizes; the wrappers here check
+what they can before anything is launched: device arguments must be
+contiguous CUDA tensors of the right dtype holding at least the elements the
+call touches (ZeroError otherwise).  A DevicePtr (another process's mapped
+buffer) is passed through unchecked.
 """
 from __future__ import annotations
 
@@ -177,6 +183,59 @@ def _ptrs(ts) -> ctypes.Array:
     return (ctypes.c_void_p * len(ts))(*[_ptr(t) for t in ts])
 
 
+_ELEM_BYTES = {ZERO_F16: 2, ZERO_BF16: 2, ZERO_F32: 4}
+
+
+def _dev(t, n: int, name: str, dtype=None) -> int:
+    """Address of a device argument after the checks the C ABI cannot make
+    (it sees bare pointers): a CUDA tensor, contiguous, of `dtype` when
+    given, holding at least `n` elements (of `dtype`, else of its own type).
+    None passes as NULL (the C call decides whether NULL is allowed); a
+    DevicePtr (another process's mapped buffer) is trusted as it is."""
+    if t is None:
+        return 0
+    if isinstance(t, DevicePtr):
+        return t.ptr
+    if not getattr(t, "is_cuda", False):
+        raise ZeroError(-1, f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ZeroError(-1, f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ZeroError(-3, f"{name} must be {dtype}, got {t.dtype}")
+    if t.numel() < n:
+        raise ZeroError(-4, f"{name} holds {t.numel()} elements, the call needs {n}")
+    return int(t.data_ptr())
+
+
+def _devs(ts, n: int, name: str) -> ctypes.Array:
+    return (ctypes.c_void_p * len(ts))(*[_dev(t, n, f"{name}[{k}]") for k, t in enumerate(ts)])
+
+
+def _f32():
+    import torch
+    return torch.float32
+
+
+def _count(padded_numel: int, world: int, partition: int) -> int:
+    """Elements one call processes: the whole bucket, or one partition."""
+    return padded_numel if partition == ZERO_ALL_PARTITIONS else padded_numel // max(1, world)
+
+
+def _flag_args(overflow_flag, grad_sqnorm, workspace):
+    import torch
+    ws_bytes = zero_step_workspace_bytes() if grad_sqnorm is not None else 0
+    if workspace is not None and not isinstance(workspace, DevicePtr) and \
+            workspace.numel() * workspace.element_size() < ws_bytes:
+        raise ZeroError(-4, f"workspace holds {workspace.numel() * workspace.element_size()} bytes, "
+                            f"the norm needs {ws_bytes}")
+    return (_dev(overflow_flag, 1, "overflow_flag", torch.int32), _dev(grad_sqnorm, 1, "grad_sqnorm", torch.float64),
+            _dev(workspace, 0, "workspace"))
+
+
+def _state_args(count, names_tensors):
+    return [_dev(t, count, nm, _f32()) for nm, t in names_tensors]
+
+
 # ---------------------------------------------------------------------------
 # Layout
 # ---------------------------------------------------------------------------
@@ -240,10 +299,18 @@ def zero_partition_layout(numels, world: int, bucket_elems: int = 0, align_elems
 
 def zero_flatten_bucket(layout: Layout, bucket: int, tensors, bucket_buf, stream=None) -> None:
     """Copy bucket `bucket`'s tensors (list indexed by tensor id) into bucket_buf."""
-    ptrs = (ctypes.c_void_p * max(1, len(tensors)))(*[_ptr(t) for t in tensors])
+    if not 0 <= bucket < layout.n_buckets:
+        raise ZeroError(-4, f"bucket {bucket} outside 0..{layout.n_buckets - 1}")
+    if len(tensors) != len(layout.tensor_numel):
+        raise ZeroError(-1, f"{len(tensors)} tensors given, the layout has {len(layout.tensor_numel)}")
+    first, cnt = layout.bucket_first[bucket], layout.bucket_count[bucket]
+    addrs = [0] * len(tensors)
+    for i in range(first, first + cnt):
+        addrs[i] = _dev(tensors[i], layout.tensor_numel[i], f"tensors[{i}]", bucket_buf.dtype)
+    ptrs = (ctypes.c_void_p * max(1, len(tensors)))(*addrs)
     c = layout._c()
     _check(lib.zero_flatten_bucket(ctypes.byref(c), bucket, ptrs, _dtype_code(bucket_buf),
-                                   _ptr(bucket_buf), _stream(stream)))
+                                   _dev(bucket_buf, layout.bucket_padded[bucket], "bucket_buf"), _stream(stream)))
 
 
 def zero_step_workspace_bytes() -> int:
@@ -261,11 +328,13 @@ def zero_reduce_scatter_adam_step(grad_bufs, padded_numel: int, partition: int,
                                   grad_sqnorm=None, workspace=None, stream=None) -> None:
     """One fused reduce-scatter + Adam pass over one bucket (see include/zero.h)."""
     world = len(grad_bufs)
+    n = _count(padded_numel, world, partition)
+    st = _state_args(n, (("master_in", master_in), ("m_in", m_in), ("v_in", v_in), ("master_out", master_out),
+                         ("m_out", m_out), ("v_out", v_out)))
     _check(lib.zero_reduce_scatter_adam_step(
-        _ptrs(grad_bufs), world, padded_numel, partition, _dtype_code(grad_bufs[0]),
-        _ptr(master_in), _ptr(m_in), _ptr(v_in), _ptr(master_out), _ptr(m_out), _ptr(v_out),
-        _ptr(param_out), _dtype_code(param_out), ctypes.byref(hp), float(loss_scale),
-        _ptr(overflow_flag), _ptr(grad_sqnorm), _ptr(workspace), _stream(stream)))
+        _devs(grad_bufs, padded_numel, "grad_bufs"), world, padded_numel, partition, _dtype_code(grad_bufs[0]),
+        *st, _dev(param_out, n, "param_out"), _dtype_code(param_out), ctypes.byref(hp), float(loss_scale),
+        *_flag_args(overflow_flag, grad_sqnorm, workspace), _stream(stream)))
 
 
 def zero_reduce_scatter_adam_step_noalloc(grad_bufs, padded_numel: int, partition: int,
@@ -276,19 +345,22 @@ def zero_reduce_scatter_adam_step_noalloc(grad_bufs, padded_numel: int, partitio
     allocate device memory: the norm's scratch lives in a fixed array inside
     libzero (see include/zero.h for its limits)."""
     world = len(grad_bufs)
+    n = _count(padded_numel, world, partition)
+    st = _state_args(n, (("master_in", master_in), ("m_in", m_in), ("v_in", v_in), ("master_out", master_out),
+                         ("m_out", m_out), ("v_out", v_out)))
+    flag, sq, _ = _flag_args(overflow_flag, grad_sqnorm, None)
     _check(lib.zero_reduce_scatter_adam_step_noalloc(
-        _ptrs(grad_bufs), world, padded_numel, partition, _dtype_code(grad_bufs[0]),
-        _ptr(master_in), _ptr(m_in), _ptr(v_in), _ptr(master_out), _ptr(m_out), _ptr(v_out),
-        _ptr(param_out), _dtype_code(param_out), ctypes.byref(hp), float(loss_scale),
-        _ptr(overflow_flag), _ptr(grad_sqnorm), _stream(stream)))
+        _devs(grad_bufs, padded_numel, "grad_bufs"), world, padded_numel, partition, _dtype_code(grad_bufs[0]),
+        *st, _dev(param_out, n, "param_out"), _dtype_code(param_out), ctypes.byref(hp), float(loss_scale),
+        flag, sq, _stream(stream)))
 
 
 def zero_grad_stats(grad_bufs, padded_numel: int, partition: int, loss_scale: float, overflow_flag,
                     grad_sqnorm=None, workspace=None, grad_divisor: float = 0.0, stream=None) -> None:
     """Overflow flag and squared norm of one bucket's reduced gradients (no update)."""
-    _check(lib.zero_grad_stats(_ptrs(grad_bufs), len(grad_bufs), padded_numel, partition,
+    _check(lib.zero_grad_stats(_devs(grad_bufs, padded_numel, "grad_bufs"), len(grad_bufs), padded_numel, partition,
                                _dtype_code(grad_bufs[0]), float(loss_scale), float(grad_divisor),
-                               _ptr(overflow_flag), _ptr(grad_sqnorm), _ptr(workspace), _stream(stream)))
+                               *_flag_args(overflow_flag, grad_sqnorm, workspace), _stream(stream)))
 
 
 def zero_reduce_scatter_adam_step_gated(grad_bufs, padded_numel: int, partition: int,
@@ -297,23 +369,27 @@ def zero_reduce_scatter_adam_step_gated(grad_bufs, padded_numel: int, partition:
                                         grad_sqnorm=None, workspace=None, gate=None, clip_sqnorm=None,
                                         max_norm: float = 0.0, stream=None) -> None:
     """The fused step, skipped entirely when *gate != 0, with optional clipping."""
+    import torch
     world = len(grad_bufs)
+    n = _count(padded_numel, world, partition)
+    st = _state_args(n, (("master_in", master_in), ("m_in", m_in), ("v_in", v_in), ("master_out", master_out),
+                         ("m_out", m_out), ("v_out", v_out)))
     _check(lib.zero_reduce_scatter_adam_step_gated(
-        _ptrs(grad_bufs), world, padded_numel, partition, _dtype_code(grad_bufs[0]),
-        _ptr(master_in), _ptr(m_in), _ptr(v_in), _ptr(master_out), _ptr(m_out), _ptr(v_out),
-        _ptr(param_out), _dtype_code(param_out), ctypes.byref(hp), float(loss_scale),
-        _ptr(overflow_flag), _ptr(grad_sqnorm), _ptr(workspace), _ptr(gate), _ptr(clip_sqnorm),
-        float(max_norm), _stream(stream)))
+        _devs(grad_bufs, padded_numel, "grad_bufs"), world, padded_numel, partition, _dtype_code(grad_bufs[0]),
+        *st, _dev(param_out, n, "param_out"), _dtype_code(param_out), ctypes.byref(hp), float(loss_scale),
+        *_flag_args(overflow_flag, grad_sqnorm, workspace), _dev(gate, 1, "gate", torch.int32),
+        _dev(clip_sqnorm, 1, "clip_sqnorm", torch.float64), float(max_norm), _stream(stream)))
 
 
 def zero_reduce_scatter_grads(grad_bufs, padded_numel: int, partition: int, loss_scale: float, reduced_out,
                               overflow_flag, grad_sqnorm=None, workspace=None, grad_divisor: float = 0.0,
                               stream=None) -> None:
     """Staged reduce-scatter: reduced_out = fp32 unscaled rank-order sums, plus flag and norm."""
-    _check(lib.zero_reduce_scatter_grads(_ptrs(grad_bufs), len(grad_bufs), padded_numel, partition,
-                                         _dtype_code(grad_bufs[0]), float(loss_scale), float(grad_divisor),
-                                         _ptr(reduced_out), _ptr(overflow_flag), _ptr(grad_sqnorm),
-                                         _ptr(workspace), _stream(stream)))
+    n = _count(padded_numel, len(grad_bufs), partition)
+    _check(lib.zero_reduce_scatter_grads(_devs(grad_bufs, padded_numel, "grad_bufs"), len(grad_bufs), padded_numel,
+                                         partition, _dtype_code(grad_bufs[0]), float(loss_scale), float(grad_divisor),
+                                         _dev(reduced_out, n, "reduced_out", _f32()),
+                                         *_flag_args(overflow_flag, grad_sqnorm, workspace), _stream(stream)))
 
 
 def zero_adam_step_reduced(reduced_grad, count: int, master_in, m_in, v_in, master_out, m_out, v_out, param_out,
@@ -321,16 +397,20 @@ def zero_adam_step_reduced(reduced_grad, count: int, master_in, m_in, v_in, mast
                            stream=None) -> None:
     """Staged update: Adam on `count` elements from fp32 reduced gradients (gated, optionally clipped);
     `status` (device int32) receives bit 1 if the kernel's copy pipeline timed out."""
+    import torch
+    st = _state_args(count, (("reduced_grad", reduced_grad), ("master_in", master_in), ("m_in", m_in),
+                             ("v_in", v_in), ("master_out", master_out), ("m_out", m_out), ("v_out", v_out)))
     _check(lib.zero_adam_step_reduced(
-        _ptr(reduced_grad), count, _ptr(master_in), _ptr(m_in), _ptr(v_in), _ptr(master_out), _ptr(m_out),
-        _ptr(v_out), _ptr(param_out), _dtype_code(param_out), ctypes.byref(hp), _ptr(status), _ptr(gate),
-        _ptr(clip_sqnorm), float(max_norm), _stream(stream)))
+        st[0], count, *st[1:], _dev(param_out, count, "param_out"), _dtype_code(param_out), ctypes.byref(hp),
+        _dev(status, 1, "status", torch.int32), _dev(gate, 1, "gate", torch.int32),
+        _dev(clip_sqnorm, 1, "clip_sqnorm", torch.float64), float(max_norm), _stream(stream)))
 
 
 def zero_allgather_params(shards, shard_offset: int, part_numel: int, dst, stream=None) -> None:
     """dst[r*part + j] = shards[r][shard_offset + j] (bit-exact copy)."""
-    _check(lib.zero_allgather_params(_ptrs(shards), len(shards), shard_offset, part_numel,
-                                     _dtype_code(dst), _ptr(dst), _stream(stream)))
+    _check(lib.zero_allgather_params(_devs(shards, shard_offset + part_numel, "shards"), len(shards), shard_offset,
+                                     part_numel, _dtype_code(dst), _dev(dst, len(shards) * part_numel, "dst"),
+                                     _stream(stream)))
 
 
 def zero_loss_scale_update(scale: float, good_steps: int, overflow: bool,
@@ -352,24 +432,31 @@ class Runner:
 
     def __init__(self, buckets, hp: AdamHParams, loss_scale: float, flag_dev, flag_host, grad_sqnorm=None,
                  workspace=None, growth_interval: int = 1000, min_scale: float = 1.0):
+        import torch
         descs = (BucketBanks * max(1, len(buckets)))()
         self._keep = []
         world = len(buckets[0][0]) if buckets else 1
         for i, (grads, master, m, v, params) in enumerate(buckets):
-            arr = _ptrs(grads)
+            n = grads[0].numel()
+            arr = _devs(grads, n, f"bucket {i} grads")
             self._keep.append(arr)
             d = descs[i]
-            d.padded_numel = grads[0].numel()
+            d.padded_numel = n
             d.grad_bufs = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
             for b in range(2):
-                d.master[b], d.m[b], d.v[b], d.params[b] = (_ptr(master[b]), _ptr(m[b]), _ptr(v[b]),
-                                                            _ptr(params[b]))
+                d.master[b], d.m[b], d.v[b] = _state_args(n, ((f"bucket {i} master[{b}]", master[b]),
+                                                              (f"bucket {i} m[{b}]", m[b]),
+                                                              (f"bucket {i} v[{b}]", v[b])))
+                d.params[b] = _dev(params[b], n, f"bucket {i} params[{b}]")
         gd = _dtype_code(buckets[0][0][0]) if buckets else ZERO_F16
         pd = _dtype_code(buckets[0][4][0]) if buckets else ZERO_F16
+        if getattr(flag_host, "is_cuda", True) or flag_host.dtype != torch.int32 or flag_host.numel() < 1:
+            raise ZeroError(-1, "flag_host must be a host (pinned) int32 tensor")
         h = ctypes.c_void_p()
         _check(lib.zero_runner_create(descs, len(buckets), world, gd, pd, ctypes.byref(hp), float(loss_scale),
-                                      growth_interval, min_scale, _ptr(flag_dev), _ptr(flag_host),
-                                      _ptr(grad_sqnorm), _ptr(workspace), ctypes.byref(h)))
+                                      growth_interval, min_scale, *_flag_args(flag_dev, None, None)[:1],
+                                      _ptr(flag_host), *_flag_args(flag_dev, grad_sqnorm, workspace)[1:],
+                                      ctypes.byref(h)))
         self._h = h
 
     def launch(self, stream=None) -> None:
@@ -400,14 +487,15 @@ class Runner:
 
 def zero_test_wait_timeout(status, limit_ns: int, stream=None) -> None:
     """Run the bounded-wait self-test: ORs 2 into status after ~limit_ns."""
-    _check(lib.zero_test_wait_timeout(_ptr(status), int(limit_ns), _stream(stream)))
+    import torch
+    _check(lib.zero_test_wait_timeout(_dev(status, 1, "status", torch.int32), int(limit_ns), _stream(stream)))
 
 
 def zero_ipc_export(tensor) -> tuple:
     """(handle bytes, byte offset) of a device buffer, for another process."""
     h = IpcHandle()
     off = ctypes.c_int64()
-    _check(lib.zero_ipc_export(_ptr(tensor), ctypes.byref(h), ctypes.byref(off)))
+    _check(lib.zero_ipc_export(_dev(tensor, 0, "tensor"), ctypes.byref(h), ctypes.byref(off)))
     return bytes(h.bytes), int(off.value)
 
 
