@@ -352,6 +352,35 @@ int zero_adam_step_reduced(const float* reduced_grad, int64_t count,
                            zero_stream_t stream);
 
 /*
+ * zero_adam_step_reduced_bcast - zero_adam_step_reduced that writes the
+ * updated parameters to several destinations: the all-gather of the
+ * updated parameters done by the update's own stores.
+ *
+ * Source: ZeRO explainer, "Stage 2 - Gradient Partitioning (P_os+g)" (after
+ * the update the parameters are all-gathered, so every rank again holds all
+ * of them).  Rank r passes, for every rank q, the address of slot r of rank
+ * q's parameter buffer (peers' buffers mapped into this process, e.g. with
+ * zero_ipc_import); each updated parameter is stored to all of them, so no
+ * separate gather is needed once every rank's call has completed.  Results
+ * equal those of zero_adam_step_reduced at every destination.
+ *
+ * param_dsts  host array of n_dsts device pointers (1 .. ZERO_MAX_WORLD),
+ *             each `count` elements of param_dtype, 2-byte aligned, not
+ *             overlapping each other or any input or state array.  When
+ *             their 16-byte phases differ from the first's, every element
+ *             is stored on its own (slower, same results).
+ * other arguments: as for zero_adam_step_reduced.
+ * Errors: those of zero_adam_step_reduced.
+ */
+int zero_adam_step_reduced_bcast(const float* reduced_grad, int64_t count,
+                                 const float* master_in, const float* m_in, const float* v_in,
+                                 float* master_out, float* m_out, float* v_out,
+                                 void* const* param_dsts, int32_t n_dsts, zero_dtype_t param_dtype,
+                                 const zero_adam_hparams_t* hp, int32_t* status,
+                                 const int32_t* gate, const double* clip_sqnorm, float max_norm,
+                                 zero_stream_t stream);
+
+/*
  * zero_reduce_scatter_adam_step_noalloc - zero_reduce_scatter_adam_step for
  * callers that cannot allocate device memory.
  *
@@ -463,7 +492,8 @@ typedef struct zero_runner zero_runner_t;   /* opaque, host memory */
  * *flag_dev (and *grad_sqnorm), the fused step over every bucket reading bank
  * `cur` and writing bank `cur ^ 1` with hyper-parameters hp (step = t + 1)
  * and the current loss scale, and a copy of *flag_dev into *flag_host.
- * zero_runner_commit waits for the stream, reads *flag_host and, when it is
+ * zero_runner_commit waits for the stream (pass the stream the launch used),
+ * reads *flag_host and, when it is
  * 0, makes bank `cur ^ 1` current and advances t; it then applies
  * zero_loss_scale_update and reports *applied (1 = update applied).  A launch
  * must be followed by a commit before the next launch.

@@ -340,3 +340,24 @@ def test_binding_partition_sizes_and_staged_checks():
     with pytest.raises(Z.ZeroError) as e:           # gather source shorter than offset + part
         Z.zero_allgather_params([_FakeCuda(100, torch.float16)] * 2, 60, 50, _FakeCuda(100, torch.float16), stream=0)
     assert e.value.code == -4
+
+
+def test_broadcast_update_rejects_bad_destinations():
+    L = Z.lib
+    base = 0x7000_0000
+    st = [base + 0x100_0000 * i for i in range(1, 7)]
+    red, status, hp = base + 0x100_0000 * 12, base + 0x100_0000 * 13, Z.hparams()
+
+    def call(dsts, n_dsts=None):
+        arr = None if dsts is None else (ctypes.c_void_p * max(1, len(dsts)))(*dsts)
+        return L.zero_adam_step_reduced_bcast(red, 64, *st, arr, len(dsts or []) if n_dsts is None else n_dsts, 0,
+                                              ctypes.byref(hp), status, None, None, 0.0, None)
+    assert call(None, 1) == -1                                      # no destination array
+    assert call([0x7E00_0000], 0) == -1                             # no destinations
+    assert call([0x7E00_0000] * 129) == -1                          # more than ZERO_MAX_WORLD
+    assert call([0x7E00_0000, 0]) == -1                             # NULL destination
+    assert call([0x7E00_0000, 0x7F00_0001]) == -2                   # misaligned destination
+    assert call([0x7E00_0000, 0x7E00_0040]) == -1                   # destinations overlap
+    assert call([0x7E00_0000, st[0] + 16]) == -1                    # destination overlaps master_in
+    assert L.zero_adam_step_reduced_bcast(red, 0, *st, (ctypes.c_void_p * 1)(0x7E00_0000), 1, 0,
+                                          ctypes.byref(hp), status, None, None, 0.0, None) == 0

@@ -17,7 +17,7 @@ import torch
 import oracle
 import workloads
 import zero_sharded_optimizer_reduce_b200 as Z
-from _gpu import Guarded, assert_f32_close, host_f32, to_dev_f32, to_dev_u16
+from _gpu import Guarded, host_f32, host_u16, to_dev_f32, to_dev_u16
 from test_gpu_gated import _norm_tol
 from test_gpu_step import Case, _adam, _hp
 
@@ -163,3 +163,25 @@ def test_staged_clip_matches_oracle():
     diffs = c.compare(ref)
     if oracle.clip_coefficient(float(c.norm.item()), np.float32(max_norm)) == clip:
         assert diffs == [0, 0, 0, 0], diffs
+
+
+@pytest.mark.parametrize("shift", [0, 3])
+def test_staged_update_broadcasts_parameters(shift):
+    """zero_adam_step_reduced_bcast: the same update, its parameters stored to
+    several destinations (one of them off the 16-byte phase when shift > 0:
+    then every element is stored on its own); each equals the oracle."""
+    world, padded = 4, 4 * 600_007          # the pipeline size
+    c = Staged(padded, world, seed=590, scale=65536.0, inplace=True)
+    c.reduce_scatter()
+    dsts = [c.p_dev] + [Guarded(c.n, torch.float16, shift if k == 1 else 0) for k in range(2)]
+    adam = _adam(0.01)
+    Z.zero_adam_step_reduced_bcast(c.red.t, c.n, *[b.t for b in c.in_dev], *[b.t for b in c.out_dev],
+                                   [d.t for d in dsts], _hp(adam, 2), c.status, gate=c.flag)
+    torch.cuda.synchronize()
+    assert int(c.status.item()) == 0
+    for b in c.in_dev + dsts + [c.red]:
+        b.check()
+    ref, _, _ = c.expect(adam, t=2)
+    assert c.compare(ref) == [0, 0, 0, 0]
+    for d in dsts[1:]:
+        assert np.array_equal(host_u16(d.t), ref.params)

@@ -116,6 +116,9 @@ def _load():
     L.zero_adam_step_reduced.argtypes = [vp, i64, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int,
                                          ctypes.POINTER(AdamHParams), vp, vp, vp, f32, vp]
     L.zero_adam_step_reduced.restype = ctypes.c_int
+    L.zero_adam_step_reduced_bcast.argtypes = [vp, i64, vp, vp, vp, vp, vp, vp, ctypes.POINTER(vp), i32, ctypes.c_int,
+                                               ctypes.POINTER(AdamHParams), vp, vp, vp, f32, vp]
+    L.zero_adam_step_reduced_bcast.restype = ctypes.c_int
     L.zero_ipc_export.argtypes = [vp, ctypes.POINTER(IpcHandle), ctypes.POINTER(i64)]
     L.zero_ipc_export.restype = ctypes.c_int
     L.zero_ipc_import.argtypes = [ctypes.POINTER(IpcHandle), i64, ctypes.POINTER(vp), ctypes.POINTER(vp)]
@@ -404,6 +407,23 @@ def zero_adam_step_reduced(reduced_grad, count: int, master_in, m_in, v_in, mast
         st[0], count, *st[1:], _dev(param_out, count, "param_out"), _dtype_code(param_out), ctypes.byref(hp),
         _dev(status, 1, "status", torch.int32), _dev(gate, 1, "gate", torch.int32),
         _dev(clip_sqnorm, 1, "clip_sqnorm", torch.float64), float(max_norm), _stream(stream)))
+
+
+def zero_adam_step_reduced_bcast(reduced_grad, count: int, master_in, m_in, v_in, master_out, m_out, v_out,
+                                 param_dsts, hp: AdamHParams, status, gate=None, clip_sqnorm=None,
+                                 max_norm: float = 0.0, stream=None) -> None:
+    """zero_adam_step_reduced storing the updated parameters to every tensor
+    (or mapped DevicePtr) in `param_dsts`: the all-gather done by the
+    update's own stores."""
+    import torch
+    st = _state_args(count, (("reduced_grad", reduced_grad), ("master_in", master_in), ("m_in", m_in),
+                             ("v_in", v_in), ("master_out", master_out), ("m_out", m_out), ("v_out", v_out)))
+    dsts = _devs(param_dsts, count, "param_dsts")
+    _check(lib.zero_adam_step_reduced_bcast(
+        st[0], count, *st[1:], ctypes.cast(dsts, ctypes.POINTER(ctypes.c_void_p)), len(param_dsts),
+        _dtype_code(param_dsts[0]), ctypes.byref(hp), _dev(status, 1, "status", torch.int32),
+        _dev(gate, 1, "gate", torch.int32), _dev(clip_sqnorm, 1, "clip_sqnorm", torch.float64), float(max_norm),
+        _stream(stream)))
 
 
 def zero_allgather_params(shards, shard_offset: int, part_numel: int, dst, stream=None) -> None:

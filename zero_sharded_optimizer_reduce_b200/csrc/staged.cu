@@ -26,43 +26,50 @@ inline uint32_t reduced_pipe_smem_bytes(int tile) {
     return static_cast<uint32_t>(kReducedStages) * 16u * static_cast<uint32_t>(tile);
 }
 
-inline KernelFn pick_reduced_kernel(zero_dtype_t pd) {
-    return pd == ZERO_F16 ? adam_reduced_kernel<__half> : adam_reduced_kernel<__nv_bfloat16>;
+using ReducedKernelFn = void (*)(StepParams, ParamDsts);
+
+inline ReducedKernelFn pick_reduced_kernel(zero_dtype_t pd, bool bcast) {
+    if (bcast) return pd == ZERO_F16 ? adam_reduced_kernel<__half, true> : adam_reduced_kernel<__nv_bfloat16, true>;
+    return pd == ZERO_F16 ? adam_reduced_kernel<__half, false> : adam_reduced_kernel<__nv_bfloat16, false>;
 }
 
-inline KernelFn pick_reduced_pipe_kernel(zero_dtype_t pd) {
-    return pd == ZERO_F16 ? adam_reduced_pipe_kernel<__half> : adam_reduced_pipe_kernel<__nv_bfloat16>;
+inline ReducedKernelFn pick_reduced_pipe_kernel(zero_dtype_t pd, bool bcast) {
+    if (bcast)
+        return pd == ZERO_F16 ? adam_reduced_pipe_kernel<__half, true> : adam_reduced_pipe_kernel<__nv_bfloat16, true>;
+    return pd == ZERO_F16 ? adam_reduced_pipe_kernel<__half, false> : adam_reduced_pipe_kernel<__nv_bfloat16, false>;
 }
 
 struct ReducedDevice {
     int sms = 0;
-    int blocks_per_sm[2] = {0, 0};
-    bool pipe_ready[2] = {false, false};
+    int blocks_per_sm[4] = {0, 0, 0, 0};        // [dtype * 2 + bcast]
+    bool pipe_ready[4] = {false, false, false, false};
 };
 
 std::mutex g_red_mu;
 ReducedDevice g_red[64];
 
 // SM count, resident blocks of the register kernel, and the pipeline
-// kernel's shared-memory limit, queried or set once per device and dtype.
-inline int reduced_device(zero_dtype_t pd, ReducedDevice** out) {
+// kernel's shared-memory limit, queried or set once per device, dtype and
+// store mode.
+inline int reduced_device(zero_dtype_t pd, bool bcast, ReducedDevice** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return fail(ZERO_ERR_CUDA, "cudaGetDevice failed");
     std::lock_guard<std::mutex> lk(g_red_mu);
     ReducedDevice& d = g_red[dev];
-    const int w = pd == ZERO_F16 ? 0 : 1;
+    const int w = (pd == ZERO_F16 ? 0 : 2) + (bcast ? 1 : 0);
     if (d.sms == 0 && cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
         d.sms = 0;
         return fail(ZERO_ERR_CUDA, "cannot query the SM count");
     }
     if (d.blocks_per_sm[w] == 0) {
         int n = 0;
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, pick_reduced_kernel(pd), kThreads, 0);
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, pick_reduced_kernel(pd, bcast), kThreads, 0);
         if (e != cudaSuccess || n < 1) return fail(ZERO_ERR_CUDA, "occupancy query failed: %s", cudaGetErrorString(e));
         d.blocks_per_sm[w] = n;
     }
     if (!d.pipe_ready[w]) {
-        cudaError_t e = cudaFuncSetAttribute(pick_reduced_pipe_kernel(pd), cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(pick_reduced_pipe_kernel(pd, bcast),
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(reduced_pipe_smem_bytes(kReducedTile)));
         if (e != cudaSuccess) return fail(ZERO_ERR_CUDA, "cannot raise the shared-memory limit: %s", cudaGetErrorString(e));
         d.pipe_ready[w] = true;
@@ -144,6 +151,35 @@ inline int prepare_reduced(const char* fn, const float* reduced, int64_t count, 
     return ZERO_OK;
 }
 
+// Enqueue the update prepared by prepare_reduced: the pipeline kernel when
+// the aligned part gives every SM at least two tiles, else the register
+// kernel.  `work` as returned by prepare_reduced (> 0).
+inline int launch_reduced(const char* fn, StepParams prm, const ParamDsts& d, int64_t work, zero_dtype_t pd,
+                          bool bcast, zero_stream_t stream) {
+    ReducedDevice* dev = nullptr;
+    if (int rc = reduced_device(pd, bcast, &dev)) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t ntiles = prm.nvec > 0 ? (prm.count - prm.head) / kReducedTile : 0;
+    if (ntiles >= 2 * static_cast<int64_t>(dev->sms)) {
+        // the pipeline kernel takes the whole tiles; the rest goes through
+        // its scalar path
+        prm.tile = kReducedTile;
+        prm.nvec = ntiles * kReducedTile / kVec;
+        pick_reduced_pipe_kernel(pd, bcast)<<<static_cast<unsigned int>(dev->sms), kPipeThreads,
+                                             reduced_pipe_smem_bytes(kReducedTile), s>>>(prm, d);
+    } else {
+        const int w = (pd == ZERO_F16 ? 0 : 2) + (bcast ? 1 : 0);
+        const int64_t limit = static_cast<int64_t>(dev->sms) * dev->blocks_per_sm[w];
+        int64_t blocks = (work + kThreads - 1) / kThreads;
+        if (blocks > limit) blocks = limit;
+        if (blocks > kMaxBlocks) blocks = kMaxBlocks;
+        pick_reduced_kernel(pd, bcast)<<<static_cast<unsigned int>(blocks), kThreads, 0, s>>>(prm, d);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(ZERO_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
+    return ZERO_OK;
+}
+
 }  // namespace
 }  // namespace fused
 }  // namespace zero
@@ -182,25 +218,54 @@ extern "C" int zero_adam_step_reduced(const float* reduced_grad, int64_t count, 
     prm.overflow = status;
     if (int rc = add_gate_and_clip(fn, &prm, gate, clip_sqnorm, max_norm)) return rc;
     if (work == 0) return zero::ok();
-    ReducedDevice* d = nullptr;
-    if (int rc = reduced_device(param_dtype, &d)) return rc;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const int64_t ntiles = prm.nvec > 0 ? (count - prm.head) / kReducedTile : 0;
-    if (ntiles >= 2 * static_cast<int64_t>(d->sms)) {
-        // the pipeline kernel takes the whole tiles; the rest goes through
-        // its scalar path
-        prm.tile = kReducedTile;
-        prm.nvec = ntiles * kReducedTile / kVec;
-        pick_reduced_pipe_kernel(param_dtype)<<<static_cast<unsigned int>(d->sms), kPipeThreads,
-                                                reduced_pipe_smem_bytes(kReducedTile), s>>>(prm);
-    } else {
-        const int64_t limit = static_cast<int64_t>(d->sms) * d->blocks_per_sm[param_dtype == ZERO_F16 ? 0 : 1];
-        int64_t blocks = (work + kThreads - 1) / kThreads;
-        if (blocks > limit) blocks = limit;
-        if (blocks > kMaxBlocks) blocks = kMaxBlocks;
-        pick_reduced_kernel(param_dtype)<<<static_cast<unsigned int>(blocks), kThreads, 0, s>>>(prm);
+    ParamDsts d{};
+    if (int rc = launch_reduced(fn, prm, d, work, param_dtype, false, stream)) return rc;
+    return zero::ok();
+}
+
+extern "C" int zero_adam_step_reduced_bcast(const float* reduced_grad, int64_t count, const float* master_in,
+                                            const float* m_in, const float* v_in, float* master_out, float* m_out,
+                                            float* v_out, void* const* param_dsts, int32_t n_dsts,
+                                            zero_dtype_t param_dtype, const zero_adam_hparams_t* hp, int32_t* status,
+                                            const int32_t* gate, const double* clip_sqnorm, float max_norm,
+                                            zero_stream_t stream) {
+    using namespace zero::fused;
+    const char* fn = "zero_adam_step_reduced_bcast";
+    if (!status) return fail(ZERO_ERR_ARG, "%s: NULL status", fn);
+    if (!zero::aligned(status, 4)) return fail(ZERO_ERR_ALIGN, "%s: status misaligned", fn);
+    if (!param_dsts || n_dsts < 1 || n_dsts > ZERO_MAX_WORLD)
+        return fail(ZERO_ERR_ARG, "%s: param_dsts must hold 1..%d destinations", fn, ZERO_MAX_WORLD);
+    StepParams prm{};
+    int64_t work = 0;
+    // the first destination stands for all in the shared checks
+    if (int rc = prepare_reduced(fn, reduced_grad, count, master_in, m_in, v_in, master_out, m_out, v_out,
+                                 param_dsts[0], param_dtype, hp, &prm, &work))
+        return rc;
+    prm.overflow = status;
+    if (int rc = add_gate_and_clip(fn, &prm, gate, clip_sqnorm, max_norm)) return rc;
+    if (work == 0) return zero::ok();
+    ParamDsts d{};
+    d.n = n_dsts;
+    const void* others[] = {reduced_grad, master_in, m_in, v_in, master_out, m_out, v_out};
+    bool same_phase = true;
+    for (int k = 0; k < n_dsts; ++k) {
+        if (!param_dsts[k]) return fail(ZERO_ERR_ARG, "%s: param_dsts[%d] is NULL", fn, k);
+        if (!zero::aligned(param_dsts[k], 2)) return fail(ZERO_ERR_ALIGN, "%s: param_dsts[%d] misaligned", fn, k);
+        for (const void* o : others)
+            if (zero::overlaps(param_dsts[k], count * 2, o, count * 4))
+                return fail(ZERO_ERR_ARG, "%s: param_dsts[%d] overlaps an input or state array", fn, k);
+        for (int j = 0; j < k; ++j)
+            if (zero::overlaps(param_dsts[k], count * 2, param_dsts[j], count * 2))
+                return fail(ZERO_ERR_ARG, "%s: param_dsts[%d] overlaps param_dsts[%d]", fn, k, j);
+        same_phase = same_phase && ((reinterpret_cast<uintptr_t>(param_dsts[k]) -
+                                     reinterpret_cast<uintptr_t>(param_dsts[0])) % 16) == 0;
+        d.dst[k] = param_dsts[k];
     }
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return fail(ZERO_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
+    if (!same_phase) {      // the destinations' 16-byte phases differ: element-wise stores only
+        prm.head = count;
+        prm.nvec = 0;
+        work = count;
+    }
+    if (int rc = launch_reduced(fn, prm, d, work, param_dtype, true, stream)) return rc;
     return zero::ok();
 }

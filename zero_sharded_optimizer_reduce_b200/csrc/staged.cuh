@@ -12,6 +12,43 @@ namespace zero {
 namespace fused {
 namespace {
 
+// Destinations of the updated parameters when they are broadcast: this
+// rank's slot in every rank's parameter buffer (peers' buffers mapped into
+// this process), i.e. the all-gather done by the update's own stores.
+struct ParamDsts {
+    void* dst[ZERO_MAX_WORLD];  // each already offset to the call's first element
+    int32_t n;
+};
+
+// Parameter stores of 8, 4 or 1 element(s) at element e: to p.param_out, or
+// (kBcast) to every destination in d.
+template <bool kBcast>
+__device__ __forceinline__ void store_params8(const StepParams& p, const ParamDsts& d, int64_t e, uint4 q) {
+    if constexpr (kBcast) {
+        for (int k = 0; k < d.n; ++k) st_u16x8(static_cast<uint16_t*>(d.dst[k]) + e, q);
+    } else {
+        st_u16x8(static_cast<uint16_t*>(p.param_out) + e, q);
+    }
+}
+
+template <bool kBcast>
+__device__ __forceinline__ void store_params4(const StepParams& p, const ParamDsts& d, int64_t e, uint2 q) {
+    if constexpr (kBcast) {
+        for (int k = 0; k < d.n; ++k) st_u16x4(static_cast<uint16_t*>(d.dst[k]) + e, q);
+    } else {
+        st_u16x4(static_cast<uint16_t*>(p.param_out) + e, q);
+    }
+}
+
+template <bool kBcast>
+__device__ __forceinline__ void store_param1(const StepParams& p, const ParamDsts& d, int64_t e, uint16_t q) {
+    if constexpr (kBcast) {
+        for (int k = 0; k < d.n; ++k) static_cast<uint16_t*>(d.dst[k])[e] = q;
+    } else {
+        static_cast<uint16_t*>(p.param_out)[e] = q;
+    }
+}
+
 __device__ __forceinline__ float4 ld_once16(const float* p) {
     const uint4 r = ld_grad16(p);
     return make_float4(__uint_as_float(r.x), __uint_as_float(r.y), __uint_as_float(r.z), __uint_as_float(r.w));
@@ -20,9 +57,11 @@ __device__ __forceinline__ float4 ld_once16(const float* p) {
 // p.grads[0] holds the reduced fp32 gradients g (already unscaled), indexed
 // like the state arrays; p.c.inv is 1, so adam() forms g * clip exactly as
 // the fused step forms (s * inv) * clip.  Gate and clip as in the fused
-// step; no flag or norm (the reduce-scatter produced them).
-template <typename PT>
-__global__ void __launch_bounds__(kThreads) adam_reduced_kernel(const __grid_constant__ StepParams p) {
+// step; no flag or norm (the reduce-scatter produced them).  kBcast: the
+// parameters go to every destination of d instead of p.param_out.
+template <typename PT, bool kBcast>
+__global__ void __launch_bounds__(kThreads) adam_reduced_kernel(const __grid_constant__ StepParams p,
+                                                                const __grid_constant__ ParamDsts d) {
     const int64_t tid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
     const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
     Consts c = p.c;
@@ -52,7 +91,7 @@ __global__ void __launch_bounds__(kThreads) adam_reduced_kernel(const __grid_con
         q.y = Fmt<PT>::pack(pw[2], pw[3]);
         q.z = Fmt<PT>::pack(pw[4], pw[5]);
         q.w = Fmt<PT>::pack(pw[6], pw[7]);
-        st_u16x8(static_cast<uint16_t*>(p.param_out) + e0, q);
+        store_params8<kBcast>(p, d, e0, q);
     }
 
     // head and tail, one element per thread and iteration
@@ -65,7 +104,7 @@ __global__ void __launch_bounds__(kThreads) adam_reduced_kernel(const __grid_con
         p.master_out[e] = pw;
         p.m_out[e] = mw;
         p.v_out[e] = vw;
-        static_cast<uint16_t*>(p.param_out)[e] = Fmt<PT>::round1(pw);
+        store_param1<kBcast>(p, d, e, Fmt<PT>::round1(pw));
     }
 }
 
@@ -80,8 +119,9 @@ __global__ void __launch_bounds__(kThreads) adam_reduced_kernel(const __grid_con
 // Stages of the pipeline kernel's ring.
 constexpr int kReducedStages = 2;
 
-template <typename PT>
-__global__ void __launch_bounds__(kPipeThreads, 1) adam_reduced_pipe_kernel(const __grid_constant__ StepParams p) {
+template <typename PT, bool kBcast>
+__global__ void __launch_bounds__(kPipeThreads, 1) adam_reduced_pipe_kernel(const __grid_constant__ StepParams p,
+                                                                            const __grid_constant__ ParamDsts d) {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t full[kReducedStages];
     __shared__ __align__(8) uint64_t empty[kReducedStages];
@@ -178,7 +218,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) adam_reduced_pipe_kernel(cons
                 uint2 pk;
                 pk.x = Fmt<PT>::pack(pw[0], pw[1]);
                 pk.y = Fmt<PT>::pack(pw[2], pw[3]);
-                st_u16x4(static_cast<uint16_t*>(p.param_out) + base + j, pk);
+                store_params4<kBcast>(p, d, base + j, pk);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
@@ -195,7 +235,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) adam_reduced_pipe_kernel(cons
             p.master_out[e] = pw;
             p.m_out[e] = mw;
             p.v_out[e] = vw;
-            static_cast<uint16_t*>(p.param_out)[e] = Fmt<PT>::round1(pw);
+            store_param1<kBcast>(p, d, e, Fmt<PT>::round1(pw));
         }
     }
 }

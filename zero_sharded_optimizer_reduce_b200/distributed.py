@@ -25,7 +25,10 @@ bytes) plus the partition's reduced fp32 gradients (4 Psi / N): step 2 is
 the staged reduce-scatter (the same peer reads, storing the reduced
 gradients and the flag), the flags are OR-ed over the group, and only when
 no rank overflowed does every rank run the update from its reduced
-gradients in place, writing its slot of the parameter buffer directly.
+gradients in place.  That update stores the new parameters of its slot
+straight into every rank's parameter buffer (peer stores through the same
+mappings), so the all-gather needs no step of its own: one barrier after
+the update and every rank holds every slot.
 
 No kernel waits on another rank: all cross-rank ordering is host barriers,
 so the ranks may also share one GPU (each with its own context).  This class
@@ -36,7 +39,7 @@ from __future__ import annotations
 import torch
 import torch.distributed as dist
 
-from . import (DevicePtr, hparams, zero_adam_step_reduced, zero_allgather_params, zero_ipc_close,
+from . import (DevicePtr, hparams, zero_adam_step_reduced_bcast, zero_allgather_params, zero_ipc_close,
                zero_ipc_export, zero_ipc_import, zero_loss_scale_update, zero_partition_layout,
                zero_reduce_scatter_adam_step, zero_reduce_scatter_grads)
 
@@ -161,11 +164,15 @@ class DistributedZeroAdam:
         applied = ovf == 0
         if applied and self.mode == "staged":
             # every rank knows the verdict of the whole group: update in place
+            # and store slot r of every rank's parameter buffer
             for b in range(L.n_buckets):
                 P = L.part(b)
                 st = (self.master[b][0], self.m[b][0], self.v[b][0])
-                zero_adam_step_reduced(self.reduced[b], P, *st, *st, self.params[b][r * P:(r + 1) * P], hp,
-                                       self.flags[1:2])
+                esz = self.params[b].element_size()
+                dsts = [self.params[b][r * P:(r + 1) * P] if q == r else
+                        DevicePtr(self.peer_params[b][q].data_ptr() + r * P * esz, self.param_dtype)
+                        for q in range(self.world)]
+                zero_adam_step_reduced_bcast(self.reduced[b], P, *st, *st, dsts, hp, self.flags[1:2])
             if int(self.flags[1].item()) & 2:
                 raise RuntimeError("staged update timed out waiting on its copy pipeline; states incomplete")
             self.t += 1
@@ -177,7 +184,10 @@ class DistributedZeroAdam:
             self.t += 1
         self.scale, self.good_steps = zero_loss_scale_update(self.scale, self.good_steps, not applied,
                                                              self.growth_interval, self.min_scale)
-        if applied:
+        if applied and self.mode == "staged":
+            torch.cuda.synchronize()
+            dist.barrier(group=self.group)              # every rank's slot is in every buffer
+        elif applied:
             torch.cuda.synchronize()
             dist.barrier(group=self.group)              # every rank's own slot is updated
             for b in range(L.n_buckets):
