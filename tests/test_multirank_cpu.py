@@ -76,3 +76,35 @@ def test_reference_arm_two_ranks_only_rank0_prints():
     line = json.loads(outs[0].splitlines()[-1])
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def _verdict_worker(rank, world, port, flags, q):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from zero_sharded_optimizer_reduce_b200.distributed import DistributedZeroAdam
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        opt = object.__new__(DistributedZeroAdam)      # only the group-verdict logic, no device state
+        opt.group, opt.device = None, "cpu"
+        q.put((rank, [opt._or_over_ranks(f[rank]) for f in flags]))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_distributed_step_verdict_is_shared_by_every_rank():
+    """DistributedZeroAdam's skip decision: every rank's local flag word is
+    OR-ed (max) over the group, so one rank's overflow (1) or pipeline
+    timeout (2) makes every rank skip."""
+    world, port = 3, _free_port()
+    flags = [(0, 0, 0), (0, 1, 0), (2, 0, 0), (1, 1, 1)]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_verdict_worker, args=(r, world, port, flags, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    assert all(r[1] == [0, 1, 2, 1] for r in res)
