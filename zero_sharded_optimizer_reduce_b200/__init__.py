@@ -76,11 +76,14 @@ class AdamHParams(ctypes.Structure):
                 ("step", ctypes.c_int64), ("grad_divisor", ctypes.c_float)]
 
 
-def _load():
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with "
+def load_library(path: str = LIB_PATH):
+    """Load a build of libzero (this package's, or a variant such as the
+    bounds-checking debug build) and declare its signatures.  The wrappers
+    call the module-level `lib`; tests may swap it for a variant."""
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with "
                           "`python zero_sharded_optimizer_reduce_b200/build.py` (nvcc, sm_100a)")
-    L = ctypes.CDLL(LIB_PATH)
+    L = ctypes.CDLL(path)
     vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
     L.zero_partition_layout.argtypes = [ctypes.POINTER(ctypes.c_int64), i64, i32, i64, i32,
                                         ctypes.POINTER(_Layout)]
@@ -155,7 +158,7 @@ def _load():
     return L
 
 
-lib = _load()
+lib = load_library()
 
 
 def _check(rc: int) -> None:

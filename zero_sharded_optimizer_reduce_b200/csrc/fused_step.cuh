@@ -169,6 +169,24 @@ __device__ __forceinline__ double warp_sum_d(double x) {
     return x;
 }
 
+// Flag bit of debug builds (ZERO_DEBUG_BOUNDS): an index check failed.
+constexpr int32_t kFlagBounds = 4;
+
+// Index check of debug builds: when `ok` is false, record kFlagBounds in
+// *flag and return true so that the caller skips the access.  In release
+// builds it is the constant false and compiles away.
+__device__ __forceinline__ bool out_of_bounds(bool ok, int32_t* flag) {
+#ifdef ZERO_DEBUG_BOUNDS
+    if (!ok) {
+        atomicOr(flag, kFlagBounds);
+        return true;
+    }
+#endif
+    (void)ok;
+    (void)flag;
+    return false;
+}
+
 // Gate and clip, read once per thread from device memory: returns false
 // (write nothing) when the gate is set; otherwise sets c.clip from the
 // global squared norm, min(1, max_norm / (sqrt(sqnorm) + 1e-6)) computed in
@@ -193,6 +211,7 @@ __device__ __forceinline__ void scalar_elements(const StepParams& p, const Const
     const int64_t nscalar = p.head + (p.count - vec_end);
     for (int64_t q = tid; q < nscalar; q += nthreads) {
         const int64_t e = q < p.head ? q : vec_end + (q - p.head);
+        if (out_of_bounds(e >= 0 && e < p.count, p.overflow)) continue;
         float s = Fmt<GT>::one(static_cast<const uint16_t*>(p.grads[0])[e]);
         for (int k = 1; k < world; ++k)
             s = __fadd_rn(s, Fmt<GT>::one(static_cast<const uint16_t*>(p.grads[k])[e]));
@@ -259,6 +278,7 @@ __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_const
     // ---- vector path: kVec elements per iteration, 16-byte accesses
     for (int64_t vi = tid; vi < p.nvec; vi += nthreads) {
         const int64_t e0 = p.head + vi * kVec;
+        if (out_of_bounds(e0 + kVec <= p.count, p.overflow)) continue;
         // state first, so that its loads are in flight while gradients arrive
         const float4 pa = ld_state16(p.master_in + e0), pb = ld_state16(p.master_in + e0 + 4);
         const float4 ma = ld_state16(p.m_in + e0), mb = ld_state16(p.m_in + e0 + 4);
@@ -432,9 +452,13 @@ __global__ void __launch_bounds__(kPipeThreads, 1) fused_step_pipe_kernel(const 
             }
             if (__shfl_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&abort_flag), 0)) break;
             unsigned char* st = smem + static_cast<size_t>(s) * stage;
+            const int64_t e0 = p.head + tile * T;
+            if (out_of_bounds(e0 + T <= p.count, p.overflow)) {   // uniform over the warp
+                if (lane == 0) abort_flag = 1;
+                break;
+            }
             if (lane == 0) mbar_arrive_expect_tx(&full[s], stage);
             __syncwarp();
-            const int64_t e0 = p.head + tile * T;
             for (int q = lane; q < world + 3; q += 32) {
                 if (q < 3) {
                     const float* src = q == 0 ? p.master_in : (q == 1 ? p.m_in : p.v_in);
@@ -479,6 +503,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) fused_step_pipe_kernel(const 
             const int64_t base = p.head + tile * T;
             for (int ch = t; ch < T / 4; ch += C) {
                 const int j = 4 * ch;
+                if (out_of_bounds(j + 4 <= T && base + j + 4 <= p.count, p.overflow)) continue;
                 float sacc[4];
                 const uint2 r0 = *reinterpret_cast<const uint2*>(st + 2 * j);
                 sacc[0] = Fmt<GT>::lo(r0.x);

@@ -31,6 +31,7 @@ __device__ __forceinline__ void stats_scalar_elements(const StepParams& p, float
     const int64_t nscalar = p.head + (p.count - vec_end);
     for (int64_t q = tid; q < nscalar; q += nthreads) {
         const int64_t e = q < p.head ? q : vec_end + (q - p.head);
+        if (out_of_bounds(e >= 0 && e < p.count, p.overflow)) continue;
         const float s = replica_sum<GT>(p, e);
         bad |= !isfinite(s);
         const float g = __fmul_rn(s, inv);
@@ -57,6 +58,7 @@ __global__ void __launch_bounds__(kThreads) grad_stats_kernel(const __grid_const
     double sq = 0.0;
     for (int64_t vi = tid; vi < p.nvec; vi += nthreads) {
         const int64_t e0 = p.head + vi * kVec;
+        if (out_of_bounds(e0 + kVec <= p.count, p.overflow)) continue;
         float s[kVec];
         {
             uint4 r[kBatch];
@@ -141,9 +143,13 @@ __global__ void __launch_bounds__(kPipeThreads, 1) grad_stats_pipe_kernel(const 
             }
             if (__shfl_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&abort_flag), 0)) break;
             unsigned char* st = smem + static_cast<size_t>(s) * stage;
+            const int64_t e0 = p.head + tile * T;
+            if (out_of_bounds(e0 + T <= p.count, p.overflow)) {   // uniform over the warp
+                if (lane == 0) abort_flag = 1;
+                break;
+            }
             if (lane == 0) mbar_arrive_expect_tx(&full[s], stage);
             __syncwarp();
-            const int64_t e0 = p.head + tile * T;
             for (int k = lane; k < world; k += 32)
                 bulk_load(st + static_cast<size_t>(k) * gbytes, static_cast<const uint16_t*>(p.grads[k]) + e0, gbytes,
                           &full[s]);
@@ -176,6 +182,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) grad_stats_pipe_kernel(const 
             const int64_t base = p.head + tile * T;
             for (int ch = t; ch < T / 4; ch += C) {
                 const int j = 4 * ch;
+                if (out_of_bounds(j + 4 <= T && base + j + 4 <= p.count, p.overflow)) continue;
                 const uint2 r0 = *reinterpret_cast<const uint2*>(st + 2 * j);
                 float a0 = Fmt<GT>::lo(r0.x), a1 = Fmt<GT>::hi(r0.x), a2 = Fmt<GT>::lo(r0.y), a3 = Fmt<GT>::hi(r0.y);
 #pragma unroll 4

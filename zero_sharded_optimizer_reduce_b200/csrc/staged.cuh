@@ -70,6 +70,7 @@ __global__ void __launch_bounds__(kThreads) adam_reduced_kernel(const __grid_con
 
     for (int64_t vi = tid; vi < p.nvec; vi += nthreads) {
         const int64_t e0 = p.head + vi * kVec;
+        if (out_of_bounds(e0 + kVec <= p.count, p.overflow)) continue;
         const float4 ga = ld_once16(gin + e0), gb = ld_once16(gin + e0 + 4);
         const float4 pa = ld_state16(p.master_in + e0), pb = ld_state16(p.master_in + e0 + 4);
         const float4 ma = ld_state16(p.m_in + e0), mb = ld_state16(p.m_in + e0 + 4);
@@ -99,6 +100,7 @@ __global__ void __launch_bounds__(kThreads) adam_reduced_kernel(const __grid_con
     const int64_t nscalar = p.head + (p.count - vec_end);
     for (int64_t q = tid; q < nscalar; q += nthreads) {
         const int64_t e = q < p.head ? q : vec_end + (q - p.head);
+        if (out_of_bounds(e >= 0 && e < p.count, p.overflow)) continue;
         float pw = p.master_in[e], mw = p.m_in[e], vw = p.v_in[e];
         adam(gin[e], pw, mw, vw, c);
         p.master_out[e] = pw;
@@ -161,9 +163,13 @@ __global__ void __launch_bounds__(kPipeThreads, 1) adam_reduced_pipe_kernel(cons
             }
             if (__shfl_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&abort_flag), 0)) break;
             unsigned char* st = smem + static_cast<size_t>(s) * stage;
+            const int64_t e0 = p.head + tile * T;
+            if (out_of_bounds(e0 + T <= p.count, p.overflow)) {   // uniform over the warp
+                if (lane == 0) abort_flag = 1;
+                break;
+            }
             if (lane == 0) mbar_arrive_expect_tx(&full[s], stage);
             __syncwarp();
-            const int64_t e0 = p.head + tile * T;
             if (lane < 4) {
                 const float* src = lane == 0 ? static_cast<const float*>(p.grads[0])
                                              : (lane == 1 ? p.master_in : (lane == 2 ? p.m_in : p.v_in));
@@ -202,6 +208,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) adam_reduced_pipe_kernel(cons
             const int64_t base = p.head + tile * T;
             for (int ch = t; ch < T / 4; ch += C) {
                 const int j = 4 * ch;
+                if (out_of_bounds(j + 4 <= T && base + j + 4 <= p.count, p.overflow)) continue;
                 const float4 g4 = *reinterpret_cast<const float4*>(sg + j);
                 const float4 p4 = *reinterpret_cast<const float4*>(sp + j);
                 const float4 m4 = *reinterpret_cast<const float4*>(sm + j);
@@ -230,6 +237,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) adam_reduced_pipe_kernel(cons
         for (int64_t q = static_cast<int64_t>(blockIdx.x) * C + t; q < nscalar;
              q += static_cast<int64_t>(gridDim.x) * C) {
             const int64_t e = q < p.head ? q : vec_end + (q - p.head);
+            if (out_of_bounds(e >= 0 && e < p.count, p.overflow)) continue;
             float pw = p.master_in[e], mw = p.m_in[e], vw = p.v_in[e];
             adam(gin[e], pw, mw, vw, c);
             p.master_out[e] = pw;
