@@ -17,8 +17,6 @@ import numpy as np
 import pytest
 import torch
 
-import oracle
-import workloads
 import zero_sharded_optimizer_reduce_b200 as Z
 from _gpu import Guarded, host_u16
 from test_gpu_staged import Staged
