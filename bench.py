@@ -152,7 +152,8 @@ def source_digest(files=("fused_step.cuh",)) -> str:
 
 # timed kernel -> (committed ncu traffic record, the sources it was taken on)
 TRAFFIC_RECORDS = {"fused": ("fused_step_traffic.json", ("fused_step.cuh",)),
-                   "staged": ("adam_reduced_traffic.json", ("fused_step.cuh", "staged.cuh"))}
+                   "staged": ("adam_reduced_traffic.json", ("fused_step.cuh", "staged.cuh")),
+                   "staged_step": ("staged_step_traffic.json", ("fused_step.cuh", "grad_stats.cuh", "staged.cuh"))}
 
 
 def profiled_traffic(elems_per_launch: float, kernel: str = "fused"):
@@ -363,14 +364,17 @@ def run_gpu(args):
     ms_per_step = ms / args.steps
     value = whole_job_gparams(psi_p, world_gpus, ms_per_step)
     bpe = step_bytes_per_elem(w.world, args.mode, args.max_grad_norm is not None)
-    kbpe = update_bytes_per_elem(w.world, args.mode)
+    # the runner's whole step (b = -1) is timed as one unit: every byte of the step
+    kbpe = bpe if -1 in ev else update_bytes_per_elem(w.world, args.mode)
     peak, peak_kind = peaks()
     kern_bytes = sum(launch_elems) * kbpe
     kern_s = sum(launch_ms) * 1e-3
     achieved = kern_bytes / kern_s / 1e9
     avg_elems = sum(launch_elems) / len(launch_elems)
-    traffic = (profiled_traffic(avg_elems, "staged") if args.mode == "staged" else
-               profiled_traffic(avg_elems) if args.mode == "banks" else None)
+    if args.mode == "staged":
+        traffic = profiled_traffic(avg_elems, "staged_step" if -1 in ev else "staged")
+    else:
+        traffic = profiled_traffic(avg_elems) if args.mode == "banks" else None
 
     # ---- end to end through the public API: host gradients in, flag out
     e2e = None
@@ -399,14 +403,16 @@ def run_gpu(args):
                 "hbm_gbs": value * 1e9 * bpe / world_gpus / 1e9,
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
                              "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
-                             "kernel": ("fused_step (shared-memory pipeline kernel for aligned calls of >= 2 tiles per SM); "
+                             "kernel": ("staged step (reduce-scatter to fp32 + update from it, pipeline kernels); "
+                                        "timed per step over all buckets" if args.mode == "staged" and -1 in ev else
+                                        "fused_step (shared-memory pipeline kernel for aligned calls of >= 2 tiles per SM); "
                                         "timed per step over all buckets" if -1 in ev else
                                         "adam_reduced_kernel (update from the fp32 reduced gradients)"
                                         if args.mode == "staged" else
                                         "fused_step (shared-memory pipeline kernel for aligned calls of >= 2 tiles per SM)"),
                              "bytes_per_elem": kbpe,
                              "elems_per_launch": avg_elems, "launches_timed": len(launch_ms),
-                             "timed_unit": ("one step: all buckets' kernels + flag clear + 4-byte read-back"
+                             "timed_unit": ("one step: all buckets' kernels + flag clear + flag read-back"
                                             if -1 in ev else "one bucket's kernel")},
                 "gpu_launches": args.steps * L.n_buckets * (2 if opt.two_pass else 1),
                 "applied_steps": applied,

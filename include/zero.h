@@ -516,6 +516,34 @@ int zero_runner_create(const zero_bucket_banks_t* buckets, int64_t n_buckets, in
                        float loss_scale, int32_t growth_interval, float min_scale,
                        int32_t* flag_dev, int32_t* flag_host, double* grad_sqnorm, void* workspace,
                        zero_runner_t** out);
+/*
+ * zero_runner_create_staged - a runner for the staged route with one bank.
+ *
+ * launch enqueues: clear flag_dev[0..1] (and *grad_sqnorm); for every bucket
+ * zero_reduce_scatter_grads into reduced[b] (flag_dev[0], the norm); then for
+ * every bucket zero_adam_step_reduced in place on bank 0 (master[0], m[0],
+ * v[0], params[0]) with gate = flag_dev[0], status = flag_dev[1] and, when
+ * max_norm > 0, clipping by the step's norm; then a copy of both flag words
+ * into flag_host[0..1].  commit: as for the two-bank runner, except that the
+ * bank never changes (an overflowing step wrote nothing); t advances on
+ * applied steps.  Bank 1 of the bucket descriptors is not used (may be NULL).
+ *
+ * reduced      host array of n_buckets device fp32 pointers, padded_numel
+ *              elements each (caller-owned)
+ * max_norm     0: no clipping; > 0: clip to this global norm (needs
+ *              grad_sqnorm and workspace)
+ * flag_dev     2 device int32 words, 8-byte aligned; flag_host 2 host words
+ * other arguments: as for zero_runner_create.  set_state accepts bank 0 only.
+ * Errors: those of zero_reduce_scatter_grads and zero_adam_step_reduced;
+ * ZERO_ERR_ARG as for zero_runner_create; ZERO_ERR_CUDA from commit on a
+ * pipeline timeout (bit 1 of either word).
+ */
+int zero_runner_create_staged(const zero_bucket_banks_t* buckets, int64_t n_buckets, int32_t world,
+                              zero_dtype_t grad_dtype, zero_dtype_t param_dtype, const zero_adam_hparams_t* hp,
+                              float loss_scale, int32_t growth_interval, float min_scale,
+                              float* const* reduced, float max_norm,
+                              int32_t* flag_dev, int32_t* flag_host, double* grad_sqnorm, void* workspace,
+                              zero_runner_t** out);
 int zero_runner_launch(zero_runner_t* runner, zero_stream_t stream);
 int zero_runner_commit(zero_runner_t* runner, zero_stream_t stream, int32_t* applied);
 int zero_runner_state(const zero_runner_t* runner, int64_t* t, float* loss_scale, int32_t* good_steps,

@@ -361,3 +361,26 @@ def test_broadcast_update_rejects_bad_destinations():
     assert call([0x7E00_0000, st[0] + 16]) == -1                    # destination overlaps master_in
     assert L.zero_adam_step_reduced_bcast(red, 0, *st, (ctypes.c_void_p * 1)(0x7E00_0000), 1, 0,
                                           ctypes.byref(hp), status, None, None, 0.0, None) == 0
+
+
+def test_staged_runner_rejects_bad_arguments():
+    L = Z.lib
+    hp = Z.hparams()
+    grads = (ctypes.c_void_p * 2)(0x10000, 0x20000)
+    desc = (Z.BucketBanks * 1)()
+    desc[0].padded_numel = 64
+    desc[0].grad_bufs = ctypes.cast(grads, ctypes.POINTER(ctypes.c_void_p))
+    red = (ctypes.c_void_p * 1)(0x30000)
+    out = ctypes.c_void_p()
+
+    def call(reduced=red, max_norm=0.0, flag=0x40000, sq=None, ws=None):
+        return L.zero_runner_create_staged(desc, 1, 2, 0, 0, ctypes.byref(hp), 1024.0, 1000, 1.0,
+                                           None if reduced is None else ctypes.cast(reduced, ctypes.POINTER(ctypes.c_void_p)),
+                                           max_norm, flag, 0x50000, sq, ws, ctypes.byref(out))
+    assert call(reduced=None) == -1                       # no reduced-gradient buffers
+    assert call(reduced=(ctypes.c_void_p * 1)(0)) == -1    # NULL reduced buffer
+    assert call(max_norm=-1.0) == -1
+    assert call(max_norm=float("nan")) == -1
+    assert call(max_norm=1.0) == -1                       # clipping without a norm
+    assert call(sq=0x60000) == -1                         # a norm without a workspace
+    assert call(flag=0x40004) == -2                       # the two flag words must be 8-byte aligned

@@ -337,3 +337,35 @@ def test_runner_protocol_and_state():
         a_state = [x.clone() for x in (a.master[bk][bank], a.m[bk][bank], a.v[bk][bank], a.params_bank[bk][bank])]
         for x, y in zip(a_state, b.state(bk)):
             assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
+
+
+def test_staged_runner_protocol_and_state():
+    """The native runner on the staged route: one bank, bank 0 stays current,
+    an injected inf skips the step (states bit-identical), and its steps
+    equal the per-bucket Python path of the same mode."""
+    numels = [700_001, 13]
+    N = 4
+    adam = workloads.AdamConfig(weight_decay=0.01)
+    L, a, _ = _opt_and_oracle(numels, N, 0, adam, "staged")
+    _, b, _ = _opt_and_oracle(numels, N, 0, adam, "staged")
+    assert a._runner is not None
+    r = a._runner
+    for step in (1, 2, 3):
+        G = _grads_for(L, N, step, a.scale)
+        if step == 2:
+            workloads.inject(G[0][3], np.array([5]), np.array([False]))
+        _upload(a, G)
+        _upload(b, G)
+        before = [x.clone() for x in a.state(0)]
+        applied = a.step()                      # runner
+        b.launch()                              # per-bucket Python path
+        assert b.commit() == applied == (step != 2)
+        if step == 2:
+            for x, y in zip(before, a.state(0)):
+                assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
+        for bk in range(L.n_buckets):
+            for x, y in zip(a.state(bk), b.state(bk)):
+                assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
+    assert r.state() == (2, 32768.0, 1, 0)
+    with pytest.raises(Z.ZeroError):
+        r.set_state(2, 32768.0, 1, 1)           # a staged runner has one bank

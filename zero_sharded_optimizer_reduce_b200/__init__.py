@@ -132,6 +132,10 @@ def load_library(path: str = LIB_PATH):
                                      ctypes.POINTER(AdamHParams), f32, i32, f32, vp, vp, vp, vp,
                                      ctypes.POINTER(vp)]
     L.zero_runner_create.restype = ctypes.c_int
+    L.zero_runner_create_staged.argtypes = [ctypes.POINTER(BucketBanks), i64, i32, ctypes.c_int, ctypes.c_int,
+                                            ctypes.POINTER(AdamHParams), f32, i32, f32, ctypes.POINTER(vp), f32,
+                                            vp, vp, vp, vp, ctypes.POINTER(vp)]
+    L.zero_runner_create_staged.restype = ctypes.c_int
     L.zero_runner_launch.argtypes = [vp, vp]
     L.zero_runner_launch.restype = ctypes.c_int
     L.zero_runner_commit.argtypes = [vp, vp, ctypes.POINTER(i32)]
@@ -451,11 +455,18 @@ class Runner:
     `buckets`: list of (grad_bufs, [master0, master1], [m0, m1], [v0, v1],
     [params0, params1]) tensors; flag_dev a device int32 tensor, flag_host a
     pinned int32 tensor; the tensors must outlive the runner.
+
+    With `reduced` (one fp32 tensor per bucket) the runner takes the staged
+    route on bank 0 only (zero_runner_create_staged): flag_dev and flag_host
+    then hold 2 words, bank 1 may be None, and max_norm > 0 clips.
     """
 
     def __init__(self, buckets, hp: AdamHParams, loss_scale: float, flag_dev, flag_host, grad_sqnorm=None,
-                 workspace=None, growth_interval: int = 1000, min_scale: float = 1.0):
+                 workspace=None, growth_interval: int = 1000, min_scale: float = 1.0, reduced=None,
+                 max_norm: float = 0.0):
         import torch
+        staged = reduced is not None
+        nbank = 1 if staged else 2
         descs = (BucketBanks * max(1, len(buckets)))()
         self._keep = []
         world = len(buckets[0][0]) if buckets else 1
@@ -466,20 +477,32 @@ class Runner:
             d = descs[i]
             d.padded_numel = n
             d.grad_bufs = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
-            for b in range(2):
+            for b in range(nbank):
                 d.master[b], d.m[b], d.v[b] = _state_args(n, ((f"bucket {i} master[{b}]", master[b]),
                                                               (f"bucket {i} m[{b}]", m[b]),
                                                               (f"bucket {i} v[{b}]", v[b])))
                 d.params[b] = _dev(params[b], n, f"bucket {i} params[{b}]")
         gd = _dtype_code(buckets[0][0][0]) if buckets else ZERO_F16
         pd = _dtype_code(buckets[0][4][0]) if buckets else ZERO_F16
-        if getattr(flag_host, "is_cuda", True) or flag_host.dtype != torch.int32 or flag_host.numel() < 1:
-            raise ZeroError(-1, "flag_host must be a host (pinned) int32 tensor")
+        words = 2 if staged else 1
+        if getattr(flag_host, "is_cuda", True) or flag_host.dtype != torch.int32 or flag_host.numel() < words:
+            raise ZeroError(-1, f"flag_host must be a host (pinned) int32 tensor of {words} word(s)")
+        flag = _dev(flag_dev, words, "flag_dev", torch.int32)
+        sq = _dev(grad_sqnorm, 1, "grad_sqnorm", torch.float64)
+        ws = _flag_args(flag_dev, grad_sqnorm, workspace)[2]
         h = ctypes.c_void_p()
-        _check(lib.zero_runner_create(descs, len(buckets), world, gd, pd, ctypes.byref(hp), float(loss_scale),
-                                      growth_interval, min_scale, *_flag_args(flag_dev, None, None)[:1],
-                                      _ptr(flag_host), *_flag_args(flag_dev, grad_sqnorm, workspace)[1:],
-                                      ctypes.byref(h)))
+        if staged:
+            red = (ctypes.c_void_p * max(1, len(buckets)))(
+                *[_dev(reduced[i], buckets[i][0][0].numel(), f"reduced[{i}]", _f32()) for i in range(len(buckets))])
+            self._keep.append(red)
+            _check(lib.zero_runner_create_staged(descs, len(buckets), world, gd, pd, ctypes.byref(hp),
+                                                 float(loss_scale), growth_interval, min_scale,
+                                                 ctypes.cast(red, ctypes.POINTER(ctypes.c_void_p)), float(max_norm),
+                                                 flag, _ptr(flag_host), sq, ws, ctypes.byref(h)))
+        else:
+            _check(lib.zero_runner_create(descs, len(buckets), world, gd, pd, ctypes.byref(hp), float(loss_scale),
+                                          growth_interval, min_scale, flag, _ptr(flag_host), sq, ws,
+                                          ctypes.byref(h)))
         self._h = h
 
     def launch(self, stream=None) -> None:

@@ -88,13 +88,19 @@ class ZeroAdam:
         # the single-pass banks mode runs through the native step runner:
         # one C call enqueues the whole step, one commits it
         self._runner = None
+        hp1 = hparams(lr, betas[0], betas[1], eps, weight_decay, 1, grad_divisor)
+        buckets = [(self.grads[b], self.master[b], self.m[b], self.v[b], self.params_bank[b])
+                   for b in range(L.n_buckets)]
         if not self.two_pass and L.n_buckets > 0:
             self._flag_pinned = torch.zeros(1, dtype=torch.int32, pin_memory=True)
-            buckets = [(self.grads[b], self.master[b], self.m[b], self.v[b], self.params_bank[b])
-                       for b in range(L.n_buckets)]
-            self._runner = Runner(buckets, hparams(lr, betas[0], betas[1], eps, weight_decay, 1, grad_divisor),
-                                  self.scale, self.flag, self._flag_pinned, self.sqnorm, self.workspace,
+            self._runner = Runner(buckets, hp1, self.scale, self.flag, self._flag_pinned, self.sqnorm, self.workspace,
                                   growth_interval, min_scale)
+        elif mode == "staged" and L.n_buckets > 0:
+            # the staged route is native too: both passes over every bucket in one C call
+            self._flag_pinned = torch.zeros(2, dtype=torch.int32, pin_memory=True)
+            self._runner = Runner(buckets, hp1, self.scale, self.flags, self._flag_pinned, self.sqnorm,
+                                  self.workspace, growth_interval, min_scale, reduced=self.reduced,
+                                  max_norm=max_grad_norm or 0.0)
 
     def _sync_runner(self) -> None:
         """Hand the Python-side step state to the runner."""
@@ -227,10 +233,11 @@ class ZeroAdam:
     def step(self, stream=None, on_launch=None) -> bool:
         """One whole step over all buckets; returns True if the update was applied.
 
-        In the single-pass banks mode the native runner enqueues and commits
-        the step; `on_launch(-1, phase)` then brackets the whole step's device
-        work (flag clear, every bucket's kernel, the flag read-back).
-        Otherwise `on_launch(b, phase)` brackets each bucket's kernel."""
+        In the single-pass banks mode and in the staged mode the native
+        runner enqueues and commits the step; `on_launch(-1, phase)` then
+        brackets the whole step's device work (flag clear, every bucket's
+        kernels, the flag read-back).  Otherwise `on_launch(b, phase)`
+        brackets each bucket's update kernel."""
         if self._runner is None:
             self.launch(stream, on_launch)
             return self.commit(stream)
