@@ -111,9 +111,12 @@ int launch_segments(const std::vector<Seg>& segs, int esize, cudaStream_t stream
         }
         if (max_bytes == 0) continue;
         // enough blocks to cover the largest segment with kUnroll 16-byte
-        // accesses per thread, at most ~8 resident blocks per SM in total
+        // accesses per thread, at most 16 blocks per SM in total (measured on
+        // B200, all-gather of 8 x 25M fp16 elements: 5.96 TB/s; with 8 per
+        // SM 5.78; 8-deep unrolling or non-streaming loads and stores were
+        // not faster)
         int64_t want = (max_bytes + int64_t(kThreads) * 16 * kUnroll - 1) / (int64_t(kThreads) * 16 * kUnroll);
-        int64_t cap = std::max<int64_t>(1, int64_t(sms) * 8 / int64_t(n));
+        int64_t cap = std::max<int64_t>(1, int64_t(sms) * 16 / int64_t(n));
         const unsigned int gx = static_cast<unsigned int>(std::max<int64_t>(1, std::min(want, cap)));
         copy_segments_kernel<<<dim3(gx, static_cast<unsigned int>(n)), kThreads, 0, stream>>>(prm);
         cudaError_t e = cudaGetLastError();
