@@ -108,3 +108,34 @@ def test_distributed_step_verdict_is_shared_by_every_rank():
         assert p.exitcode == 0
     res = sorted(q.get(timeout=10) for _ in range(world))
     assert all(r[1] == [0, 1, 2, 1] for r in res)
+
+
+def test_bench_byte_models():
+    """The bytes per element the benchmark divides by: the fused single pass
+    2N + 26, statistics + gated update 4N + 26, staged 2N + 34 (reduce-scatter
+    2N + 4, update 30); the update kernel alone in the staged mode is 30."""
+    sys.path.insert(0, ROOT)
+    import bench
+    for n in (1, 8, 64):
+        assert bench.bytes_per_elem(n) == 2 * n + 26
+        assert bench.step_bytes_per_elem(n, "banks", False) == 2 * n + 26
+        assert bench.step_bytes_per_elem(n, "banks", True) == 4 * n + 26
+        assert bench.step_bytes_per_elem(n, "inplace", False) == 4 * n + 26
+        assert bench.step_bytes_per_elem(n, "staged", False) == (2 * n + 4) + 30
+        assert bench.update_bytes_per_elem(n, "staged") == 30
+        assert bench.update_bytes_per_elem(n, "banks") == 2 * n + 26
+
+
+def test_bench_traffic_records_scale_with_elements():
+    sys.path.insert(0, ROOT)
+    import bench
+    for kind in bench.TRAFFIC_RECORDS:
+        a, b = bench.profiled_traffic(1e6, kind), bench.profiled_traffic(3e6, kind)
+        if a is None:                  # the record predates the current kernel source
+            assert b is None
+            continue
+        assert abs(b - 3 * a) < 1e-6 * b
+        # DRAM bytes never exceed the algorithmic bytes by more than a few percent
+        per = a / 1e6
+        bound = {"fused": 42, "staged": 30, "staged_step": 50}[kind]
+        assert 0.9 * bound <= per <= 1.05 * bound
