@@ -429,8 +429,10 @@ def run_gpu(args):
 def run_sweep(args):
     """Flat bandwidth sweep: psi in {1M, 16M, 256M, 1B, 2B} x N in {1..64}
     (N x 2 x psi <= 96 GB), fp16 and bf16; one JSON line per point.  Each
-    step is timed on its own with CUDA events; when a point's footprint is
-    below 4x L2 an L2-sized buffer is written between steps (untimed)."""
+    step is timed on its own with CUDA events, the median of at least 20
+    steps (at least --steps when a step moves more than 20 GB); when a
+    point's footprint is below 4x L2 an L2-sized buffer is written between
+    steps (untimed)."""
     import torch
     import zero_sharded_optimizer_reduce_b200 as Z
     torch.cuda.set_device(0)
@@ -456,7 +458,9 @@ def run_sweep(args):
             for _ in range(3):
                 opt.step()
             times = []
-            for _ in range(args.steps):
+            # median of >= 20 timed steps, >= 5 when a step moves more than 20 GB
+            reps = args.steps if psi * bpe > 20e9 else max(20, args.steps)
+            for _ in range(reps):
                 if small:
                     flush.fill_(1)
                 e0 = torch.cuda.Event(enable_timing=True)
@@ -473,7 +477,7 @@ def run_sweep(args):
             ms = statistics.median(times)
             gbs = psi * bpe / (ms * 1e-3) / 1e9
             print(json.dumps({"sweep": True, "psi": psi, "world": N, "grad_dtype": dt,
-                              "kernel_ms_median": ms, "gparams_s": psi / (ms * 1e-3) / 1e9, "gbs": gbs,
+                              "kernel_ms_median": ms, "reps": reps, "gparams_s": psi / (ms * 1e-3) / 1e9, "gbs": gbs,
                               "frac_measured": gbs / peak, "frac_nominal_8tbs": gbs / 8000.0,
                               "l2": "L2-influenced (footprint < 4x L2, flushed between steps)" if small
                               else "footprint > 4x L2"}), flush=True)
