@@ -565,3 +565,4 @@ def version() -> str:
 from .optimizer import ZeroAdam  # noqa: E402  (uses the bindings above)
 from .distributed import DistributedZeroAdam  # noqa: E402
 from .stage3 import ZeroStage3  # noqa: E402
+from .distributed_stage3 import DistributedZeroStage3  # noqa: E402
