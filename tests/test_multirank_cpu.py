@@ -84,18 +84,23 @@ def _verdict_worker(rank, world, port, flags, q):
     from zero_sharded_optimizer_reduce_b200.distributed import DistributedZeroAdam
     dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
     try:
-        opt = object.__new__(DistributedZeroAdam)      # only the group-verdict logic, no device state
-        opt.group, opt.device = None, "cpu"
-        q.put((rank, [opt._or_over_ranks(f[rank]) for f in flags]))
+        from zero_sharded_optimizer_reduce_b200.distributed_stage3 import DistributedZeroStage3
+        got = []
+        for cls in (DistributedZeroAdam, DistributedZeroStage3):
+            opt = object.__new__(cls)                  # only the group-verdict logic, no device state
+            opt.group, opt.device = None, "cpu"
+            got.append([opt._or_over_ranks(f[rank]) for f in flags])
+        q.put((rank, got))
         dist.barrier()
     finally:
         dist.destroy_process_group()
 
 
 def test_distributed_step_verdict_is_shared_by_every_rank():
-    """DistributedZeroAdam's skip decision: every rank's local flag word is
-    OR-ed (max) over the group, so one rank's overflow (1) or pipeline
-    timeout (2) makes every rank skip."""
+    """The multi-process steps' skip decision (DistributedZeroAdam per step,
+    DistributedZeroStage3 per unit): every rank's local flag word is OR-ed
+    (max) over the group, so one rank's overflow (1) or pipeline timeout (2)
+    makes every rank skip."""
     world, port = 3, _free_port()
     flags = [(0, 0, 0), (0, 1, 0), (2, 0, 0), (1, 1, 1)]
     ctx = mp.get_context("spawn")
@@ -107,7 +112,7 @@ def test_distributed_step_verdict_is_shared_by_every_rank():
         p.join(120)
         assert p.exitcode == 0
     res = sorted(q.get(timeout=10) for _ in range(world))
-    assert all(r[1] == [0, 1, 2, 1] for r in res)
+    assert all(r[1] == [[0, 1, 2, 1], [0, 1, 2, 1]] for r in res)
 
 
 def test_bench_byte_models():
