@@ -70,3 +70,27 @@ def test_staged_step_matches_oracle(world, per_rank, dtypes, offs, part, inplace
 def host_reduced(c):
     from _gpu import host_f32
     return host_f32(c.red.t).view(np.uint32)
+
+
+@settings(max_examples=25, deadline=None, derandomize=True)
+@given(numels=st.lists(st.integers(1, 3000), min_size=1, max_size=6), world=st.integers(1, 6),
+       cap=st.sampled_from([0, 1000, 4000]), dtype=st.sampled_from([oracle.F16, oracle.BF16]),
+       inject=st.booleans(), seed=st.integers(0, 1000))
+def test_oracle_stages_equal_plain_dp_on_random_layouts(numels, world, cap, dtype, inject, seed):
+    """The pages' drop-in claim on random layouts: plain DP, Stage 1, 2 and 3
+    of the oracle give bit-identical states after every step, with an
+    inf injected into one replica at step 2 (when `inject`), skipped by all."""
+    from test_oracle_stages import _assert_equal_states, _grads, _runs
+    adam = workloads.AdamConfig(weight_decay=0.01)
+    L, runs = _runs(numels, world, cap, adam, 1024.0, dtype, dtype, seed)
+    for step in (1, 2, 3):
+        G = _grads(L, step, seed, runs[0].scaler.scale, dtype, numels)
+        if inject and step == 2:
+            inf = workloads.F16_POS_INF if dtype == oracle.F16 else workloads.BF16_POS_INF
+            G[0][world - 1][0] = inf
+        flags = {s: r.step(G) for s, r in runs.items()}
+        assert set(flags.values()) == {int(inject and step == 2)}
+        for s in (1, 2, 3):
+            for b in range(L.n_buckets):
+                _assert_equal_states(runs[0].flat_state(b), runs[s].flat_state(b))
+        assert all(r.replicas_identical() for r in runs.values())
