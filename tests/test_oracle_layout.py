@@ -114,3 +114,14 @@ def test_allgather_with_offset_brute_force():
         got = oracle.allgather(shards, off, part)
         ref = np.concatenate([sh[off:off + part] for sh in shards])
         assert np.array_equal(got, ref)
+
+
+def test_bucket_filled_exactly_to_capacity():
+    """A constant-size buffer of capacity C takes tensors while their total
+    stays within C [ZeRO explainer, "Constant-size buffers"]: a bucket may end
+    exactly at C, and the next tensor opens a new one."""
+    L = oracle.partition_layout([3, 2, 5, 1, 4], 1, 5)
+    assert L.bucket_numel == [5, 5, 5]
+    assert L.bucket_tensors == [[0, 1], [2], [3, 4]]
+    L = oracle.partition_layout([3, 3], 1, 5)
+    assert L.bucket_numel == [3, 3]
