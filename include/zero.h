@@ -519,6 +519,11 @@ int zero_runner_create(const zero_bucket_banks_t* buckets, int64_t n_buckets, in
 /*
  * zero_runner_create_staged - a runner for the staged route with one bank.
  *
+ * Source: ZeRO explainer, "Stage 2 - Gradient Partitioning (P_os+g)" (the
+ * reduce-scatter leaves each rank the reduced gradients of its partition,
+ * which it then updates) and "Stage 1 - Optimizer State Partitioning (P_os)"
+ * (one copy of the optimizer states: 12 Psi / N bytes per rank).
+ *
  * launch enqueues: clear flag_dev[0..1] (and *grad_sqnorm); for every bucket
  * zero_reduce_scatter_grads into reduced[b] (flag_dev[0], the norm); then for
  * every bucket zero_adam_step_reduced in place on bank 0 (master[0], m[0],
