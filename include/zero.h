@@ -432,16 +432,25 @@ size_t zero_step_static_scratch_bytes(void);
  * r < world, j < part_numel: a bit-exact copy.  With shards that concatenate
  * each unit's slices in unit order, shard_offset selects one unit.
  *
- * shards       host array of `world` DEVICE pointers
+ * shards       host array of `world` DEVICE pointers (this GPU's memory, or
+ *              another GPU's memory mapped into this process: those slices
+ *              are read with plain loads)
  * world        1..ZERO_MAX_WORLD
  * shard_offset first element of the slice in every shard (>= 0)
- * part_numel   elements per rank (>= 0)
+ * part_numel   elements per rank (>= 0); any value: slices whose 16-byte
+ *              phase differs from their destination's are realigned in
+ *              registers, so odd sizes keep 16-byte loads and stores
  * dtype        ZERO_F16, ZERO_BF16 or ZERO_F32
  * dst          device, world*part_numel elements, must not overlap a shard
+ * status       device int32 or NULL, 4-byte aligned: bit 1 (value 2) is OR-ed
+ *              into it when a bounded wait of the bulk-copy kernel gave up (the
+ *              copy is then incomplete); never cleared by the call
+ * Reads whole aligned 16-byte blocks that hold at least one byte of a slice,
+ * so never a page outside the slices; writes exactly dst's range.
  * Errors: ZERO_ERR_ARG, ZERO_ERR_DTYPE, ZERO_ERR_ALIGN, ZERO_ERR_CUDA.
  */
 int zero_allgather_params(const void* const* shards, int32_t world, int64_t shard_offset,
-                          int64_t part_numel, zero_dtype_t dtype, void* dst,
+                          int64_t part_numel, zero_dtype_t dtype, void* dst, int32_t* status,
                           zero_stream_t stream);
 
 /*

@@ -207,15 +207,17 @@ def test_staged_reduce_scatter_rejects_bad_arguments():
 def test_allgather_and_flatten_reject_bad_arguments():
     L = Z.lib
     sh = (ctypes.c_void_p * 2)(0x10000, 0x20000)
-    assert L.zero_allgather_params(None, 2, 0, 8, 0, 0x30000, None) == -1
-    assert L.zero_allgather_params(sh, 0, 0, 8, 0, 0x30000, None) == -1
-    assert L.zero_allgather_params(sh, 2, -1, 8, 0, 0x30000, None) == -1
-    assert L.zero_allgather_params(sh, 2, 0, 8, 9, 0x30000, None) == -3
-    assert L.zero_allgather_params(sh, 2, 0, 8, 2, 0x30002, None) == -2
-    assert L.zero_allgather_params(sh, 2, 0, 8, 0, 0x10008, None) == -1   # dst overlaps shard 0
+    assert L.zero_allgather_params(None, 2, 0, 8, 0, 0x30000, None, None) == -1
+    assert L.zero_allgather_params(sh, 0, 0, 8, 0, 0x30000, None, None) == -1
+    assert L.zero_allgather_params(sh, 2, -1, 8, 0, 0x30000, None, None) == -1
+    assert L.zero_allgather_params(sh, 2, 0, 8, 9, 0x30000, None, None) == -3
+    assert L.zero_allgather_params(sh, 2, 0, 8, 2, 0x30002, None, None) == -2
+    assert L.zero_allgather_params(sh, 2, 0, 8, 0, 0x10008, None, None) == -1   # dst overlaps shard 0
     bad = (ctypes.c_void_p * 2)(0x10001, 0x20000)
-    assert L.zero_allgather_params(bad, 2, 0, 8, 0, 0x30000, None) == -2
-    assert L.zero_allgather_params(sh, 2, 0, 0, 0, 0x30000, None) == 0     # nothing to copy
+    assert L.zero_allgather_params(bad, 2, 0, 8, 0, 0x30000, None, None) == -2
+    assert L.zero_allgather_params(sh, 2, 0, 8, 0, 0x30000, 0x40002, None) == -2   # status misaligned
+    assert L.zero_allgather_params(sh, 2, 0, 8, 0, 0x30000, 0x30004, None) == -1   # status inside dst
+    assert L.zero_allgather_params(sh, 2, 0, 0, 0, 0x30000, None, None) == 0     # nothing to copy
     lay = Z.zero_partition_layout([5, 7], 2)._c()
     tp = (ctypes.c_void_p * 2)(0x10000, 0x20000)
     assert L.zero_flatten_bucket(None, 0, tp, 0, 0x30000, None) == -1

@@ -149,7 +149,7 @@ def load_library(path: str = LIB_PATH):
     L.zero_runner_destroy.restype = None
     L.zero_test_wait_timeout.argtypes = [vp, i64, vp]
     L.zero_test_wait_timeout.restype = ctypes.c_int
-    L.zero_allgather_params.argtypes = [ctypes.POINTER(vp), i32, i64, i64, ctypes.c_int, vp, vp]
+    L.zero_allgather_params.argtypes = [ctypes.POINTER(vp), i32, i64, i64, ctypes.c_int, vp, vp, vp]
     L.zero_allgather_params.restype = ctypes.c_int
     L.zero_loss_scale_update.argtypes = [ctypes.POINTER(f32), ctypes.POINTER(i32), i32, i32, f32]
     L.zero_loss_scale_update.restype = ctypes.c_int
@@ -433,11 +433,13 @@ def zero_adam_step_reduced_bcast(reduced_grad, count: int, master_in, m_in, v_in
         _stream(stream)))
 
 
-def zero_allgather_params(shards, shard_offset: int, part_numel: int, dst, stream=None) -> None:
-    """dst[r*part + j] = shards[r][shard_offset + j] (bit-exact copy)."""
+def zero_allgather_params(shards, shard_offset: int, part_numel: int, dst, stream=None, status=None) -> None:
+    """dst[r*part + j] = shards[r][shard_offset + j] (bit-exact copy); `status`
+    (device int32, optional) receives bit 1 if a copy wait timed out."""
+    import torch
     _check(lib.zero_allgather_params(_devs(shards, shard_offset + part_numel, "shards"), len(shards), shard_offset,
                                      part_numel, _dtype_code(dst), _dev(dst, len(shards) * part_numel, "dst"),
-                                     _stream(stream)))
+                                     _dev(status, 1, "status", torch.int32), _stream(stream)))
 
 
 def zero_loss_scale_update(scale: float, good_steps: int, overflow: bool,

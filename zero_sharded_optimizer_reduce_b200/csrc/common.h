@@ -2,6 +2,8 @@
 // argument checks.  No arithmetic of the method lives here.
 #pragma once
 
+#include <cuda_runtime.h>
+
 #include <cstdint>
 #include <cstdio>
 #include <string>
@@ -32,6 +34,33 @@ inline bool overlaps(const void* a, int64_t na, const void* b, int64_t nb) {
     if (na <= 0 || nb <= 0) return false;
     auto x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
     return x < y + static_cast<uintptr_t>(nb) && y < x + static_cast<uintptr_t>(na);
+}
+
+// True when `p` is device memory of device `dev` (not another GPU's memory
+// mapped into this process, not host memory).  Kernels that stage their
+// inputs with bulk copies take only such sources; other sources go to the
+// kernels that read with plain loads.  A failed query counts as "not local"
+// and its error is cleared, so that a launch check that follows is not
+// misled.
+inline bool local_device_memory(const void* p, int dev) {
+    cudaPointerAttributes a{};
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return false;
+    }
+    return a.type == cudaMemoryTypeDevice && a.device == dev;
+}
+
+// True when every one of the n pointers is device memory of the current device.
+inline bool all_local_device_memory(const void* const* ptrs, int n) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return false;
+    }
+    for (int i = 0; i < n; ++i)
+        if (!local_device_memory(ptrs[i], dev)) return false;
+    return true;
 }
 
 }  // namespace zero

@@ -298,15 +298,17 @@ inline int prepare_step(const char* fn, const void* const* grad_bufs, int32_t wo
     }
     prm.tile = 0;
 
-    // The pipeline kernel takes calls whose arrays share a 16-byte phase and
-    // that give every SM at least two tiles; the rest use the register kernel.
+    // The pipeline kernel takes calls whose arrays share a 16-byte phase, that
+    // give every SM at least two tiles and whose gradients are all this GPU's
+    // memory (its bulk copies never read another GPU's memory); the rest use
+    // the register kernel, whose plain loads read mapped peer memory too.
     int64_t blocks = 0;
     const int tile = h >= 0 ? pipe_tile(world) : 0;
     if (tile > 0) {
         int sms = 0;
         if (int rc = pipe_setup(grad_dtype, param_dtype, &sms)) return rc;
         const int64_t ntiles = (count - h) / tile;
-        if (ntiles >= 2 * static_cast<int64_t>(sms)) {
+        if (ntiles >= 2 * static_cast<int64_t>(sms) && all_local_device_memory(grad_bufs, world)) {
             prm.tile = tile;
             prm.nvec = ntiles * tile / kVec;
             blocks = sms;
@@ -412,13 +414,15 @@ inline int prepare_stats(const char* fn, const void* const* grad_bufs, int32_t w
         prm.nvec = (count - h) / kVec;
     }
     prm.tile = 0;
+    // pipeline kernel: as for the step, only when every gradient buffer is
+    // this GPU's memory
     int64_t blocks = 0;
     const int tile = h >= 0 ? stats_pipe_tile(world) : 0;
     if (tile > 0) {
         int sms = 0;
         if (int rc = stats_pipe_setup(grad_dtype, reduced != nullptr, &sms)) return rc;
         const int64_t ntiles = (count - h) / tile;
-        if (ntiles >= 2 * static_cast<int64_t>(sms)) {
+        if (ntiles >= 2 * static_cast<int64_t>(sms) && all_local_device_memory(grad_bufs, world)) {
             prm.tile = tile;
             prm.nvec = ntiles * tile / kVec;
             blocks = sms;
