@@ -1,13 +1,18 @@
 """zero_reduce_scatter_adam_step_noalloc: the fused step for callers that
 cannot allocate device memory.
 
-Such callers (code under an allocator that owns all device memory and forbids
-direct cudaMalloc, a host thread that must not take cudaMalloc's implicit
-synchronization, a C caller without a device allocator) cannot hand the
-library the workspace that the gradient norm needs.  This entry point keeps
-that scratch in a fixed array inside libzero instead.  The GPU test calls it
-through the C ABI twice in a row (the second call reuses the scratch the first
-one left behind) and checks every output against the regular entry point.
+Some callers have no way to hand the library the device workspace that the
+gradient norm needs: code running under an allocator that owns all device
+memory and forbids direct cudaMalloc, a host thread that must not take
+cudaMalloc's implicit device synchronization, or a plain C program with no
+device allocator.  This entry point keeps that scratch in a fixed array inside
+libzero instead.  The GPU test calls it through the C ABI twice in a row (the
+second call reuses the scratch the first one left behind) and checks every
+output against the regular entry point (same tolerance as the other parity
+tests, and in fact bit for bit, the norm included) and against the oracle.
+The cases reach both step kernels: the register kernel (a ragged size) and
+the shared-memory pipeline kernel (at least two tiles per SM), plus a call on
+a single partition.
 
 The file is named so that pytest collects it last.
 """
@@ -17,6 +22,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import workloads
 import zero_sharded_optimizer_reduce_b200 as Z
 from _gpu import assert_f32_close, assert_u16_close, host_f32, host_u16
@@ -46,42 +52,59 @@ def test_noalloc_entry_validates_like_the_regular_one():
     assert Z.lib.zero_step_static_scratch_bytes() == 256 + 8 * 4096
 
 
-def _inputs(world, n, seed):
-    dev = lambda a: torch.from_numpy(a).cuda()
-    grads = [dev(workloads.grads(n, seed + k, 1e-3, 65536.0).view(np.int16)).view(torch.float16)
-             for k in range(world)]
-    master = dev(workloads.master(n, seed + 100))
-    m = torch.zeros_like(master)
-    v = torch.zeros_like(master)
-    return grads, [master, m, v]
+ADAM = workloads.AdamConfig(weight_decay=0.01)
+SCALE = 65536.0
 
 
-def _run(entry, grads, state_in, t, world, n, use_ws):
+def _run(entry, grads, state_in, t, padded, partition, count, use_ws):
     out = [torch.empty_like(x) for x in state_in]
-    params = torch.empty(n, dtype=torch.float16, device="cuda")
+    params = torch.empty(count, dtype=torch.float16, device="cuda")
     flag = torch.zeros(1, dtype=torch.int32, device="cuda")
     norm = torch.zeros(1, dtype=torch.float64, device="cuda")
-    hp = Z.hparams(1e-3, 0.9, 0.999, 1e-8, 0.01, t)
+    hp = Z.hparams(ADAM.lr, ADAM.beta1, ADAM.beta2, ADAM.eps, ADAM.weight_decay, t)
     if use_ws:
         ws = torch.zeros(Z.zero_step_workspace_bytes(), dtype=torch.uint8, device="cuda")
-        entry(grads, n, Z.ZERO_ALL_PARTITIONS, *state_in, *out, params, hp, 65536.0, flag, norm, ws)
+        entry(grads, padded, partition, *state_in, *out, params, hp, SCALE, flag, norm, ws)
     else:
-        entry(grads, n, Z.ZERO_ALL_PARTITIONS, *state_in, *out, params, hp, 65536.0, flag, norm)
+        entry(grads, padded, partition, *state_in, *out, params, hp, SCALE, flag, norm)
     torch.cuda.synchronize()
     return out, params, int(flag.item()), float(norm.item())
 
 
 @pytest.mark.gpu
-def test_noalloc_matches_regular_entry_on_two_calls_in_a_row():
-    world, n = 8, 8 * 100_003 + 8          # several blocks and a ragged per-rank size
-    grads, state = _inputs(world, n, 4242)
-    ref_state, got_state = state, state
+@pytest.mark.parametrize("world,padded,partition", [
+    (8, 8 * 100_003 + 8, Z.ZERO_ALL_PARTITIONS),              # register kernel, ragged vector tail
+    (8, 8 * (2 * 148 * 3072 + 1000), Z.ZERO_ALL_PARTITIONS),  # pipeline kernel: >= 2 tiles of 3072 per SM
+    (8, 8 * 100_003 + 8, 3),                                   # one rank's partition
+])
+def test_noalloc_matches_regular_entry_and_oracle_on_two_calls_in_a_row(world, padded, partition):
+    P = padded // world
+    begin = 0 if partition < 0 else partition * P
+    count = padded if partition < 0 else P
+    G = [workloads.grads(padded, 4242 + k, 1e-3, SCALE) for k in range(world)]
+    master0 = workloads.master(count, 4342)
+    dev = lambda a: torch.from_numpy(a).cuda()
+    grads = [dev(g.view(np.int16)).view(torch.float16) for g in G]
+    ref = oracle.initial_state(master0)
+    start = [dev(master0.copy()), torch.zeros(count, device="cuda"), torch.zeros(count, device="cuda")]
+    reg_state, got_state = start, start
     for t in (1, 2):
-        ref = _run(Z.zero_reduce_scatter_adam_step, grads, ref_state, t, world, n, use_ws=True)
-        got = _run(Z.zero_reduce_scatter_adam_step_noalloc, grads, got_state, t, world, n, use_ws=False)
-        for a, b, name in zip(got[0], ref[0], ("master", "m", "v")):
-            assert_f32_close(host_f32(a), host_f32(b), f"{name} (call {t})")
-        assert_u16_close(host_u16(got[1]), host_u16(ref[1]), f"params (call {t})")
-        assert got[2] == ref[2] == 0
-        assert abs(got[3] - ref[3]) <= 1e-5 * ref[3] and ref[3] > 0
-        ref_state, got_state = ref[0], got[0]
+        reg = _run(Z.zero_reduce_scatter_adam_step, grads, reg_state, t, padded, partition, count, use_ws=True)
+        got = _run(Z.zero_reduce_scatter_adam_step_noalloc, grads, got_state, t, padded, partition, count,
+                   use_ws=False)
+        ovf, sq = oracle.flat_step(G, ref, ADAM, t, SCALE, float(world), begin=begin, count=count)
+        assert got[2] == reg[2] == ovf == 0
+        for a, b, exp, name in zip(got[0], reg[0], (ref.master, ref.m, ref.v), ("master", "m", "v")):
+            ga = host_f32(a)
+            # against the regular entry point: the parity tolerance, and bit for bit
+            assert assert_f32_close(ga, host_f32(b), f"{name} vs regular entry (call {t})") == 0
+            assert assert_f32_close(ga, exp, f"{name} vs oracle (call {t})") == 0
+        assert assert_u16_close(host_u16(got[1]), host_u16(reg[1]), f"params vs regular entry (call {t})") == 0
+        assert assert_u16_close(host_u16(got[1]), ref.params, f"params vs oracle (call {t})") == 0
+        # the same kernel on the same grid folds the same partial sums in the
+        # same order: the norms agree bit for bit; against the oracle's
+        # sequential fp64 sum of the same exact squares, within the bound of
+        # two fp64 summation orders
+        assert got[3] == reg[3] and sq > 0
+        assert abs(got[3] - sq) <= 2.0 * count * 2.0 ** -53 * sq
+        reg_state, got_state = reg[0], got[0]
