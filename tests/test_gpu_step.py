@@ -32,14 +32,16 @@ class Case:
     """Inputs of one step on the device (guarded) and on the host."""
 
     def __init__(self, padded, world, gdtype=oracle.F16, pdtype=oracle.F16, seed=0, scale=1024.0,
-                 partition=-1, goff=0, soff=0, poff=0, inplace=False, master=None, norm=False):
+                 partition=-1, goff=0, soff=0, poff=0, inplace=False, master=None, norm=False, G=None):
         self.padded, self.world, self.gdtype, self.pdtype = padded, world, gdtype, pdtype
         self.partition, self.scale, self.inplace = partition, scale, inplace
         self.P = padded // world
         n = padded if partition < 0 else self.P
         self.n = n
         self.begin = 0 if partition < 0 else partition * self.P
-        self.G = [workloads.grads(padded, 10_000 * seed + k, 1e-3, scale, gdtype) for k in range(world)]
+        # G: the same draws handed over by a caller that runs several cases on them
+        self.G = G if G is not None else [workloads.grads(padded, 10_000 * seed + k, 1e-3, scale, gdtype)
+                                          for k in range(world)]
         m0 = workloads.master(n, 10_000 * seed + 999) if master is None else master
         self.host = oracle.initial_state(m0, pdtype)
         rng = np.random.Generator(np.random.PCG64(seed + 5))

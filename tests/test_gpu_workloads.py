@@ -10,11 +10,11 @@ benchmark times (every rank's partition in one launch per bucket).
   NaN injected at 17 positions at steps 2 and 4: full arrays against the
   oracle, flag bit-exact, skipped steps leave every state bit-identical,
   scale 65536 -> 32768 -> 16384.
-- Stage 3 layer-wise path on the 6.7B GPT shape, N = 8, fp16 and bf16: per
-  unit an all-gather of the unit's parameters from 8 rank-major shards into a
-  reused layer buffer, then one fused call per rank writing its updated
-  parameters into its own shard; windows against the oracle, whole gathered
-  units bit-exact.
+- Stage 3 layer-wise path on the 6.7B GPT shape, N = 8, fp16 and bf16, three
+  steps: per unit and step an all-gather of the unit's parameters from 8
+  rank-major shards into a reused layer buffer, then one fused call per rank
+  writing its updated parameters into its own shard, moments carried between
+  steps; windows against the oracle, whole gathered units bit-exact.
 - Flat bandwidth-sweep points: windows.
 - The staged route on a bucket past 2^31 elements (64-bit indexing) and on a
   bf16 N = 16 point: windows of the reduced gradients, states, parameters.
@@ -26,55 +26,13 @@ import torch
 import oracle
 import workloads
 import zero_sharded_optimizer_reduce_b200 as Z
-from _gpu import assert_f32_close, assert_u16_close, host_f32, host_u16
+from _gpu import (assert_f32_close, assert_u16_close, device_grads as _device_grads,
+                  device_master as _device_master, free_gb as _free_gb, host_f32, host_u16,
+                  windows as _windows)
 
 pytestmark = pytest.mark.gpu
 
 TD = {oracle.F16: torch.float16, oracle.BF16: torch.bfloat16}
-
-
-def _free_gb():
-    torch.cuda.empty_cache()          # blocks cached by earlier tests count as free
-    free, _ = torch.cuda.mem_get_info()
-    return free / 1e9
-
-
-def _device_grads(buf, seed, std, scale):
-    gen = torch.Generator(device="cuda")
-    gen.manual_seed(seed)
-    n = buf.numel()
-    chunk = 1 << 27
-    for o in range(0, n, chunk):
-        e = min(n, o + chunk)
-        buf[o:e].copy_(torch.randn(e - o, generator=gen, device="cuda").mul_(std * scale))
-
-
-def _device_master(buf, seed, std=0.02):
-    gen = torch.Generator(device="cuda")
-    gen.manual_seed(seed)
-    n = buf.numel()
-    for o in range(0, n, 1 << 27):
-        e = min(n, o + (1 << 27))
-        buf[o:e].copy_(torch.randn(e - o, generator=gen, device="cuda").mul_(std))
-
-
-def _windows(padded, world, n_random=64, width=65_536, seed=0):
-    """Sorted, disjoint [lo, hi) windows: random, partition boundaries, ends."""
-    rng = np.random.Generator(np.random.PCG64(seed))
-    P = padded // world
-    spans = [(0, 4096), (padded - 4096, padded)]
-    for r in range(1, world):
-        spans.append((r * P - 4, r * P + 4))
-    for lo in rng.integers(0, max(1, padded - width), n_random):
-        spans.append((int(lo), int(lo) + width))
-    spans = sorted((max(0, a), min(padded, b)) for a, b in spans)
-    merged = []
-    for a, b in spans:
-        if merged and a <= merged[-1][1]:
-            merged[-1] = (merged[-1][0], max(merged[-1][1], b))
-        else:
-            merged.append((a, b))
-    return merged
 
 
 def _u16(t):
@@ -182,31 +140,54 @@ def test_overflow_workload_full_arrays(mode):
 
 @pytest.mark.parametrize("dtype", [oracle.F16, oracle.BF16])
 def test_stage3_layerwise_6p7b(dtype):
-    """Stage 3 on the 6.7B GPT shape: per unit, gather then fused update per rank.
+    """Stage 3 on the 6.7B GPT shape, three steps (t = 1, 2, 3).
 
-    Runs every unit when the GPU has room for the whole fp32 state (~80 GB);
-    otherwise the first, a middle and the last unit.
+    Per unit and step: the all-gather of the unit's parameters from the 8
+    rank-major shards into the reused layer buffer (after step 1 these are the
+    parameters the previous step wrote into the shards, so the gather is
+    checked against the oracle's parameters of that step), fresh seeded
+    gradients, then one fused call per rank reading the unit's fp32 state and
+    writing the rotating spare bank and rank r's shard; the banks swap, so m
+    and v carry over and steps 2 and 3 read non-zero moments with t > 1 bias
+    corrections.  Units are independent (no overflow, the same t for every
+    unit), so each unit runs its three steps before the next unit starts.
+
+    Runs every unit when the GPU has room for the whole shard set plus one
+    unit's buffers; otherwise the first, a middle and the last unit.
     """
     w = workloads.gpt_6p7b_layerwise()
     units = list(w.numels)
     N = w.world
+    steps = 3
     lay = Z.zero_partition_layout(units, N, 1)
     parts = [lay.part(u) for u in range(len(units))]
     shard_off = np.concatenate([[0], np.cumsum(parts)]).astype(np.int64)
-    need_gb = sum(lay.bucket_padded) * 14 / 1e9 + 6
-    run_units = list(range(len(units))) if _free_gb() > need_gb + 10 else [0, 16, len(units) - 1]
+    max_pad = max(lay.bucket_padded)
+    need_gb = (sum(lay.bucket_padded) * 2 + max_pad * (2 * N + 2 + 24)) / 1e9 + 6
+    run_units = list(range(len(units))) if _free_gb() > need_gb else [0, 16, len(units) - 1]
     tdt = TD[dtype]
     shards = [torch.empty(int(shard_off[-1]), dtype=tdt, device="cuda") for _ in range(N)]
-    max_pad = max(lay.bucket_padded)
     layer_buf = torch.empty(max_pad, dtype=tdt, device="cuda")
     grads = [torch.empty(max_pad, dtype=tdt, device="cuda") for _ in range(N)]
-    st = {nm: torch.empty(max_pad, dtype=torch.float32, device="cuda") for nm in ("p", "m", "v")}
-    spare = {nm: torch.empty(max_pad, dtype=torch.float32, device="cuda") for nm in ("p", "m", "v")}
+    bank = [{nm: torch.empty(max_pad, dtype=torch.float32, device="cuda") for nm in ("p", "m", "v")}
+            for _ in range(2)]
     flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
     adam = w.adam
-    hp = Z.hparams(adam.lr, adam.beta1, adam.beta2, adam.eps, adam.weight_decay, 1)
+
+    def unit_params(u, lo, hi):
+        # parameters live in the shards: element i of the unit is shard i // P, slot i % P
+        P = parts[u]
+        pieces = []
+        for r in range(lo // P, (hi - 1) // P + 1):
+            a = max(lo, r * P) - r * P
+            b = min(hi, (r + 1) * P) - r * P
+            pieces.append(_u16(shards[r][shard_off[u] + a:shard_off[u] + b]))
+        return np.concatenate(pieces)
+
     for u in run_units:
         pad, P = lay.bucket_padded[u], parts[u]
+        st, spare = bank[0], bank[1]
         # unit u's fp32 state (flat, rank-major) and its parameter slices in the shards
         _device_master(st["p"][:pad], 1200 + u)
         st["p"][lay.bucket_numel[u]:pad].zero_()
@@ -214,43 +195,47 @@ def test_stage3_layerwise_6p7b(dtype):
         st["v"][:pad].zero_()
         for r in range(N):
             shards[r][shard_off[u]:shard_off[u] + P].copy_(st["p"][r * P:(r + 1) * P])
-        # forward/backward reconstruct: all-gather the unit into the layer buffer
-        Z.zero_allgather_params(shards, int(shard_off[u]), P, layer_buf[:pad])
-        torch.cuda.synchronize()
-        if u in (0, len(units) - 1):
-            ref_full = oracle.allgather([_u16(s[shard_off[u]:shard_off[u] + P]) for s in shards], 0, P)
-            assert np.array_equal(_u16(layer_buf[:pad]), ref_full)
-        p0 = host_f32(st["p"][:pad]).copy()
-        for k in range(N):
-            _device_grads(grads[k][:pad], workloads.seed_for(w.seed, 1, k) + 17 * u, w.grad_std, w.loss_scale)
-            grads[k][lay.bucket_numel[u]:pad].zero_()
-        flag.zero_()
-        # one fused call per rank: reduce-scatter slice r, update, write rank r's shard
-        for r in range(N):
-            sl = slice(r * P, (r + 1) * P)
-            Z.zero_reduce_scatter_adam_step([g[:pad] for g in grads], pad, r,
-                                            st["p"][sl], st["m"][sl], st["v"][sl],
-                                            spare["p"][sl], spare["m"][sl], spare["v"][sl],
-                                            shards[r][shard_off[u]:shard_off[u] + P], hp, w.loss_scale, flag)
-        torch.cuda.synchronize()
-        assert int(flag.item()) == 0
         wins = _windows(pad, N, n_random=8, seed=u)
-        for lo, hi in wins:
-            G = [_u16(g[lo:hi]) for g in grads]
-            ref = oracle.initial_state(p0[lo:hi].copy(), dtype)
-            ovf, _ = oracle.flat_step(G, ref, adam, 1, w.loss_scale, float(N), dtype, dtype)
-            assert ovf == 0
-            assert assert_f32_close(host_f32(spare["p"][lo:hi]), ref.master, "master") == 0
-            assert assert_f32_close(host_f32(spare["m"][lo:hi]), ref.m, "m") == 0
-            assert assert_f32_close(host_f32(spare["v"][lo:hi]), ref.v, "v") == 0
-            # parameters live in the shards: element i of the unit is shard i // P, slot i % P
-            pieces = []
-            for r in range(lo // P, (hi - 1) // P + 1):
-                a = max(lo, r * P) - r * P
-                b = min(hi, (r + 1) * P) - r * P
-                pieces.append(_u16(shards[r][shard_off[u] + a:shard_off[u] + b]))
-            got = np.concatenate(pieces)
-            assert assert_u16_close(got, ref.params, "params") == 0
+        p0 = [host_f32(st["p"][lo:hi]).copy() for lo, hi in wins]
+        refs = [oracle.initial_state(x, dtype) for x in p0]
+        for t in range(1, steps + 1):
+            # forward/backward reconstruct: all-gather the unit into the layer buffer
+            Z.zero_allgather_params(shards, int(shard_off[u]), P, layer_buf[:pad], status=status)
+            torch.cuda.synchronize()
+            assert int(status.item()) == 0
+            if u in (0, len(units) - 1) and t == 1:
+                ref_full = oracle.allgather([_u16(s[shard_off[u]:shard_off[u] + P]) for s in shards], 0, P)
+                assert np.array_equal(_u16(layer_buf[:pad]), ref_full)
+            for (lo, hi), ref in zip(wins, refs):
+                # the gathered layer holds the previous step's parameters (at t = 1
+                # the initial ones, written into the shards above)
+                assert np.array_equal(_u16(layer_buf[lo:hi]), unit_params(u, lo, hi))
+                if t > 1:
+                    assert assert_u16_close(_u16(layer_buf[lo:hi]), ref.params, "gathered params") == 0
+            for k in range(N):
+                _device_grads(grads[k][:pad], workloads.seed_for(w.seed, t, k) + 17 * u, w.grad_std, w.loss_scale)
+                grads[k][lay.bucket_numel[u]:pad].zero_()
+            flag.zero_()
+            hp = Z.hparams(adam.lr, adam.beta1, adam.beta2, adam.eps, adam.weight_decay, t)
+            # one fused call per rank: reduce-scatter slice r, update, write rank r's shard
+            for r in range(N):
+                sl = slice(r * P, (r + 1) * P)
+                Z.zero_reduce_scatter_adam_step([g[:pad] for g in grads], pad, r,
+                                                st["p"][sl], st["m"][sl], st["v"][sl],
+                                                spare["p"][sl], spare["m"][sl], spare["v"][sl],
+                                                shards[r][shard_off[u]:shard_off[u] + P], hp, w.loss_scale, flag)
+            torch.cuda.synchronize()
+            assert int(flag.item()) == 0
+            for (lo, hi), ref in zip(wins, refs):
+                G = [_u16(g[lo:hi]) for g in grads]
+                ovf, _ = oracle.flat_step(G, ref, adam, t, w.loss_scale, float(N), dtype, dtype)
+                assert ovf == 0
+                what = f"unit {u} t={t}"
+                assert assert_f32_close(host_f32(spare["p"][lo:hi]), ref.master, what + " master") == 0
+                assert assert_f32_close(host_f32(spare["m"][lo:hi]), ref.m, what + " m") == 0
+                assert assert_f32_close(host_f32(spare["v"][lo:hi]), ref.v, what + " v") == 0
+                assert assert_u16_close(unit_params(u, lo, hi), ref.params, what + " params") == 0
+            st, spare = spare, st
 
 
 @pytest.mark.parametrize("psi,world,dtype", [(1 << 20, 64, oracle.F16), (16 << 20, 16, oracle.BF16),
