@@ -36,6 +36,8 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+import numpy as np  # noqa: E402
+
 import workloads  # noqa: E402
 
 METRIC = "fused ZeRO step: Gparams/s and achieved HBM GB/s vs B200 peak (1 GPU)"
@@ -173,36 +175,72 @@ def profiled_traffic(elems_per_launch: float, kernel: str = "fused"):
 
 # --------------------------------------------------------------- CPU side
 
-def cpu_baseline(w: workloads.Workload, sample_elems: int, min_seconds: float = 10.0, max_seconds: float = 30.0):
-    """The oracle on this host's cores on a contiguous slice of bucket 0
-    (OpenMP over every core), plus the same slice on one thread."""
+def _oracle_rate(G, master, adam, loss_scale, divisor, min_seconds, max_steps=None):
+    """Elements per second of the oracle's flat step (reduce-scatter, overflow
+    test, Adam) over the given replicas: whole steps until min_seconds have
+    passed (at least one).  Returns (Gparams/s, steps, seconds)."""
     import oracle
+    n = G[0].size
+    st = oracle.initial_state(master)
+    done, t0, t = 0, time.perf_counter(), 0
+    while True:
+        t += 1
+        oracle.flat_step(G, st, adam, t, loss_scale, divisor)
+        done += n
+        el = time.perf_counter() - t0
+        if el >= min_seconds or (max_steps is not None and t >= max_steps):
+            return done / el / 1e9, t, el
+
+
+def cpu_baseline(w: workloads.Workload, sample_elems: int, min_seconds: float = 8.0):
+    """The oracle on this host's cores (OpenMP over every core, and one
+    thread): on a contiguous slice of the benchmark workload (its unit), plus
+    the full arrays of the tiny and the dynamic-loss-scale workloads."""
+    import oracle
+    cores = oracle.threads()
+
+    def both(G, master, loss_scale, divisor, adam, secs, single_steps=1):
+        v, steps, el = _oracle_rate(G, master, adam, loss_scale, divisor, secs)
+        oracle.set_threads(1)
+        try:
+            v1, steps1, el1 = _oracle_rate(G, master, adam, loss_scale, divisor, float("inf"),
+                                              max_steps=single_steps)
+        finally:
+            oracle.set_threads(cores)
+        return {"value": v, "single_thread_value": v1, "steps": steps, "seconds": el,
+                "single_thread_steps": steps1, "single_thread_seconds": el1}
+
     N = w.world
     G = [workloads.grads(sample_elems, workloads.seed_for(w.seed, 1, k), w.grad_std, w.loss_scale)
          for k in range(N)]
-
-    def timed(seconds):
-        st = oracle.initial_state(workloads.master(sample_elems, 7 * w.seed))
-        done, t0, t = 0, time.perf_counter(), 0
-        while True:
-            t += 1
-            oracle.flat_step(G, st, w.adam, t, w.loss_scale, float(N))
-            done += sample_elems
-            el = time.perf_counter() - t0
-            if el >= seconds or el >= max_seconds:
-                return done / el / 1e9, t, el
-
-    cores = oracle.threads()
-    value, steps, el = timed(min_seconds)
-    oracle.set_threads(1)
-    try:
-        single, _, _ = timed(min(5.0, min_seconds))
-    finally:
-        oracle.set_threads(cores)
-    return {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "single_thread_value": single,
-            "sample": f"{steps} oracle steps (reduce-scatter, overflow test, AdamW) over a {sample_elems:,}-element "
-                      f"slice of bucket 0 with N={N} replicas, {el:.1f} s on {cores} threads; "
-                      f"single_thread_value: the same slice on 1 thread"}
+    head = both(G, workloads.master(sample_elems, 7 * w.seed), w.loss_scale, float(N), w.adam, min_seconds)
+    del G
+    configs = {}
+    tiny = workloads.tiny_flat()
+    padded = -(-tiny.numels[0] // tiny.world) * tiny.world
+    G = [workloads.grads(padded, workloads.seed_for(tiny.seed, 1, k), tiny.grad_std, tiny.loss_scale)
+         for k in range(tiny.world)]
+    r = both(G, workloads.master(padded, 7 * tiny.seed), tiny.loss_scale, float(tiny.world), tiny.adam, 2.0,
+             single_steps=3)
+    configs[tiny.name] = dict(r, elements=padded, world=tiny.world, sample="full arrays")
+    ovf = workloads.overflow_flat()
+    psi = ovf.numels[0]
+    # two seeded draws; the other replicas are seeded rotations of them (the
+    # same distribution; the oracle's time does not depend on the values)
+    base = [workloads.grads(psi, workloads.seed_for(ovf.seed, 1, k), ovf.grad_std, ovf.loss_scale) for k in range(2)]
+    G = [np.roll(base[k % 2], 7919 * k) for k in range(ovf.world)]
+    r = both(G, workloads.master(psi, 7 * ovf.seed), ovf.loss_scale, float(ovf.world), ovf.adam, 2.0)
+    configs[ovf.name] = dict(r, elements=psi, world=ovf.world,
+                             sample="full arrays (replicas 2-15 are seeded rotations of two draws)")
+    del G, base
+    return {"value": head["value"], "unit": UNIT, "cores": cores, "kind": "oracle",
+            "single_thread_value": head["single_thread_value"],
+            "sample": f"{head['steps']} oracle steps (reduce-scatter, overflow test, AdamW) over a "
+                      f"{sample_elems:,}-element contiguous slice of bucket 0 of {w.name} with N={N} replicas, "
+                      f"{head['seconds']:.1f} s on {cores} threads; single_thread_value: "
+                      f"{head['single_thread_steps']} step(s) of the same slice on 1 thread; configs: the full "
+                      f"arrays of the tiny and the dynamic-loss-scale workloads, same protocol",
+            "configs": configs}
 
 
 def run_reference(args):
@@ -345,13 +383,20 @@ def run_gpu(args):
     torch.cuda.profiler.start()      # ncu --profile-from-start off captures only the timed steps
     t_start.record(stream)
     applied = 0
-    for _ in range(args.steps):
+    step_ev = [t_start]              # an event at every step boundary: per-step device times
+    for i in range(args.steps):
         applied += bool(opt.step(on_launch=on_launch))
+        if i + 1 < args.steps:
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            step_ev.append(e)
     t_end.record(stream)
+    step_ev.append(t_end)
     barrier()
     torch.cuda.profiler.stop()
     clock = clocks.stop()
     ms = t_start.elapsed_time(t_end)
+    step_ms = [a.elapsed_time(b) for a, b in zip(step_ev[:-1], step_ev[1:])]
     # per-launch durations of the fused kernel
     launch_ms, launch_elems = [], []
     for b, es in ev.items():
@@ -362,6 +407,7 @@ def run_gpu(args):
             launch_elems.append(psi_p if b < 0 else L.bucket_padded[b])
     ms = max_over_ranks(ms, "cuda")
     ms_per_step = ms / args.steps
+    ms_median = max_over_ranks(statistics.median(step_ms), "cuda")
     value = whole_job_gparams(psi_p, world_gpus, ms_per_step)
     bpe = step_bytes_per_elem(w.world, args.mode, args.max_grad_norm is not None)
     # the runner's whole step (b = -1) is timed as one unit: every byte of the step
@@ -389,6 +435,9 @@ def run_gpu(args):
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world_gpus, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+                "ms_per_step_median": ms_median,
+                "ms_per_step_min_max": [min(step_ms), max(step_ms)],
+                "value_from_median": whole_job_gparams(psi_p, world_gpus, ms_median),
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic (seeded N(0,1e-3)x65536 fp16 gradients, N(0,0.02) fp32 master)",
                 "config": {"workload": w.name, "psi": sum(w.numels), "psi_padded": psi_p, "world": w.world,
@@ -432,7 +481,8 @@ def run_sweep(args):
     step is timed on its own with CUDA events, the median of at least 20
     steps (at least --steps when a step moves more than 20 GB); when a
     point's footprint is below 4x L2 an L2-sized buffer is written between
-    steps (untimed)."""
+    steps (untimed).  A short sleep kernel is queued before each timed step
+    so that the host's launch latency falls outside the events."""
     import torch
     import zero_sharded_optimizer_reduce_b200 as Z
     torch.cuda.set_device(0)
@@ -463,6 +513,9 @@ def run_sweep(args):
             for _ in range(reps):
                 if small:
                     flush.fill_(1)
+                # keep the device busy (untimed) while the host enqueues the
+                # step, so that the events bracket device time, not launch latency
+                torch.cuda._sleep(200_000)
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
                 ms_launch = []
@@ -557,6 +610,166 @@ def run_stage3(args):
     return 0
 
 
+def p2p_bytes_per_rank(parts, world: int, grad_esize: int, param_esize: int, mode: str) -> dict:
+    """Bytes one rank moves between GPUs per step of the one-process-per-GPU
+    routes, from its partition (or unit slice) sizes `parts`:
+
+    - ZeRO-2 (mode "banks" / "staged"): the reduce-scatter reads slice r of
+      every peer's gradient buffer, (N - 1) P gradient elements per bucket;
+      the all-gather moves every peer's slot of P parameters, (N - 1) P
+      elements (the banks mode reads the peers' slots, the staged update
+      stores its own slot into every peer's buffer).  Together 2 (N - 1) P
+      elements, which sums to 2 Psi (N - 1) / N per rank: the pages' "2 Psi
+      per GPU" of data parallelism (ZeRO explainer, communication-volume
+      paragraphs).
+    - Stage 3 (mode "stage3"): two gathers of every unit (forward and
+      backward) plus its reduce-scatter: 3 (N - 1) P elements, 1.5 x the
+      above.
+    """
+    peers = world - 1
+    pull = sum(peers * P * grad_esize for P in parts)
+    gather = sum(peers * P * param_esize for P in parts) * (2 if mode == "stage3" else 1)
+    elems = sum(peers * P for P in parts) * (3 if mode == "stage3" else 2)
+    kind = {"banks": "peer reads after the commit", "staged": "the update's own stores into every peer's buffer",
+            "stage3": "peer reads, forward and backward"}[mode]
+    return {"pull_bytes": pull, "gather_bytes": gather, "gather_kind": kind, "elements_moved": elems}
+
+
+def run_distributed(args):
+    """The ZeRO-2 step (or, with --stage3, the layer-wise ZeRO-3 step) with one
+    process per GPU: each process is one data-parallel rank of the real
+    method, holding its own replica's gradients, its 1/N of the fp32 states
+    and (ZeRO-2) the full parameter buckets or (ZeRO-3) its parameter shard;
+    the reduce-scatter pulls the peers' gradient slices through CUDA IPC
+    mappings inside the kernel, the all-gather moves the updated slots.
+    World size = number of processes (the data-parallel degree).  Each step
+    is timed with CUDA events on every rank; the slowest rank's time is
+    reported.  Host barriers order the ranks (no kernel waits on another
+    rank), so several ranks may share one GPU for a functional run
+    (--dist-backend gloo)."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    import zero_sharded_optimizer_reduce_b200 as Z
+
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ.setdefault("MASTER_PORT", "29531")
+    os.environ.setdefault("RANK", "0")
+    os.environ.setdefault("WORLD_SIZE", "1")
+    world = int(os.environ["WORLD_SIZE"])
+    rank = int(os.environ["RANK"])
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local % torch.cuda.device_count())
+    torch.cuda.set_device(dev)
+    kw = {"device_id": dev} if args.dist_backend == "nccl" else {}
+    dist.init_process_group(args.dist_backend, timeout=datetime.timedelta(seconds=300), **kw)
+    red_dev = "cuda" if args.dist_backend == "nccl" else "cpu"
+    gdt = torch.bfloat16 if args.grad_dtype == "bf16" else torch.float16
+    chunk = 1 << 27
+
+    def randn_into(buf, seed, std):
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed)
+        for o in range(0, buf.numel(), chunk):
+            e = min(buf.numel(), o + chunk)
+            buf[o:e].copy_(torch.randn(e - o, generator=g, device=dev).mul_(std))
+
+    if args.stage3:
+        w = workloads.gpt_6p7b_layerwise()
+        if args.flat:       # a small stand-in shape: 4 units of --flat elements
+            w = workloads.Workload(f"flat_4x{args.flat}_layerwise", (args.flat,) * 4, w.world, w.loss_scale, 1,
+                                   w.adam, seed=w.seed)
+        opt = Z.DistributedZeroStage3(w.numels, lr=w.adam.lr, betas=(w.adam.beta1, w.adam.beta2), eps=w.adam.eps,
+                                      weight_decay=w.adam.weight_decay, loss_scale=w.loss_scale, grad_dtype=gdt,
+                                      param_dtype=gdt)
+        L = opt.layout
+        masters = []
+        for u in range(opt.U):
+            m = torch.empty(L.bucket_padded[u], dtype=torch.float32, device=dev)
+            randn_into(m, 4000 + u, w.master_std)
+            m[L.bucket_numel[u]:].zero_()
+            masters.append(m)
+        opt.load(masters)
+        del masters
+        # this rank's replica gradients: one seeded buffer the size of the
+        # largest unit; each unit's backward copies its prefix in (the copy
+        # stands in for the backward pass writing the unit's gradients)
+        src = torch.empty(max(L.bucket_padded), dtype=gdt, device=dev)
+        randn_into(src, workloads.seed_for(w.seed + 100, 1, rank), w.grad_std * w.loss_scale)
+
+        def grad_fill(u, buf):
+            buf.copy_(src[:buf.numel()])
+            buf[L.bucket_numel[u]:].zero_()
+
+        step = lambda: opt.step(grad_fill)
+        parts = opt.parts
+        mode = "stage3"
+        metric = "ZeRO-3 layer-wise step, one process per GPU: Gparams/s"
+    else:
+        w = select_workload(args)
+        opt = Z.DistributedZeroAdam(w.numels, w.bucket_elems, 8, lr=w.adam.lr, betas=(w.adam.beta1, w.adam.beta2),
+                                    eps=w.adam.eps, weight_decay=w.adam.weight_decay, loss_scale=w.loss_scale,
+                                    grad_dtype=gdt, param_dtype=gdt, mode=args.distributed)
+        L = opt.layout
+        masters, params = [], []
+        for b in range(L.n_buckets):
+            randn_into(opt.grads[b], workloads.seed_for(w.seed + 100, 1, rank) + 7919 * b, w.grad_std * w.loss_scale)
+            opt.grads[b][L.bucket_numel[b]:].zero_()
+            m = torch.empty(L.bucket_padded[b], dtype=torch.float32, device=dev)
+            randn_into(m, 7 * w.seed + b, w.master_std)        # the same on every rank
+            m[L.bucket_numel[b]:].zero_()
+            masters.append(m)
+            params.append(m.to(gdt))
+        opt.load(masters, params)
+        del masters, params
+        step = opt.step
+        parts = [L.part(b) for b in range(L.n_buckets)]
+        mode = args.distributed
+        metric = "ZeRO-2 step, one process per GPU (P2P reduce-scatter + update + all-gather): Gparams/s"
+    psi_p = sum(L.bucket_padded)
+    torch.cuda.synchronize()
+
+    def barrier():
+        torch.cuda.synchronize()
+        dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    stream = torch.cuda.current_stream()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    applied = 0
+    evs[0].record(stream)
+    for i in range(args.steps):
+        applied += bool(step())
+        evs[i + 1].record(stream)
+    barrier()
+    step_ms = [a.elapsed_time(b) for a, b in zip(evs[:-1], evs[1:])]
+    ms = max_over_ranks(sum(step_ms) / args.steps, red_dev)
+    ms_median = max_over_ranks(statistics.median(step_ms), red_dev)
+    esize = torch.empty((), dtype=gdt).element_size()
+    moved = p2p_bytes_per_rank(parts, world, esize, esize, mode)
+    per_rank_gbs = (moved["pull_bytes"] + moved["gather_bytes"]) / (ms * 1e-3) / 1e9
+    if rank == 0:
+        line = {"metric": metric, "value": psi_p / (ms * 1e-3) / 1e9, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "ms_per_step_median": ms_median,
+                "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic (seeded, per-rank gradients)",
+                "config": {"workload": w.name, "psi_padded": psi_p, "world": world, "mode": f"distributed-{mode}",
+                           "units_or_buckets": L.n_buckets, "backend": args.dist_backend,
+                           "gpus_visible": torch.cuda.device_count(),
+                           "parallelism": f"dp{world}: one process per rank, P2P through CUDA IPC"},
+                "p2p": dict(moved, per_rank_gbs=per_rank_gbs,
+                            note="bytes each rank moves between GPUs per step; GB/s over the whole step time "
+                                 "(host barriers and the local HBM passes included)"),
+                "applied_steps": applied}
+        print(json.dumps(line), flush=True)
+    opt.close()
+    del opt
+    dist.destroy_process_group()
+    return 0
+
+
 def run_e2e(opt, args, stream, barrier, world_gpus):
     """Same step through ZeroAdam.step_from_host: every step copies the N
     replicas' gradients from pinned host memory and reads the flag back."""
@@ -601,11 +814,11 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--cpu-sample", type=int, default=1 << 23)
-    ap.add_argument("--ref-sample", type=int, default=1 << 23)
+    ap.add_argument("--cpu-sample", type=int, default=1 << 26)
+    ap.add_argument("--ref-sample", type=int, default=1 << 26)
     ap.add_argument("--flat", type=int, default=0, help="flat workload of this many elements instead of GPT-2")
     ap.add_argument("--world", type=int, default=8, help="simulated replicas of the flat workload")
     ap.add_argument("--grad-dtype", choices=["f16", "bf16"], default="f16")
@@ -616,6 +829,11 @@ def main(argv=None):
                          "staged: one bank, reduce-scatter to fp32 + gated update")
     ap.add_argument("--max-grad-norm", type=float, default=None, help="clip gradients to this global norm")
     ap.add_argument("--sweep-dtype-only", action="store_true", help="sweep only --grad-dtype")
+    ap.add_argument("--distributed", choices=["banks", "staged"], default=None,
+                    help="one process per GPU (under torchrun): the multi-process ZeRO-2 route in this mode; "
+                         "with --stage3 the multi-process layer-wise ZeRO-3 route")
+    ap.add_argument("--dist-backend", choices=["nccl", "gloo"], default="nccl",
+                    help="process-group backend of the --distributed host barriers (gloo lets ranks share a GPU)")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -623,6 +841,8 @@ def main(argv=None):
         return run_reference(args)
     if args.sweep:
         return run_sweep(args)
+    if args.distributed is not None:
+        return run_distributed(args)
     if args.stage3:
         return run_stage3(args)
     return run_gpu(args)

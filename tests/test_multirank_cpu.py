@@ -144,3 +144,34 @@ def test_bench_traffic_records_scale_with_elements():
         per = a / 1e6
         bound = {"fused": 42, "staged": 30, "staged_step": 50}[kind]
         assert 0.9 * bound <= per <= 1.05 * bound
+
+
+def test_p2p_byte_model_matches_the_pages_volumes():
+    """Bytes one rank moves between GPUs per step of the one-process-per-GPU
+    routes (bench.p2p_bytes_per_rank), against the pages' communication
+    volumes (ZeRO explainer, communication-volume paragraphs): Stage 1/2 move
+    2 Psi (N - 1) / N elements per rank (reduce-scatter + all-gather, the same
+    as data parallelism's all-reduce), Stage 3 moves 1.5 x that."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import oracle
+    import workloads
+    for numels, world, cap in [(workloads.gpt2_1p5b_tensor_numels(), 8, 500_000_000), ([1_000_003], 4, 0),
+                               ([100_000_000], 16, 0), ([7, 5000, 123], 3, 4000)]:
+        L = oracle.partition_layout(numels, world, cap)
+        parts = [L.bucket_padded[b] // world for b in range(L.n_buckets)]
+        psi_p = sum(L.bucket_padded)
+        for mode in ("banks", "staged"):
+            m = bench.p2p_bytes_per_rank(parts, world, 2, 2, mode)
+            assert m["elements_moved"] == 2 * (world - 1) * psi_p // world
+            assert m["pull_bytes"] == m["gather_bytes"] == 2 * (world - 1) * psi_p // world
+            # the oracle's own ring count for the same layout
+            assert m["elements_moved"] == oracle.comm_elements(2, L)
+        s3 = bench.p2p_bytes_per_rank(parts, world, 2, 2, "stage3")
+        assert s3["elements_moved"] == 3 * (world - 1) * psi_p // world == oracle.comm_elements(3, L)
+        assert s3["gather_bytes"] == 2 * s3["pull_bytes"]
+        assert s3["elements_moved"] * 2 == 3 * bench.p2p_bytes_per_rank(parts, world, 2, 2, "banks")["elements_moved"]
+    # fp32 gradients, bf16 parameters: bytes follow the element sizes
+    m = bench.p2p_bytes_per_rank([10], 3, 4, 2, "banks")
+    assert (m["pull_bytes"], m["gather_bytes"]) == (80, 40)
+    assert bench.p2p_bytes_per_rank([10], 1, 2, 2, "staged")["elements_moved"] == 0
