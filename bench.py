@@ -153,9 +153,10 @@ def source_digest(files=("fused_step.cuh",)) -> str:
 
 
 # timed kernel -> (committed ncu traffic record, the sources it was taken on)
-TRAFFIC_RECORDS = {"fused": ("fused_step_traffic.json", ("fused_step.cuh",)),
-                   "staged": ("adam_reduced_traffic.json", ("fused_step.cuh", "staged.cuh")),
-                   "staged_step": ("staged_step_traffic.json", ("fused_step.cuh", "grad_stats.cuh", "staged.cuh"))}
+TRAFFIC_RECORDS = {"fused": ("fused_step_traffic.json", ("bulk.cuh", "fused_step.cuh")),
+                   "staged": ("adam_reduced_traffic.json", ("bulk.cuh", "fused_step.cuh", "staged.cuh")),
+                   "staged_step": ("staged_step_traffic.json",
+                                   ("bulk.cuh", "fused_step.cuh", "grad_stats.cuh", "staged.cuh"))}
 
 
 def profiled_traffic(elems_per_launch: float, kernel: str = "fused"):
@@ -481,8 +482,10 @@ def run_sweep(args):
     step is timed on its own with CUDA events, the median of at least 20
     steps (at least --steps when a step moves more than 20 GB); when a
     point's footprint is below 4x L2 an L2-sized buffer is written between
-    steps (untimed).  A short sleep kernel is queued before each timed step
-    so that the host's launch latency falls outside the events."""
+    steps (untimed).  Each timed unit is the fused kernel call alone
+    (zero_reduce_scatter_adam_step over the bucket, banks alternating); a
+    short sleep kernel is queued before it so that the host's launch latency
+    falls outside the events."""
     import torch
     import zero_sharded_optimizer_reduce_b200 as Z
     torch.cuda.set_device(0)
@@ -505,28 +508,38 @@ def run_sweep(args):
             fill_workload(opt, w, w.seed)
             bpe = bytes_per_elem(N)
             small = psi * bpe < 4 * 126e6
+            banks = [[opt.master[0][i], opt.m[0][i], opt.v[0][i]] for i in (0, 1)]
+            ncall = [0]
+
+            def call():
+                # the fused kernel call alone, banks alternating (the step's
+                # flag clear and read-back stay outside the timed region)
+                i = ncall[0]
+                ncall[0] += 1
+                hp = Z.hparams(w.adam.lr, w.adam.beta1, w.adam.beta2, w.adam.eps, w.adam.weight_decay, i + 1)
+                Z.zero_reduce_scatter_adam_step(opt.grads[0], psi, Z.ZERO_ALL_PARTITIONS, *banks[i % 2],
+                                                *banks[(i + 1) % 2], opt.params_bank[0][(i + 1) % 2], hp, 65536.0,
+                                                opt.flag)
             for _ in range(3):
-                opt.step()
+                call()
             times = []
-            # median of >= 20 timed steps, >= 5 when a step moves more than 20 GB
+            # median of >= 20 timed calls, >= 5 when a call moves more than 20 GB
             reps = args.steps if psi * bpe > 20e9 else max(20, args.steps)
             for _ in range(reps):
+                opt.flag.zero_()
                 if small:
                     flush.fill_(1)
                 # keep the device busy (untimed) while the host enqueues the
-                # step, so that the events bracket device time, not launch latency
+                # call, so that the events bracket device time, not launch latency
                 torch.cuda._sleep(200_000)
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
-                ms_launch = []
-
-                def on_launch(b, phase, _l=ms_launch):
-                    e = torch.cuda.Event(enable_timing=True)
-                    e.record()
-                    _l.append(e)
-                opt.step(on_launch=on_launch)
+                e0.record()
+                call()
+                e1.record()
                 torch.cuda.synchronize()
-                times.append(ms_launch[0].elapsed_time(ms_launch[1]))
+                times.append(e0.elapsed_time(e1))
+            assert int(opt.flag.item()) == 0
             ms = statistics.median(times)
             gbs = psi * bpe / (ms * 1e-3) / 1e9
             print(json.dumps({"sweep": True, "psi": psi, "world": N, "grad_dtype": dt,
@@ -770,6 +783,66 @@ def run_distributed(args):
     return 0
 
 
+def run_allgather(args):
+    """The all-gather reconstruct alone (zero_allgather_params): --world
+    slices of --allgather elements (fp16 or bf16) gathered into one buffer,
+    the L2 written over between calls (untimed) and a short sleep kernel
+    queued before each, CUDA events around the call, median of at least 20.
+    An odd slice size puts every rank but the first off its destination's
+    16-byte phase (the realigning kernel).  torch.cat of the same slices is
+    timed the same way, for comparison.  4 bytes per element (2 read, 2
+    written).  One JSON line."""
+    import torch
+    import zero_sharded_optimizer_reduce_b200 as Z
+    torch.cuda.set_device(0)
+    N, P = args.world, args.allgather
+    dt = torch.bfloat16 if args.grad_dtype == "bf16" else torch.float16
+    gen = torch.Generator(device="cuda")
+    shards = []
+    for r in range(N):
+        gen.manual_seed(8000 + r)
+        shards.append(torch.randn(P, generator=gen, device="cuda").to(dt))
+    dst = torch.empty(N * P, dtype=dt, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    Z.zero_allgather_params(shards, 0, P, dst, status=status)
+    torch.cuda.synchronize()
+    assert torch.equal(dst.view(torch.int16), torch.cat(shards).view(torch.int16)) and int(status.item()) == 0
+
+    def timed(fn, reps):
+        for _ in range(3):
+            fn()
+        t = []
+        for _ in range(reps):
+            flush.fill_(1)
+            torch.cuda._sleep(200_000)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            t.append(e0.elapsed_time(e1))
+        return statistics.median(t)
+
+    reps = max(20, args.steps)
+    torch.cuda.profiler.start()
+    ms = timed(lambda: Z.zero_allgather_params(shards, 0, P, dst, status=status), reps)
+    torch.cuda.profiler.stop()
+    ms_cat = timed(lambda: torch.cat(shards, out=dst), reps)
+    peak, peak_kind = peaks()
+    gbs = 4.0 * N * P / (ms * 1e-3) / 1e9
+    gbs_cat = 4.0 * N * P / (ms_cat * 1e-3) / 1e9
+    phases = sorted({(2 * r * P) % 16 for r in range(N)})
+    print(json.dumps({"metric": "all-gather reconstruct (zero_allgather_params): achieved HBM GB/s",
+                      "value": gbs, "unit": "GB/s", "ms_median": ms, "reps": reps, "world": N, "part_numel": P,
+                      "dtype": args.grad_dtype, "bytes_per_elem": 4, "frac_measured": gbs / peak, "peak": peak,
+                      "peak_kind": peak_kind, "dst_phases_bytes": phases,
+                      "l2": "512 MB written between calls (untimed)",
+                      "torch_cat": {"ms_median": ms_cat, "gbs": gbs_cat, "frac_measured": gbs_cat / peak}}),
+          flush=True)
+    return 0
+
+
 def run_e2e(opt, args, stream, barrier, world_gpus):
     """Same step through ZeroAdam.step_from_host: every step copies the N
     replicas' gradients from pinned host memory and reads the flag back."""
@@ -829,6 +902,8 @@ def main(argv=None):
                          "staged: one bank, reduce-scatter to fp32 + gated update")
     ap.add_argument("--max-grad-norm", type=float, default=None, help="clip gradients to this global norm")
     ap.add_argument("--sweep-dtype-only", action="store_true", help="sweep only --grad-dtype")
+    ap.add_argument("--allgather", type=int, default=0,
+                    help="time the all-gather of --world slices of this many elements, one JSON line")
     ap.add_argument("--distributed", choices=["banks", "staged"], default=None,
                     help="one process per GPU (under torchrun): the multi-process ZeRO-2 route in this mode; "
                          "with --stage3 the multi-process layer-wise ZeRO-3 route")
@@ -841,6 +916,8 @@ def main(argv=None):
         return run_reference(args)
     if args.sweep:
         return run_sweep(args)
+    if args.allgather:
+        return run_allgather(args)
     if args.distributed is not None:
         return run_distributed(args)
     if args.stage3:

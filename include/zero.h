@@ -396,9 +396,9 @@ int zero_adam_step_reduced_bcast(const float* reduced_grad, int64_t count,
  * allocating routine.  Inputs and outputs are still the caller's.
  *
  * Results equal those of zero_reduce_scatter_adam_step.  Limits:
- *  - the scratch holds 4096 per-block partial sums; the kernel's grid is
- *    SM count x resident blocks (at most 296 on a B200), so every input
- *    size fits, and a call whose grid would exceed 4096 blocks returns
+ *  - the scratch holds 4096 per-block partial sums; the kernels' grids are
+ *    at most 16 blocks per SM (2368 on a B200), so every input size fits,
+ *    and a call whose grid would exceed 4096 blocks returns
  *    ZERO_ERR_RANGE;
  *  - all calls on a device share the scratch: calls that overlap on the GPU
  *    (other streams, other host threads) race on it; each call clears the
@@ -433,8 +433,8 @@ size_t zero_step_static_scratch_bytes(void);
  * each unit's slices in unit order, shard_offset selects one unit.
  *
  * shards       host array of `world` DEVICE pointers (this GPU's memory, or
- *              another GPU's memory mapped into this process: those slices
- *              are read with plain loads)
+ *              another GPU's memory mapped into this process: the copy uses
+ *              plain loads only)
  * world        1..ZERO_MAX_WORLD
  * shard_offset first element of the slice in every shard (>= 0)
  * part_numel   elements per rank (>= 0); any value: slices whose 16-byte
@@ -442,9 +442,9 @@ size_t zero_step_static_scratch_bytes(void);
  *              registers, so odd sizes keep 16-byte loads and stores
  * dtype        ZERO_F16, ZERO_BF16 or ZERO_F32
  * dst          device, world*part_numel elements, must not overlap a shard
- * status       device int32 or NULL, 4-byte aligned: bit 1 (value 2) is OR-ed
- *              into it when a bounded wait of the bulk-copy kernel gave up (the
- *              copy is then incomplete); never cleared by the call
+ * status       device int32 or NULL, 4-byte aligned: the bounds-checking
+ *              debug build ORs 4 into it when an index check fails (the access
+ *              is then skipped); the release build never writes it
  * Reads whole aligned 16-byte blocks that hold at least one byte of a slice,
  * so never a page outside the slices; writes exactly dst's range.
  * Errors: ZERO_ERR_ARG, ZERO_ERR_DTYPE, ZERO_ERR_ALIGN, ZERO_ERR_CUDA.
@@ -469,6 +469,24 @@ int zero_allgather_params(const void* const* shards, int32_t world, int64_t shar
  * Errors: ZERO_ERR_ARG, ZERO_ERR_ALIGN, ZERO_ERR_CUDA.
  */
 int zero_test_wait_timeout(int32_t* status, int64_t limit_ns, zero_stream_t stream);
+
+/*
+ * zero_test_force_step_kernel - choose the fused step's kernel by hand.
+ *
+ * The paper has no counterpart: a test hook of this library.  Every fused
+ * step call (zero_reduce_scatter_adam_step, its gated and no-alloc variants,
+ * the runner) normally picks one of three kernels that compute the same bits:
+ * the shared-memory pipeline kernel for large calls with N >= 3, the
+ * quad-streaming kernel for N <= 2, mid-size calls and peer memory, the
+ * register kernel for N > 20 or arrays off a common 16-byte phase.  This call
+ * makes the process's later calls take `kind` instead wherever that kernel
+ * can run the call (the pipeline kernel needs a common phase, N <= 20, one
+ * whole tile and gradients in this GPU's memory; the quad kernel a common
+ * phase), so that tests reach each kernel at small sizes.
+ * kind  -1 automatic (the default), 0 register, 1 pipeline, 2 quad
+ * Errors: ZERO_ERR_ARG.  Host only, no CUDA call.
+ */
+int zero_test_force_step_kernel(int32_t kind);
 
 /* ------------------------------------------------------------------------ */
 /* Step runner: the whole step over every bucket                             */

@@ -46,18 +46,26 @@ def _pipe_T(world):
     return min(8192, (180 * 1024 // (2 * (2 * world + 12))) // 512 * 512)
 
 
+@pytest.mark.parametrize("kind", [Z.STEP_KERNEL_AUTO, Z.STEP_KERNEL_REGISTER, Z.STEP_KERNEL_PIPE, Z.STEP_KERNEL_QUAD])
 @pytest.mark.parametrize("world,padded,part,offs", [
-    (3, 3 * 50_001, -1, (0, 0, 0)),                                  # register kernel, ragged
+    (3, 3 * 50_001, -1, (0, 0, 0)),                                  # ragged
     (4, 4 * 20_011, -1, (3, 5, 1)),                                  # scalar path (phases differ)
-    (8, 8 * ((2 * SMS * _pipe_T(8) + 4099) // 8), -1, (0, 0, 0)),    # pipeline kernel + tail
-    (4, 4 * (2 * SMS * _pipe_T(4) + 8 * 100 + 4), 1, (0, 0, 0)),     # pipeline, one partition, head
+    (8, 8 * ((2 * SMS * _pipe_T(8) + 4099) // 8), -1, (0, 0, 0)),    # two tiles per SM + tail
+    (4, 4 * (2 * SMS * _pipe_T(4) + 8 * 100 + 4), 1, (0, 0, 0)),     # one partition, head
+    (2, 2 * 1_000_003, -1, (0, 0, 0)),                               # N = 2 (quad kernel), ragged
     (64, 64 * 4099, -1, (0, 0, 0)),                                  # large N (register)
 ])
-def test_fused_step_in_bounds(world, padded, part, offs):
+def test_fused_step_in_bounds(world, padded, part, offs, kind):
+    # every step kernel that can run the case (the hook falls back to the
+    # automatic choice where the forced one cannot)
     c = Case(padded, world, seed=700 + world, partition=part, goff=offs[0], soff=offs[1], poff=offs[2], norm=True,
              scale=65536.0)
     ref, ovf, _ = c.expect(_adam(0.01), t=2)
-    c.run(_adam(0.01), t=2)
+    Z.zero_test_force_step_kernel(kind)
+    try:
+        c.run(_adam(0.01), t=2)
+    finally:
+        Z.zero_test_force_step_kernel(Z.STEP_KERNEL_AUTO)
     assert int(c.flag.item()) == ovf == 0
     assert c.compare(ref) == [0, 0, 0, 0]
 
@@ -94,3 +102,42 @@ def test_broadcast_update_in_bounds():
     ref, _, _ = c.expect(adam, t=1)
     assert c.compare(ref) == [0, 0, 0, 0]
     assert np.array_equal(host_u16(dsts[1].t), ref.params)
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.float32])
+@pytest.mark.parametrize("world,part,src_off,dst_off", [
+    (8, 300_000, 0, 0),          # every slice on its destination's phase
+    (4, 250_001, 0, 0),          # ranks 1-3 realigned (odd partition)
+    (5, 123_457, 3, 1),          # everything off the phase, heads and tails
+    (3, 5, 1, 2),                # slices shorter than one 16-byte block
+])
+def test_allgather_in_bounds(dtype, world, part, src_off, dst_off):
+    """Both copy kernels (phase-matched and realigned) with their element
+    edges, through the debug build: the status word stays 0, every byte of
+    the destination is the oracle's, the guard bytes around it are intact."""
+    import oracle
+    es = torch.empty((), dtype=dtype).element_size()
+    npdt = np.uint16 if es == 2 else np.uint32
+    rng = np.random.Generator(np.random.PCG64(world * part + src_off))
+    host, dev, keep = [], [], []
+    for _ in range(world):
+        h = rng.integers(0, 2 ** (8 * es), src_off + part + 3, dtype=np.uint64).astype(npdt)
+        base = torch.empty(h.size + src_off + 8, dtype=dtype, device="cuda")
+        view = base[src_off:src_off + h.size]
+        view.view(torch.int16 if es == 2 else torch.int32).copy_(
+            torch.from_numpy(h.view(np.int16 if es == 2 else np.int32)))
+        host.append(h)
+        dev.append(view)
+        keep.append(base)
+    dst = Guarded(world * part, dtype, dst_off)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    Z.zero_allgather_params(dev, src_off, part, dst.t, status=status)
+    torch.cuda.synchronize()
+    dst.check()
+    assert int(status.item()) == 0
+    got = dst.t.view(torch.int16 if es == 2 else torch.int32).cpu().numpy().view(npdt)
+    if es == 2:
+        ref = oracle.allgather(host, src_off, part)
+    else:
+        ref = oracle.allgather([h.view(np.uint16) for h in host], 2 * src_off, 2 * part).view(np.uint32)
+    assert np.array_equal(got, ref)

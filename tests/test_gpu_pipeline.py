@@ -1,9 +1,10 @@
 """Parity of the shared-memory pipeline kernel against the oracle.
 
-Calls whose arrays share a 16-byte phase and that give every SM at least two
-tiles run the bulk-copy pipeline kernel; these sizes are chosen above that
-threshold (two stages of at most 180 KB: 6144 elements per tile at N = 1
-down to 1536 at N = 20, on 148 SMs), with ragged tails, a shifted
+Calls whose arrays share a 16-byte phase, with N >= 3 and at least 128 tiles
+per SM, run the bulk-copy pipeline kernel; this module forces it (the test
+hook zero_test_force_step_kernel) at sizes that give every SM a few tiles
+(two stages of at most 180 KB: 6144 elements per tile at N = 1 down to 1536
+at N = 20, on 148 SMs), with ragged tails, a shifted
 common phase (scalar head), single partitions, bf16 and overflow.  Above
 N = 20 the register kernel runs at the same sizes; those cases (N up to 128)
 check that the kernel choice at the boundary keeps parity.
@@ -19,6 +20,19 @@ from test_gpu_step import Case, _adam
 pytestmark = pytest.mark.gpu
 
 SMS = 148
+
+
+@pytest.fixture(scope="module", autouse=True)
+def pipeline_kernel():
+    """These sizes give every SM a few tiles; in normal use such calls take
+    the quad kernel (the pipeline kernel runs calls of 128 tiles per SM and
+    more), so the module forces the pipeline kernel wherever it can run."""
+    import zero_sharded_optimizer_reduce_b200 as Z
+    Z.zero_test_force_step_kernel(Z.STEP_KERNEL_PIPE)
+    try:
+        yield
+    finally:
+        Z.zero_test_force_step_kernel(Z.STEP_KERNEL_AUTO)
 
 
 def _tile(world):

@@ -149,6 +149,8 @@ def load_library(path: str = LIB_PATH):
     L.zero_runner_destroy.restype = None
     L.zero_test_wait_timeout.argtypes = [vp, i64, vp]
     L.zero_test_wait_timeout.restype = ctypes.c_int
+    L.zero_test_force_step_kernel.argtypes = [i32]
+    L.zero_test_force_step_kernel.restype = ctypes.c_int
     L.zero_allgather_params.argtypes = [ctypes.POINTER(vp), i32, i64, i64, ctypes.c_int, vp, vp, vp]
     L.zero_allgather_params.restype = ctypes.c_int
     L.zero_loss_scale_update.argtypes = [ctypes.POINTER(f32), ctypes.POINTER(i32), i32, i32, f32]
@@ -435,7 +437,8 @@ def zero_adam_step_reduced_bcast(reduced_grad, count: int, master_in, m_in, v_in
 
 def zero_allgather_params(shards, shard_offset: int, part_numel: int, dst, stream=None, status=None) -> None:
     """dst[r*part + j] = shards[r][shard_offset + j] (bit-exact copy); `status`
-    (device int32, optional) receives bit 1 if a copy wait timed out."""
+    (device int32, optional) receives 4 from the debug build when an index
+    check fails."""
     import torch
     _check(lib.zero_allgather_params(_devs(shards, shard_offset + part_numel, "shards"), len(shards), shard_offset,
                                      part_numel, _dtype_code(dst), _dev(dst, len(shards) * part_numel, "dst"),
@@ -537,6 +540,16 @@ def zero_test_wait_timeout(status, limit_ns: int, stream=None) -> None:
     """Run the bounded-wait self-test: ORs 2 into status after ~limit_ns."""
     import torch
     _check(lib.zero_test_wait_timeout(_dev(status, 1, "status", torch.int32), int(limit_ns), _stream(stream)))
+
+
+STEP_KERNEL_AUTO, STEP_KERNEL_REGISTER, STEP_KERNEL_PIPE, STEP_KERNEL_QUAD = -1, 0, 1, 2
+
+
+def zero_test_force_step_kernel(kind: int) -> None:
+    """Test hook: make later fused-step calls of this process take `kind`
+    (STEP_KERNEL_*) wherever that kernel can run the call; -1 restores the
+    automatic choice."""
+    _check(lib.zero_test_force_step_kernel(int(kind)))
 
 
 def zero_ipc_export(tensor) -> tuple:

@@ -36,6 +36,10 @@ inline bool overlaps(const void* a, int64_t na, const void* b, int64_t nb) {
     return x < y + static_cast<uintptr_t>(nb) && y < x + static_cast<uintptr_t>(na);
 }
 
+// Step-kernel override of zero_test_force_step_kernel (-1: the automatic
+// choice), shared by every translation unit that prepares a step launch.
+int step_kernel_override();
+
 // True when `p` is device memory of device `dev` (not another GPU's memory
 // mapped into this process, not host memory).  Kernels that stage their
 // inputs with bulk copies take only such sources; other sources go to the

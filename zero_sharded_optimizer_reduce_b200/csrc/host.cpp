@@ -1,5 +1,6 @@
 // Host-only parts of the libzero C ABI: partition layout of constant-size
 // buffers, the dynamic loss-scale rule, and error strings.
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdlib>
@@ -25,6 +26,10 @@ int ok() {
     return ZERO_OK;
 }
 
+static std::atomic<int> g_step_kernel_override{-1};
+
+int step_kernel_override() { return g_step_kernel_override.load(std::memory_order_relaxed); }
+
 }  // namespace zero
 
 using zero::fail;
@@ -32,6 +37,12 @@ using zero::fail;
 extern "C" {
 
 const char* zero_last_error(void) { return zero::g_last_error; }
+
+int zero_test_force_step_kernel(int32_t kind) {
+    if (kind < -1 || kind > 2) return fail(ZERO_ERR_ARG, "zero_test_force_step_kernel: kind %d outside -1..2", kind);
+    zero::g_step_kernel_override.store(kind, std::memory_order_relaxed);
+    return zero::ok();
+}
 
 const char* zero_strerror(int code) {
     switch (code) {

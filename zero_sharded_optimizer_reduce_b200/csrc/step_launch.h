@@ -16,6 +16,7 @@ constexpr uint32_t kPipeSmemTarget = 180u * 1024u;  // shared memory of both sta
 constexpr uint32_t kPipeMinTile = 1536;             // elements: 3/4 of 4 x consumer threads
 constexpr uint32_t kPipeSmemMax = 220u * 1024u;     // dynamic shared memory cap
 constexpr int kPipeMaxWorld = 20;                   // largest N measured to gain from the pipeline
+constexpr int64_t kPipeMinTilesPerSm = 128;         // calls with fewer tiles per SM take the quad kernel
 
 using KernelFn = void (*)(StepParams);
 using StatsKernelFn = void (*)(StepParams, float*);
@@ -38,6 +39,26 @@ inline StatsKernelFn pick_stats_pipe_kernel(zero_dtype_t g, bool write) {
     if (write)
         return g == ZERO_F16 ? grad_stats_pipe_kernel<__half, true> : grad_stats_pipe_kernel<__nv_bfloat16, true>;
     return g == ZERO_F16 ? grad_stats_pipe_kernel<__half, false> : grad_stats_pipe_kernel<__nv_bfloat16, false>;
+}
+
+template <int B>
+inline KernelFn pick_quad_b(zero_dtype_t g, zero_dtype_t pd) {
+    constexpr int U = QuadShape<B>::U, NT = QuadShape<B>::NT;
+    if (g == ZERO_F16 && pd == ZERO_F16) return fused_step_quad_kernel<__half, __half, B, U, NT>;
+    if (g == ZERO_F16 && pd == ZERO_BF16) return fused_step_quad_kernel<__half, __nv_bfloat16, B, U, NT>;
+    if (g == ZERO_BF16 && pd == ZERO_F16) return fused_step_quad_kernel<__nv_bfloat16, __half, B, U, NT>;
+    return fused_step_quad_kernel<__nv_bfloat16, __nv_bfloat16, B, U, NT>;
+}
+
+// The quad-kernel instance for N replicas (N <= kQuadMaxWorld), its threads
+// per block and quads per thread and iteration.
+inline KernelFn pick_quad_kernel(zero_dtype_t g, zero_dtype_t pd, int world, int* nt, int* u) {
+    if (world <= 2) { *nt = QuadShape<2>::NT; *u = QuadShape<2>::U; return pick_quad_b<2>(g, pd); }
+    if (world <= 4) { *nt = QuadShape<4>::NT; *u = QuadShape<4>::U; return pick_quad_b<4>(g, pd); }
+    if (world <= 8) { *nt = QuadShape<8>::NT; *u = QuadShape<8>::U; return pick_quad_b<8>(g, pd); }
+    *nt = QuadShape<16>::NT;
+    *u = QuadShape<16>::U;
+    return pick_quad_b<16>(g, pd);
 }
 
 inline KernelFn pick_pipe_kernel(zero_dtype_t g, zero_dtype_t pd) {
@@ -297,26 +318,68 @@ inline int prepare_step(const char* fn, const void* const* grad_bufs, int32_t wo
         prm.nvec = (count - h) / kVec;
     }
     prm.tile = 0;
+    prm.kind = kKindRegister;
 
-    // The pipeline kernel takes calls whose arrays share a 16-byte phase, that
-    // give every SM at least two tiles and whose gradients are all this GPU's
-    // memory (its bulk copies never read another GPU's memory); the rest use
-    // the register kernel, whose plain loads read mapped peer memory too.
+    // Kernel choice (measured on B200 against the copy rate, L2 cold):
+    //  - arrays whose 16-byte phases never coincide, or N > kPipeMaxWorld: the
+    //    register kernel (its scalar path when unaligned; at N = 64 it runs at
+    //    the copy rate);
+    //  - N >= 3 with at least kPipeMinTilesPerSm tiles per SM and every
+    //    gradient buffer in this GPU's memory: the pipeline kernel (its bulk
+    //    copies never read another GPU's memory; 1.05 of the copy rate at
+    //    N = 4..16, 1B elements, against 0.99-1.05 for the quad kernel);
+    //  - N <= 16 otherwise: the quad kernel (N <= 2, where half of the bytes
+    //    are writes: 0.98 against 0.97; 16M elements at N = 1..16: 0.95-1.06
+    //    against 0.84-1.03, no pipeline to fill and drain; peer memory);
+    //  - 17 <= N <= 20 calls below the pipeline threshold: the pipeline kernel
+    //    when the gradients are local and every SM gets two tiles, else the
+    //    register kernel.
+    // zero_test_force_step_kernel overrides the choice where the forced
+    // kernel can run the call.
     int64_t blocks = 0;
-    const int tile = h >= 0 ? pipe_tile(world) : 0;
-    if (tile > 0) {
-        int sms = 0;
-        if (int rc = pipe_setup(grad_dtype, param_dtype, &sms)) return rc;
-        const int64_t ntiles = (count - h) / tile;
-        if (ntiles >= 2 * static_cast<int64_t>(sms) && all_local_device_memory(grad_bufs, world)) {
-            prm.tile = tile;
-            prm.nvec = ntiles * tile / kVec;
-            blocks = sms;
-        }
+    int sms = 0;
+    {
+        std::lock_guard<std::mutex> lk(g_dev_mu);
+        DeviceInfo* d = nullptr;
+        if (int rc = device_info(&d)) return rc;
+        sms = d->sms;
     }
-    if (prm.tile == 0) {
+    const int force = step_kernel_override();
+    const int tile = h >= 0 ? pipe_tile(world) : 0;
+    const int64_t ntiles = tile > 0 ? (count - h) / tile : 0;
+    int kind = kKindRegister;
+    if (h >= 0 && world <= kPipeMaxWorld) {
+        const bool big = ntiles >= kPipeMinTilesPerSm * static_cast<int64_t>(sms);
+        const bool local = all_local_device_memory(grad_bufs, world);
+        if (world <= kQuadMaxWorld && (world <= 2 || !big || !local)) kind = kKindQuad;
+        else if (local && ntiles >= 2 * static_cast<int64_t>(sms)) kind = kKindPipe;
+    }
+    if (force == kKindRegister) kind = kKindRegister;
+    if (force == kKindQuad && h >= 0 && world <= kQuadMaxWorld) kind = kKindQuad;
+    if (force == kKindPipe && tile > 0 && ntiles >= 1 && all_local_device_memory(grad_bufs, world)) kind = kKindPipe;
+    if (kind == kKindPipe) {
+        if (int rc = pipe_setup(grad_dtype, param_dtype, &sms)) return rc;
+        prm.tile = tile;
+        prm.nvec = ntiles * tile / kVec;
+        prm.kind = kKindPipe;
+        blocks = sms;
+    } else if (kind == kKindQuad) {
+        prm.kind = kKindQuad;
+        int nt = 0, u = 0;
+        (void)pick_quad_kernel(grad_dtype, param_dtype, world, &nt, &u);
+        const int64_t per_block = static_cast<int64_t>(nt) * u;
+        const int64_t work = prm.nvec > 0 ? 2 * prm.nvec : count;
+        blocks = (work + per_block - 1) / per_block;
+        const int64_t cap = static_cast<int64_t>(sms) * kQuadBlocksPerSm;
+        if (blocks > cap) blocks = cap;
+        if (blocks < 1) blocks = 1;
+    } else {
         int limit = 0;
         if (int rc = grid_limit(grad_dtype, param_dtype, &limit)) return rc;
+        if (h < 0 || h >= count) {
+            prm.head = count;
+            prm.nvec = 0;
+        }
         const int64_t work = prm.nvec > 0 ? prm.nvec : count;
         blocks = (work + kThreads - 1) / kThreads;
         if (blocks > limit) blocks = limit;
@@ -481,9 +544,13 @@ inline int launch_step(const char* fn, const StepParams& prm, int64_t blocks, ze
                        zero_dtype_t param_dtype, zero_stream_t stream) {
     if (blocks == 0) return ok();
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (prm.tile > 0) {
+    if (prm.kind == kKindPipe) {
         pick_pipe_kernel(grad_dtype, param_dtype)<<<static_cast<unsigned int>(blocks), kPipeThreads,
                                                      pipe_smem_bytes(prm.world, prm.tile), s>>>(prm);
+    } else if (prm.kind == kKindQuad) {
+        int nt = 0, u = 0;
+        KernelFn k = pick_quad_kernel(grad_dtype, param_dtype, prm.world, &nt, &u);
+        k<<<static_cast<unsigned int>(blocks), nt, 0, s>>>(prm);
     } else {
         pick_kernel(grad_dtype, param_dtype)<<<static_cast<unsigned int>(blocks), kThreads, 0, s>>>(prm);
     }

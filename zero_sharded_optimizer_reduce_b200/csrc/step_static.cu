@@ -14,9 +14,9 @@
 // Limits and rules:
 //  - the array holds the ticket and kStaticMaxBlocks (4096) fp64 partial
 //    sums, 33,024 bytes; every GPU that loads the library holds it until exit;
-//  - the fused kernels' grids are at most SM count x resident blocks (148 or
-//    296 blocks on a B200), so any input size fits; a call whose grid would
-//    need more than 4096 blocks is rejected with ZERO_ERR_RANGE;
+//  - the fused kernels' grids are at most 16 blocks per SM (2368 blocks on a
+//    B200), so any input size fits; a call whose grid would need more than
+//    4096 blocks is rejected with ZERO_ERR_RANGE;
 //  - every call on a device shares the array: calls that overlap on the GPU
 //    (different streams, or several host threads) race on it;
 //  - the first call on a device that asks for the norm looks up the array's
