@@ -555,14 +555,15 @@ def run_sweep(args):
 def run_stage3(args):
     """Layer-wise ZeRO-3 step on the 6.7B GPT shape (32 layers + embedding
     unit, N = 8): two gathers per unit plus the per-unit staged reduce-scatter
-    and gated in-place update, timed with and without gather prefetch, and
-    with the statistics-pass update for comparison.  One JSON line."""
+    and gated in-place update, timed without gather prefetch (the value) and
+    with it, and with the statistics-pass update for comparison.  One JSON
+    line."""
     import torch
     import zero_sharded_optimizer_reduce_b200 as Z
     torch.cuda.set_device(0)
     w = workloads.gpt_6p7b_layerwise()
     out = {}
-    for prefetch, update in ((False, "staged"), (True, "stats"), (True, "staged")):
+    for prefetch, update in ((False, "staged"), (False, "stats"), (True, "staged")):
         s3 = Z.ZeroStage3(w.numels, w.world, lr=w.adam.lr, betas=(w.adam.beta1, w.adam.beta2), eps=w.adam.eps,
                           weight_decay=w.adam.weight_decay, loss_scale=w.loss_scale, prefetch=prefetch,
                           update=update)
@@ -603,18 +604,20 @@ def run_stage3(args):
     N = w.world
     bpe = 8 + 2 * N + 34          # 2 gathers x (2 read + 2 write) + reduce-scatter to fp32 + update
     bpe_stats = 8 + 4 * N + 26    # 2 gathers + statistics pass + fused gated update
-    best = out[(True, "staged")]
+    # the default configuration (no prefetch: on one GPU the side stream only
+    # competes for the same HBM) is the line's value; prefetch is reported beside it
+    best = out[(False, "staged")]
     peak, peak_kind = peaks()
     line = {"metric": "ZeRO-3 layer-wise step (gathers + staged reduce-scatter + gated in-place update)",
             "unit": "Gparams/s", "value": psi / (best * 1e-3) / 1e9, "ms_per_step": best,
-            "ms_per_step_no_prefetch": out[(False, "staged")],
-            "prefetch_gain": out[(False, "staged")] / best - 1.0, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step_prefetch": out[(True, "staged")],
+            "prefetch_gain": best / out[(True, "staged")] - 1.0, "steps": args.steps, "warmup": args.warmup,
             "config": {"workload": w.name, "psi_padded": psi, "world": N, "units": len(w.numels)},
             "hbm_gbs": psi * bpe / (best * 1e-3) / 1e9, "bytes_per_elem": bpe,
             "frac_measured": psi * bpe / (best * 1e-3) / 1e9 / peak, "peak_kind": peak_kind,
-            "stats_update": {"ms_per_step": out[(True, "stats")], "bytes_per_elem": bpe_stats,
-                             "value": psi / (out[(True, "stats")] * 1e-3) / 1e9,
-                             "frac_measured": psi * bpe_stats / (out[(True, "stats")] * 1e-3) / 1e9 / peak},
+            "stats_update": {"ms_per_step": out[(False, "stats")], "bytes_per_elem": bpe_stats,
+                             "value": psi / (out[(False, "stats")] * 1e-3) / 1e9,
+                             "frac_measured": psi * bpe_stats / (out[(False, "stats")] * 1e-3) / 1e9 / peak},
             "allgather": {"elements": gather_elems, "ms": gather_ms, "bytes_per_elem": 4,
                           "gbs": gather_elems * 4 / (gather_ms * 1e-3) / 1e9,
                           "frac_measured": gather_elems * 4 / (gather_ms * 1e-3) / 1e9 / peak,

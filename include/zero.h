@@ -482,7 +482,10 @@ int zero_test_wait_timeout(int32_t* status, int64_t limit_ns, zero_stream_t stre
  * makes the process's later calls take `kind` instead wherever that kernel
  * can run the call (the pipeline kernel needs a common phase, N <= 20, one
  * whole tile and gradients in this GPU's memory; the quad kernel a common
- * phase), so that tests reach each kernel at small sizes.
+ * phase and N <= 16), so that tests reach each kernel at small sizes.  The
+ * statistics pass, the staged reduce-scatter and the staged update follow it
+ * too: 1 forces their pipeline kernels, 0 their register kernels (2 leaves
+ * their automatic choice).
  * kind  -1 automatic (the default), 0 register, 1 pipeline, 2 quad
  * Errors: ZERO_ERR_ARG.  Host only, no CUDA call.
  */

@@ -386,3 +386,16 @@ def test_staged_runner_rejects_bad_arguments():
     assert call(max_norm=1.0) == -1                       # clipping without a norm
     assert call(sq=0x60000) == -1                         # a norm without a workspace
     assert call(flag=0x40004) == -2                       # the two flag words must be 8-byte aligned
+
+
+def test_step_kernel_hook_validates_and_resets():
+    """zero_test_force_step_kernel: host only, -1..2 accepted, anything else
+    ZERO_ERR_ARG; the binding's names match the C values."""
+    L = Z.lib
+    for kind in (Z.STEP_KERNEL_REGISTER, Z.STEP_KERNEL_PIPE, Z.STEP_KERNEL_QUAD, Z.STEP_KERNEL_AUTO):
+        assert L.zero_test_force_step_kernel(kind) == 0
+    assert L.zero_test_force_step_kernel(3) == -1
+    assert L.zero_test_force_step_kernel(-2) == -1
+    assert b"kind" in L.zero_last_error()
+    assert (Z.STEP_KERNEL_AUTO, Z.STEP_KERNEL_REGISTER, Z.STEP_KERNEL_PIPE, Z.STEP_KERNEL_QUAD) == (-1, 0, 1, 2)
+    Z.zero_test_force_step_kernel(Z.STEP_KERNEL_AUTO)

@@ -4,8 +4,10 @@ No Python and no torch on the data path: the program allocates every buffer
 with the CUDA runtime, reads seeded inputs from a file, runs three steps
 through the native runner (zero_runner_create / _launch / _commit, one of
 them with an injected inf so that it is skipped), then the staged route
-(zero_reduce_scatter_grads + zero_adam_step_reduced) for one more step, and
-writes the committed state back to a file.  The test compares every array
+(zero_reduce_scatter_grads + zero_adam_step_reduced) for one more step,
+writes the committed state back to a file, and rebuilds the parameters from 4
+rank shards with zero_allgather_params (an odd partition: ranks 1-3 sit off
+their destination's 16-byte phase).  The test compares every array
 with the oracle bit for bit, and the runner's t and loss scale with the
 oracle's rule.
 """
@@ -110,6 +112,27 @@ int main(int argc, char** argv) {
     }
     CK(cudaMemcpy(params_host, bk.params[bank], (size_t)n * 2, cudaMemcpyDeviceToHost));
     fwrite(params_host, 2, (size_t)n, out);
+
+    /* the all-gather: the parameters split into `world` rank shards of their
+       own, rebuilt into one buffer (P odd: ranks 1.. are realigned) */
+    const int64_t P = n / world;
+    void* shards[ZERO_MAX_WORLD];
+    for (int k = 0; k < world; ++k) {
+        if (!(shards[k] = dalloc((size_t)P * 2))) return 2;
+        CK(cudaMemcpy(shards[k], (const uint16_t*)bk.params[bank] + (size_t)k * P, (size_t)P * 2,
+                      cudaMemcpyDeviceToDevice));
+    }
+    uint16_t* full = dalloc((size_t)n * 2);
+    int32_t* status = dalloc(4);
+    if (!full || !status) return 2;
+    CK(cudaMemset(full, 0xEE, (size_t)n * 2));
+    CK(cudaMemset(status, 0, 4));
+    ZK(zero_allgather_params((const void* const*)shards, world, 0, P, ZERO_F16, full, status, NULL));
+    int32_t st = -1;
+    CK(cudaMemcpy(&st, status, 4, cudaMemcpyDeviceToHost));
+    printf("gather %d\n", st);
+    CK(cudaMemcpy(params_host, full, (size_t)n * 2, cudaMemcpyDeviceToHost));
+    fwrite(params_host, 2, (size_t)n, out);
     fclose(out);
     return 0;
 }
@@ -169,3 +192,8 @@ def test_c_program_runs_the_step_through_the_abi(tmp_path):
     for arr, name in zip(got, ("master", "m", "v")):
         assert np.array_equal(arr.view(np.uint32), getattr(ref, name).view(np.uint32)), name
     assert np.array_equal(params, ref.params)
+    # the all-gather of the 4 rank shards through the C ABI
+    assert lines[5] == "gather 0"
+    P = n // world
+    gathered = np.frombuffer(data, np.uint16, n, 14 * n)
+    assert np.array_equal(gathered, oracle.allgather([ref.params[r * P:(r + 1) * P] for r in range(world)], 0, P))

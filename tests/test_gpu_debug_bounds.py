@@ -70,9 +70,18 @@ def test_fused_step_in_bounds(world, padded, part, offs, kind):
     assert c.compare(ref) == [0, 0, 0, 0]
 
 
+@pytest.mark.parametrize("kind", [Z.STEP_KERNEL_AUTO, Z.STEP_KERNEL_REGISTER, Z.STEP_KERNEL_PIPE])
 @pytest.mark.parametrize("world,padded,part", [(8, 8 * 250_003, -1), (16, 16 * 60_001, -1), (3, 3 * 7_001, 2),
                                                 (2, 2 * 1_900_003, 1)])
-def test_staged_route_and_statistics_in_bounds(world, padded, part):
+def test_staged_route_and_statistics_in_bounds(world, padded, part, kind):
+    Z.zero_test_force_step_kernel(kind)
+    try:
+        _staged_route_and_statistics(world, padded, part)
+    finally:
+        Z.zero_test_force_step_kernel(Z.STEP_KERNEL_AUTO)
+
+
+def _staged_route_and_statistics(world, padded, part):
     c = Staged(padded, world, seed=720 + world, scale=65536.0, partition=part, inplace=True)
     c.reduce_scatter()
     s, inv, g = c.oracle_reduced()

@@ -260,15 +260,25 @@ def test_checkpoint_resume_bit_identical(mode):
             assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
 
 
+@pytest.fixture
+def force_pipeline():
+    Z.zero_test_force_step_kernel(Z.STEP_KERNEL_PIPE)
+    try:
+        yield
+    finally:
+        Z.zero_test_force_step_kernel(Z.STEP_KERNEL_AUTO)
+
+
 def _stats_tile(world):
     return min(8192, (180 * 1024 // (2 * 2 * world)) // 512 * 512)
 
 
 @pytest.mark.parametrize("world,dtype,goff", [(8, oracle.F16, 0), (8, oracle.F16, 3), (16, oracle.BF16, 0),
                                               (1, oracle.F16, 5), (3, oracle.BF16, 1)])
-def test_stats_pipeline(world, dtype, goff):
-    """Sizes that give every SM at least two tiles: the statistics pipeline
-    kernel runs, with ragged tails and (goff > 0) a scalar head."""
+def test_stats_pipeline(world, dtype, goff, force_pipeline):
+    """Sizes that give every SM at least two tiles, the statistics pipeline
+    kernel forced (in normal use it takes calls of 128 tiles per SM and
+    more), with ragged tails and (goff > 0) a scalar head."""
     T = _stats_tile(world)
     per_rank = (2 * 148 * T + 777) // world + 3
     c = Case(world * per_rank, world, gdtype=dtype, pdtype=dtype, seed=460 + world, goff=goff, scale=65536.0)

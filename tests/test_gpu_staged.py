@@ -4,11 +4,12 @@ zero_adam_step_reduced) against the oracle.
 The reduce-scatter's fp32 output must equal the oracle's unscaled rank-order
 sums bit for bit (flag exact, norm within the fp64 reordering bound); the
 update from it must equal the oracle's step on the same inputs bit for bit,
-in and out of place, gated and clipped.  Sizes cover the register and the
-pipeline statistics kernels (N <= 20 and enough tiles), ragged tails,
+in and out of place, gated and clipped.  Every case runs twice: with the
+automatic kernel choice and with the pipeline kernels forced (the
+test hook zero_test_force_step_kernel), so that both the register and the
+pipeline statistics and update kernels run at these sizes; ragged tails,
 single partitions, bf16, a reduced buffer off the gradients' 16-byte phase
-(scalar path), N up to 64, and sizes that take the update's pipeline
-kernel (at least two 6144-element tiles per SM).
+(scalar path), N up to 64, and sizes of at least two update tiles per SM.
 """
 import numpy as np
 import pytest
@@ -24,6 +25,18 @@ from test_gpu_step import Case, _adam, _hp
 pytestmark = pytest.mark.gpu
 
 SMS = 148
+
+
+@pytest.fixture(autouse=True, params=["auto", "pipeline"])
+def kernel_choice(request):
+    """Every case twice: the automatic choice (the statistics and update
+    pipelines take calls of 128 tiles per SM and more, so these sizes run the
+    register kernels) and the pipeline kernels forced wherever they can run."""
+    Z.zero_test_force_step_kernel(Z.STEP_KERNEL_PIPE if request.param == "pipeline" else Z.STEP_KERNEL_AUTO)
+    try:
+        yield request.param
+    finally:
+        Z.zero_test_force_step_kernel(Z.STEP_KERNEL_AUTO)
 
 
 class Staged(Case):

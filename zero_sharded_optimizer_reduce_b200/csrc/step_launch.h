@@ -138,7 +138,7 @@ inline int grid_limit(zero_dtype_t g, zero_dtype_t pd, int* out) {
         if (e != cudaSuccess || n < 1) return fail(ZERO_ERR_CUDA, "occupancy query failed: %s", cudaGetErrorString(e));
         d->blocks_per_sm[which] = n;
     }
-    int lim = d->sms * d->blocks_per_sm[which];
+    int lim = kRegWaves * d->sms * d->blocks_per_sm[which];
     *out = lim < kMaxBlocks ? lim : kMaxBlocks;
     return ZERO_OK;
 }
@@ -154,7 +154,7 @@ inline int stats_grid_limit(zero_dtype_t g, bool write, int* out) {
         if (e != cudaSuccess || n < 1) return fail(ZERO_ERR_CUDA, "occupancy query failed: %s", cudaGetErrorString(e));
         d->stats_blocks_per_sm[which] = n;
     }
-    int lim = d->sms * d->stats_blocks_per_sm[which];
+    int lim = kRegWaves * d->sms * d->stats_blocks_per_sm[which];
     *out = lim < kMaxBlocks ? lim : kMaxBlocks;
     return ZERO_OK;
 }
@@ -349,10 +349,15 @@ inline int prepare_step(const char* fn, const void* const* grad_bufs, int32_t wo
     const int64_t ntiles = tile > 0 ? (count - h) / tile : 0;
     int kind = kKindRegister;
     if (h >= 0 && world <= kPipeMaxWorld) {
+        const bool quad_ok = world <= kQuadMaxWorld;
         const bool big = ntiles >= kPipeMinTilesPerSm * static_cast<int64_t>(sms);
-        const bool local = all_local_device_memory(grad_bufs, world);
-        if (world <= kQuadMaxWorld && (world <= 2 || !big || !local)) kind = kKindQuad;
-        else if (local && ntiles >= 2 * static_cast<int64_t>(sms)) kind = kKindPipe;
+        if (quad_ok && (world <= 2 || !big)) {
+            kind = kKindQuad;
+        } else if (all_local_device_memory(grad_bufs, world)) {   // queried only where it decides
+            if (big || ntiles >= 2 * static_cast<int64_t>(sms)) kind = kKindPipe;
+        } else if (quad_ok) {
+            kind = kKindQuad;
+        }
     }
     if (force == kKindRegister) kind = kKindRegister;
     if (force == kKindQuad && h >= 0 && world <= kQuadMaxWorld) kind = kKindQuad;
@@ -485,7 +490,14 @@ inline int prepare_stats(const char* fn, const void* const* grad_bufs, int32_t w
         int sms = 0;
         if (int rc = stats_pipe_setup(grad_dtype, reduced != nullptr, &sms)) return rc;
         const int64_t ntiles = (count - h) / tile;
-        if (ntiles >= 2 * static_cast<int64_t>(sms) && all_local_device_memory(grad_bufs, world)) {
+        // from two tiles per SM (unlike the step and the staged update: with
+        // gradients alone, the register kernel keeps too few bytes in flight
+        // at small N; measured on B200, 16M x N = 4: 0.85 pipeline against
+        // 0.71 register for the reduce-scatter, 64M x N = 8: 1.05 against 1.03)
+        const int force = step_kernel_override();
+        const bool want = force == kKindPipe ? ntiles >= 1
+                                             : force != kKindRegister && ntiles >= 2 * static_cast<int64_t>(sms);
+        if (want && all_local_device_memory(grad_bufs, world)) {
             prm.tile = tile;
             prm.nvec = ntiles * tile / kVec;
             blocks = sms;

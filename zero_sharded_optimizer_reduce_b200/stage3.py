@@ -1,4 +1,4 @@
-"""ZeroStage3: the ZeRO-3 layer-wise step on one GPU, with gather prefetch.
+"""ZeroStage3: the ZeRO-3 layer-wise step on one GPU, optional gather prefetch.
 
 ZeRO explainer, "Stage 3 - Parameter Partitioning (P_os+g+p)": each rank
 keeps only its 1/N slice of every parameter; a layer's full parameters are
@@ -23,7 +23,9 @@ Step: forward gathers u = 0 .. U-1, then for u = U-1 .. 0: gather, gradients,
 update.  With prefetch, the gather of the next unit runs on a side stream
 into the other layer buffer while the current unit's work runs; events order
 the buffers.  On one GPU both streams share HBM, so prefetch can only fill
-the gaps between kernels.
+the gaps between kernels: measured on B200 (6.7B shape) it cost 3 % (62.5
+against 60.6 ms per step), so it is off by default here; it pays where the
+gathers come over NVLink.
 
 Skip scope: each unit's update is gated by that unit's own statistics (the
 units' gradients never coexist in memory); the host reads the per-unit flags
@@ -42,7 +44,7 @@ class ZeroStage3:
     def __init__(self, unit_numels, world: int, *, align_elems: int = 8, lr: float = 1e-3, betas=(0.9, 0.999),
                  eps: float = 1e-8, weight_decay: float = 0.0, grad_dtype=torch.float16,
                  param_dtype=torch.float16, loss_scale: float = 65536.0, growth_interval: int = 1000,
-                 min_scale: float = 1.0, prefetch: bool = True, update: str = "staged", device="cuda"):
+                 min_scale: float = 1.0, prefetch: bool = False, update: str = "staged", device="cuda"):
         if update not in ("staged", "stats"):
             raise ValueError("update must be 'staged' or 'stats'")
         self.update_mode = update
