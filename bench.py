@@ -21,6 +21,15 @@ step time is the max over ranks, and `value` sums all ranks' elements.
 
 --impl reference times the CPU oracle (C, OpenMP) on the host cores, each
 step a bounded slice of the same workload.
+
+Other modes (each prints JSON lines of its own):
+  --mode {inplace,staged}, --max-grad-norm X   the one-bank step routes, clipping
+  --flat PSI --world N                         a flat workload instead of GPT-2
+  --sweep                                      the flat bandwidth sweep (kernel calls alone)
+  --allgather P --world N                      the all-gather of N slices of P elements
+  --stage3                                     the layer-wise ZeRO-3 step, 6.7B shape
+  --distributed {banks,staged} [--stage3]      one process per GPU under torchrun (real ranks)
+  --cpu-configs                                the CPU oracle on every workload (no GPU)
 """
 from __future__ import annotations
 
@@ -242,6 +251,62 @@ def cpu_baseline(w: workloads.Workload, sample_elems: int, min_seconds: float = 
                       f"{head['single_thread_steps']} step(s) of the same slice on 1 thread; configs: the full "
                       f"arrays of the tiny and the dynamic-loss-scale workloads, same protocol",
             "configs": configs}
+
+
+def run_cpu_configs(args):
+    """The oracle timed on every workload the way the survey's measurement
+    plan asks: the full arrays of the tiny and the dynamic-loss-scale
+    workloads, 64M-element slices of the GPT-2 1.5B bucket, of one 6.7B unit
+    and of the sweep's flat buffers (N = 1, 8, 16 and 64), each on every host
+    core and on one thread.  One JSON line; no GPU is used."""
+    import oracle
+    cores = oracle.threads()
+    S = args.cpu_sample
+
+    def rate(G, master, adam, loss_scale, divisor, secs=4.0):
+        v, steps, el = _oracle_rate(G, master, adam, loss_scale, divisor, secs)
+        oracle.set_threads(1)
+        try:
+            v1, _, el1 = _oracle_rate(G, master, adam, loss_scale, divisor, float("inf"), max_steps=1)
+        finally:
+            oracle.set_threads(cores)
+        return {"value": v, "single_thread_value": v1, "steps": steps, "seconds": round(el, 2),
+                "single_thread_seconds": round(el1, 2)}
+
+    def draws(n, world, seed, std, scale, distinct=2):
+        # `distinct` seeded draws; further replicas are seeded rotations of them
+        base = [workloads.grads(n, workloads.seed_for(seed, 1, k), std, scale) for k in range(min(distinct, world))]
+        return [base[k] if k < len(base) else np.roll(base[k % len(base)], 7919 * k) for k in range(world)]
+
+    out = {}
+    tiny = workloads.tiny_flat()
+    padded = -(-tiny.numels[0] // tiny.world) * tiny.world
+    out[tiny.name] = dict(rate(draws(padded, tiny.world, tiny.seed, tiny.grad_std, tiny.loss_scale, tiny.world),
+                               workloads.master(padded, 7), tiny.adam, tiny.loss_scale, float(tiny.world)),
+                          elements=padded, world=tiny.world, sample="full arrays")
+    g2 = workloads.gpt2_1p5b()
+    out[g2.name] = dict(rate(draws(S, g2.world, g2.seed, g2.grad_std, g2.loss_scale), workloads.master(S, 14),
+                             g2.adam, g2.loss_scale, float(g2.world)),
+                        elements=S, world=g2.world, sample=f"{S:,}-element slice of bucket 0")
+    ov = workloads.overflow_flat()
+    out[ov.name] = dict(rate(draws(ov.numels[0], ov.world, ov.seed, ov.grad_std, ov.loss_scale),
+                             workloads.master(ov.numels[0], 21), ov.adam, ov.loss_scale, float(ov.world)),
+                        elements=ov.numels[0], world=ov.world, sample="full arrays")
+    g3 = workloads.gpt_6p7b_layerwise()
+    out[g3.name] = dict(rate(draws(S, g3.world, g3.seed, g3.grad_std, g3.loss_scale), workloads.master(S, 28),
+                             g3.adam, g3.loss_scale, float(g3.world)),
+                        elements=S, world=g3.world, sample=f"{S:,}-element slice of unit 0")
+    for N in (1, 8, 16, 64):
+        adam = workloads.AdamConfig(weight_decay=0.01)
+        out[f"sweep_flat_n{N}"] = dict(rate(draws(S, N, 5, 1e-3, 65536.0), workloads.master(S, 35), adam, 65536.0,
+                                            float(N)),
+                                       elements=S, world=N, sample=f"{S:,}-element slice of a flat buffer")
+    print(json.dumps({"metric": "CPU oracle: Gparams/s per workload (reduce-scatter, overflow test, Adam)",
+                      "unit": UNIT, "cores": cores, "kind": "oracle",
+                      "note": "replicas past the first two of each workload are seeded rotations of those "
+                              "draws (the same distribution; the oracle's time does not depend on the values)",
+                      "configs": out}), flush=True)
+    return 0
 
 
 def run_reference(args):
@@ -905,6 +970,8 @@ def main(argv=None):
                          "staged: one bank, reduce-scatter to fp32 + gated update")
     ap.add_argument("--max-grad-norm", type=float, default=None, help="clip gradients to this global norm")
     ap.add_argument("--sweep-dtype-only", action="store_true", help="sweep only --grad-dtype")
+    ap.add_argument("--cpu-configs", action="store_true",
+                    help="time the CPU oracle on every workload (full arrays or 64M slices), one JSON line")
     ap.add_argument("--allgather", type=int, default=0,
                     help="time the all-gather of --world slices of this many elements, one JSON line")
     ap.add_argument("--distributed", choices=["banks", "staged"], default=None,
@@ -917,6 +984,8 @@ def main(argv=None):
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         return run_reference(args)
+    if args.cpu_configs:
+        return run_cpu_configs(args)
     if args.sweep:
         return run_sweep(args)
     if args.allgather:

@@ -149,7 +149,7 @@ inline int prepare_reduced(const char* fn, const float* reduced, int64_t count, 
 // the register kernel (plain loads, a grid of kRegWaves waves).  Measured on
 // B200 (fp32 reduced gradients in, 30 bytes per element): 16M elements 0.93
 // register against 0.88 pipeline, 64M 0.98 against 0.96, 256M both 0.97-0.98
-// of the copy rate this pool measures.  `work` as returned by prepare_reduced (> 0).
+// of a measured B200 copy rate (6.43 TB/s).  `work` as returned by prepare_reduced (> 0).
 inline int launch_reduced(const char* fn, StepParams prm, const ParamDsts& d, int64_t work, zero_dtype_t pd,
                           bool bcast, zero_stream_t stream) {
     ReducedDevice* dev = nullptr;
