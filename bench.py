@@ -483,10 +483,21 @@ def run_gpu(args):
     kern_s = sum(launch_ms) * 1e-3
     achieved = kern_bytes / kern_s / 1e9
     avg_elems = sum(launch_elems) / len(launch_elems)
+    # the fused-step kernel each bucket ran (single-pass banks mode): the
+    # committed traffic record is the pipeline kernel's
+    kinds = opt.bucket_kernels()
     if args.mode == "staged":
         traffic = profiled_traffic(avg_elems, "staged_step" if -1 in ev else "staged")
     else:
-        traffic = profiled_traffic(avg_elems) if args.mode == "banks" else None
+        traffic = (profiled_traffic(avg_elems) if kinds and all(k == Z.STEP_KERNEL_PIPE for k in kinds)
+                   else None)
+    if kinds:
+        names = {Z.STEP_KERNEL_REGISTER: "register-streaming", Z.STEP_KERNEL_PIPE: "shared-memory pipeline",
+                 Z.STEP_KERNEL_QUAD: "quad-streaming"}
+        fused_label = "fused_step per bucket: " + ", ".join(
+            f"{kinds.count(k)} x {names[k]} kernel" for k in sorted(set(kinds)))
+    else:
+        fused_label = "statistics pass + gated update kernels"
 
     # ---- end to end through the public API: host gradients in, flag out
     e2e = None
@@ -518,13 +529,11 @@ def run_gpu(args):
                 "hbm_gbs": value * 1e9 * bpe / world_gpus / 1e9,
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
                              "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
-                             "kernel": ("staged step (reduce-scatter to fp32 + update from it, pipeline kernels); "
+                             "kernel": ("staged step (reduce-scatter to fp32 + update from it); "
                                         "timed per step over all buckets" if args.mode == "staged" and -1 in ev else
-                                        "fused_step (shared-memory pipeline kernel for aligned calls of >= 2 tiles per SM); "
-                                        "timed per step over all buckets" if -1 in ev else
-                                        "adam_reduced_kernel (update from the fp32 reduced gradients)"
-                                        if args.mode == "staged" else
-                                        "fused_step (shared-memory pipeline kernel for aligned calls of >= 2 tiles per SM)"),
+                                        fused_label + "; timed per step over all buckets" if -1 in ev else
+                                        "adam_reduced kernels (update from the fp32 reduced gradients)"
+                                        if args.mode == "staged" else fused_label),
                              "bytes_per_elem": kbpe,
                              "elems_per_launch": avg_elems, "launches_timed": len(launch_ms),
                              "timed_unit": ("one step: all buckets' kernels + flag clear + flag read-back"

@@ -585,6 +585,21 @@ int zero_runner_state(const zero_runner_t* runner, int64_t* t, float* loss_scale
                       int32_t* bank);
 int zero_runner_set_state(zero_runner_t* runner, int64_t t, float loss_scale, int32_t good_steps, int32_t bank);
 void zero_runner_destroy(zero_runner_t* runner);
+/*
+ * zero_runner_bucket_kernel - which fused-step kernel the next
+ * zero_runner_launch runs for bucket `bucket` of a two-bank runner: 0 the
+ * register-streaming kernel, 1 the shared-memory pipeline kernel, 2 the
+ * quad-streaming kernel (the numbering of zero_test_force_step_kernel).  It
+ * makes the launch's own preparation (bank cur, the current t and loss
+ * scale, the kernel override in force) without enqueueing anything; the
+ * choice depends on the bucket's size, N, the buffers' 16-byte phase and
+ * whether every gradient buffer is this device's memory.
+ * Errors: ZERO_ERR_ARG for a NULL argument, a bucket outside
+ * 0..n_buckets-1 or a staged runner; else those of
+ * zero_reduce_scatter_adam_step's validation.
+ */
+int zero_runner_bucket_kernel(const zero_runner_t* runner, int64_t bucket, int32_t* kind);
+
 
 /* ------------------------------------------------------------------------ */
 /* Multi-process ranks: sharing gradient and parameter buffers               */

@@ -399,3 +399,13 @@ def test_step_kernel_hook_validates_and_resets():
     assert b"kind" in L.zero_last_error()
     assert (Z.STEP_KERNEL_AUTO, Z.STEP_KERNEL_REGISTER, Z.STEP_KERNEL_PIPE, Z.STEP_KERNEL_QUAD) == (-1, 0, 1, 2)
     Z.zero_test_force_step_kernel(Z.STEP_KERNEL_AUTO)
+
+
+def test_runner_bucket_kernel_rejects_bad_arguments():
+    """zero_runner_bucket_kernel: a NULL runner or a NULL result is
+    ZERO_ERR_ARG before anything touches CUDA."""
+    L = Z.lib
+    kind = ctypes.c_int32(7)
+    assert L.zero_runner_bucket_kernel(None, 0, ctypes.byref(kind)) == -1
+    assert kind.value == 7
+    assert b"NULL" in L.zero_last_error()

@@ -86,3 +86,24 @@ def test_automatic_choice_mid_size(world):
     ref, ovf, sq = c.expect(_adam(0.01), t=1)
     c.run(_adam(0.01), t=1)
     assert ovf == 0 and c.compare(ref) == [0, 0, 0, 0]
+
+
+def test_runner_reports_the_kernel_choice():
+    """zero_runner_bucket_kernel names the kernel the next launch runs: the
+    pipeline kernel for a 64M-element bucket at N = 8 (147 tiles per SM), the
+    quad kernel for a 1M-element bucket, the register kernel above N = 20,
+    and whatever the override forces."""
+    from zero_sharded_optimizer_reduce_b200.optimizer import ZeroAdam
+    opt = ZeroAdam([64 << 20, 1 << 20], world=8, bucket_elems=64 << 20)
+    assert opt.layout.n_buckets == 2
+    assert opt.bucket_kernels() == [Z.STEP_KERNEL_PIPE, Z.STEP_KERNEL_QUAD]
+    Z.zero_test_force_step_kernel(Z.STEP_KERNEL_REGISTER)
+    try:
+        assert opt.bucket_kernels() == [Z.STEP_KERNEL_REGISTER, Z.STEP_KERNEL_REGISTER]
+    finally:
+        Z.zero_test_force_step_kernel(Z.STEP_KERNEL_AUTO)
+    del opt
+    assert ZeroAdam([240_000], world=24).bucket_kernels() == [Z.STEP_KERNEL_REGISTER]
+    assert ZeroAdam([240_000], world=2).bucket_kernels() == [Z.STEP_KERNEL_QUAD]
+    assert ZeroAdam([240_000], world=4, mode="staged").bucket_kernels() is None
+    torch.cuda.empty_cache()

@@ -147,6 +147,8 @@ def load_library(path: str = LIB_PATH):
     L.zero_runner_set_state.restype = ctypes.c_int
     L.zero_runner_destroy.argtypes = [vp]
     L.zero_runner_destroy.restype = None
+    L.zero_runner_bucket_kernel.argtypes = [vp, i64, ctypes.POINTER(i32)]
+    L.zero_runner_bucket_kernel.restype = ctypes.c_int
     L.zero_test_wait_timeout.argtypes = [vp, i64, vp]
     L.zero_test_wait_timeout.restype = ctypes.c_int
     L.zero_test_force_step_kernel.argtypes = [i32]
@@ -525,6 +527,13 @@ class Runner:
 
     def set_state(self, t: int, scale: float, good: int, bank: int) -> None:
         _check(lib.zero_runner_set_state(self._h, t, scale, good, bank))
+
+    def bucket_kernel(self, bucket: int) -> int:
+        """The fused-step kernel the next launch runs for `bucket`:
+        STEP_KERNEL_REGISTER, STEP_KERNEL_PIPE or STEP_KERNEL_QUAD."""
+        kind = ctypes.c_int32()
+        _check(lib.zero_runner_bucket_kernel(self._h, bucket, ctypes.byref(kind)))
+        return kind.value
 
     def __del__(self):
         h = getattr(self, "_h", None)

@@ -276,4 +276,27 @@ extern "C" int zero_runner_set_state(zero_runner_t* r, int64_t t, float loss_sca
     return zero::ok();
 }
 
+extern "C" int zero_runner_bucket_kernel(const zero_runner_t* r, int64_t bucket, int32_t* kind) {
+    const char* fn = "zero_runner_bucket_kernel";
+    if (!r || !kind) return fail(ZERO_ERR_ARG, "%s: NULL argument", fn);
+    if (r->staged) return fail(ZERO_ERR_ARG, "%s: a staged runner has no fused-step kernel", fn);
+    if (bucket < 0 || bucket >= static_cast<int64_t>(r->banks.size()))
+        return fail(ZERO_ERR_ARG, "%s: bucket %lld outside 0..%lld", fn, (long long)bucket,
+                    (long long)r->banks.size() - 1);
+    // the same preparation the next launch makes (bank cur -> cur ^ 1)
+    const int c = r->cur, n = c ^ 1;
+    const zero_bucket_banks_t& d = r->banks[bucket];
+    zero_adam_hparams_t hp = r->hp;
+    hp.step = r->t + 1;
+    zero::fused::StepParams prm{};
+    int64_t blocks = 0;
+    if (int rc = zero::fused::prepare_step(fn, r->grads[bucket].data(), r->world, r->numel[bucket],
+                                           ZERO_ALL_PARTITIONS, r->grad_dtype, d.master[c], d.m[c], d.v[c],
+                                           d.master[n], d.m[n], d.v[n], d.params[n], r->param_dtype, &hp, r->scale,
+                                           r->flag_dev, r->sqnorm, r->workspace, &prm, &blocks))
+        return rc;
+    *kind = prm.kind;
+    return zero::ok();
+}
+
 extern "C" void zero_runner_destroy(zero_runner_t* r) { delete r; }

@@ -135,6 +135,14 @@ class ZeroAdam:
         c = self.cur
         return self.master[b][c], self.m[b][c], self.v[b][c], self.params_bank[b][c]
 
+    def bucket_kernels(self):
+        """The fused-step kernel each bucket's next step runs (STEP_KERNEL_REGISTER,
+        _PIPE or _QUAD, per zero_runner_bucket_kernel); None in the two-pass
+        modes, which run the statistics and update kernels instead."""
+        if self._runner is None or self.two_pass:
+            return None
+        return [self._runner.bucket_kernel(b) for b in range(self.layout.n_buckets)]
+
     def grad_buffers(self, b: int):
         """The N replicas' gradient buffers of bucket b (write gradients here)."""
         return self.grads[b]
