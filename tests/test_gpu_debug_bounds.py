@@ -70,7 +70,8 @@ def test_fused_step_in_bounds(world, padded, part, offs, kind):
     assert c.compare(ref) == [0, 0, 0, 0]
 
 
-@pytest.mark.parametrize("kind", [Z.STEP_KERNEL_AUTO, Z.STEP_KERNEL_REGISTER, Z.STEP_KERNEL_PIPE])
+@pytest.mark.parametrize("kind", [Z.STEP_KERNEL_AUTO, Z.STEP_KERNEL_REGISTER, Z.STEP_KERNEL_PIPE,
+                                  Z.STEP_KERNEL_QUAD])
 @pytest.mark.parametrize("world,padded,part", [(8, 8 * 250_003, -1), (16, 16 * 60_001, -1), (3, 3 * 7_001, 2),
                                                 (2, 2 * 1_900_003, 1)])
 def test_staged_route_and_statistics_in_bounds(world, padded, part, kind):

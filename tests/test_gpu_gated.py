@@ -277,8 +277,9 @@ def _stats_tile(world):
                                               (1, oracle.F16, 5), (3, oracle.BF16, 1)])
 def test_stats_pipeline(world, dtype, goff, force_pipeline):
     """Sizes that give every SM at least two tiles, the statistics pipeline
-    kernel forced (in normal use it takes calls of 128 tiles per SM and
-    more), with ragged tails and (goff > 0) a scalar head."""
+    kernel forced (in normal use it takes the reduce-scatter at N = 3..8 from
+    128 tiles per SM, and N = 17..20), with ragged tails and (goff > 0) a
+    scalar head."""
     T = _stats_tile(world)
     per_rank = (2 * 148 * T + 777) // world + 3
     c = Case(world * per_rank, world, gdtype=dtype, pdtype=dtype, seed=460 + world, goff=goff, scale=65536.0)
@@ -295,6 +296,30 @@ def test_stats_pipeline(world, dtype, goff, force_pipeline):
         assert flag == 1 == _oracle_stats(c)[0]
         c.G[world - 1] = g
         to_dev_u16(g, TD[dtype], buf=c.g_dev[world - 1])
+
+
+@pytest.mark.parametrize("kind", [Z.STEP_KERNEL_REGISTER, Z.STEP_KERNEL_PIPE, Z.STEP_KERNEL_QUAD])
+@pytest.mark.parametrize("world,goff", [(1, 0), (2, 3), (3, 0), (5, 1), (8, 0), (9, 2), (16, 0), (17, 0)])
+def test_stats_every_kernel_and_world(kind, world, goff):
+    """Each statistics kernel forced (where it can run the call; the quad
+    kernel takes N <= 16) on a ragged size, bf16 at odd N: flag and norm
+    against the oracle, then one injected inf in the last replica."""
+    Z.zero_test_force_step_kernel(kind)
+    try:
+        dtype = oracle.BF16 if world % 2 else oracle.F16
+        per_rank = 61_111 + world
+        c = Case(world * per_rank, world, gdtype=dtype, pdtype=dtype, seed=470 + world, goff=goff, scale=65536.0)
+        flag, norm = _stats(c)
+        ovf, sq, _, _ = _oracle_stats(c)
+        assert flag == ovf == 0 and abs(norm - sq) <= _norm_tol(c.n) * sq
+        g = c.G[world - 1].copy()
+        workloads.inject(c.G[world - 1], np.array([c.n - 5]), np.array([True]), dtype)
+        to_dev_u16(c.G[world - 1], TD[dtype], buf=c.g_dev[world - 1])
+        flag, _ = _stats(c)
+        assert flag == 1 == _oracle_stats(c)[0]
+        c.G[world - 1] = g
+    finally:
+        Z.zero_test_force_step_kernel(Z.STEP_KERNEL_AUTO)
 
 
 @pytest.mark.parametrize("mode", ["banks", "inplace", "staged"])

@@ -27,12 +27,16 @@ pytestmark = pytest.mark.gpu
 SMS = 148
 
 
-@pytest.fixture(autouse=True, params=["auto", "pipeline"])
+_KINDS = {"auto": Z.STEP_KERNEL_AUTO, "pipeline": Z.STEP_KERNEL_PIPE, "register": Z.STEP_KERNEL_REGISTER}
+
+
+@pytest.fixture(autouse=True, params=list(_KINDS))
 def kernel_choice(request):
-    """Every case twice: the automatic choice (the statistics and update
-    pipelines take calls of 128 tiles per SM and more, so these sizes run the
-    register kernels) and the pipeline kernels forced wherever they can run."""
-    Z.zero_test_force_step_kernel(Z.STEP_KERNEL_PIPE if request.param == "pipeline" else Z.STEP_KERNEL_AUTO)
+    """Every case three times: the automatic choice (at these sizes the
+    reduce-scatter takes the quad kernel up to N = 16 and the update the
+    register kernel), the pipeline kernels forced wherever they can run, and
+    the register kernels forced."""
+    Z.zero_test_force_step_kernel(_KINDS[request.param])
     try:
         yield request.param
     finally:

@@ -95,6 +95,77 @@ __global__ void __launch_bounds__(kThreads) grad_stats_kernel(const __grid_const
     finish_block<kThreads>(p, bad, sq);
 }
 
+// Quad-streaming statistics kernel for N <= B replicas: thread t sums quads
+// (4 consecutive elements) t, t + T, ..., U of them per iteration, issuing
+// every replica's 8-byte load of those U quads before the first add (plain
+// loads, a grid of several waves), as the quad step kernel does for the
+// fused step.  For calls too short for the pipeline kernel to fill and
+// drain its stages.  kWrite: also store g = s * inv with one 16-byte store
+// per quad.
+template <typename GT, bool kWrite, int B, int U, int NT>
+__global__ void __launch_bounds__(NT, 2) grad_stats_quad_kernel(const __grid_constant__ StepParams p,
+                                                                  float* __restrict__ reduced) {
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * NT + threadIdx.x;
+    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * NT;
+    const int world = p.world;
+    const float inv = p.c.inv;
+    const bool want_sq = p.sqnorm != nullptr;
+    bool bad = false;
+    double sq = 0.0;
+    const int64_t nq = 2 * p.nvec;
+    for (int64_t q0 = tid; q0 < nq; q0 += U * nthreads) {
+        uint2 r[U][B];
+        bool live[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t e0 = p.head + 4 * (q0 + u * nthreads);
+            live[u] = q0 + u * nthreads < nq && !out_of_bounds(e0 + 4 <= p.count, p.overflow);
+            if (!live[u]) continue;
+#pragma unroll
+            for (int k = 0; k < B; ++k)
+                if (k < world) r[u][k] = ld_u2(static_cast<const uint16_t*>(p.grads[k]) + e0);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (!live[u]) continue;
+            const int64_t e0 = p.head + 4 * (q0 + u * nthreads);
+            // rank-order fp32 sum
+            float s0 = Fmt<GT>::lo(r[u][0].x), s1 = Fmt<GT>::hi(r[u][0].x);
+            float s2 = Fmt<GT>::lo(r[u][0].y), s3 = Fmt<GT>::hi(r[u][0].y);
+#pragma unroll
+            for (int k = 1; k < B; ++k) {
+                if (k >= world) break;
+                s0 = __fadd_rn(s0, Fmt<GT>::lo(r[u][k].x));
+                s1 = __fadd_rn(s1, Fmt<GT>::hi(r[u][k].x));
+                s2 = __fadd_rn(s2, Fmt<GT>::lo(r[u][k].y));
+                s3 = __fadd_rn(s3, Fmt<GT>::hi(r[u][k].y));
+            }
+            bad |= !isfinite(s0) | !isfinite(s1) | !isfinite(s2) | !isfinite(s3);
+            const float g0 = __fmul_rn(s0, inv), g1 = __fmul_rn(s1, inv);
+            const float g2 = __fmul_rn(s2, inv), g3 = __fmul_rn(s3, inv);
+            if (want_sq) {
+                sq = fma(static_cast<double>(g0), static_cast<double>(g0), sq);
+                sq = fma(static_cast<double>(g1), static_cast<double>(g1), sq);
+                sq = fma(static_cast<double>(g2), static_cast<double>(g2), sq);
+                sq = fma(static_cast<double>(g3), static_cast<double>(g3), sq);
+            }
+            if constexpr (kWrite) st_state16(reduced + e0, g0, g1, g2, g3);
+        }
+    }
+    stats_scalar_elements<GT, kWrite>(p, reduced, tid, nthreads, bad, sq);
+    finish_block<NT>(p, bad, sq);
+}
+
+// Shapes of the quad statistics kernel by replica count: U quads per thread
+// per iteration (B x U 8-byte loads: 128 bytes in flight per thread at
+// N = B >= 2, 64 at N = 1, where U = 16 would spill), NT threads per block.
+template <int B> struct StatsQuadShape;
+template <> struct StatsQuadShape<1> { static constexpr int U = 8, NT = 512; };
+template <> struct StatsQuadShape<2> { static constexpr int U = 8, NT = 512; };
+template <> struct StatsQuadShape<4> { static constexpr int U = 4, NT = 512; };
+template <> struct StatsQuadShape<8> { static constexpr int U = 2, NT = 512; };
+template <> struct StatsQuadShape<16> { static constexpr int U = 1, NT = 512; };
+
 // Pipeline statistics kernel: the producer warp streams tiles of the N
 // gradient slices into two shared-memory stages with 1-D bulk copies (no
 // multicast, this CTA's own shared memory); 16 consumer warps sum each

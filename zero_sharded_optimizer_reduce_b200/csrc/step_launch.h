@@ -17,6 +17,8 @@ constexpr uint32_t kPipeMinTile = 1536;             // elements: 3/4 of 4 x cons
 constexpr uint32_t kPipeSmemMax = 220u * 1024u;     // dynamic shared memory cap
 constexpr int kPipeMaxWorld = 20;                   // largest N measured to gain from the pipeline
 constexpr int64_t kPipeMinTilesPerSm = 128;         // calls with fewer tiles per SM take the quad kernel
+constexpr int64_t kStatsPipeMinTilesPerSm = 128;    // the same for the staged reduce-scatter
+constexpr int kStatsPipeMaxWorldWrite = 8;          // largest N whose reduce-scatter takes that pipeline
 
 using KernelFn = void (*)(StepParams);
 using StatsKernelFn = void (*)(StepParams, float*);
@@ -59,6 +61,28 @@ inline KernelFn pick_quad_kernel(zero_dtype_t g, zero_dtype_t pd, int world, int
     *nt = QuadShape<16>::NT;
     *u = QuadShape<16>::U;
     return pick_quad_b<16>(g, pd);
+}
+
+template <int B>
+inline StatsKernelFn pick_stats_quad_b(zero_dtype_t g, bool write) {
+    constexpr int U = StatsQuadShape<B>::U, NT = StatsQuadShape<B>::NT;
+    if (write)
+        return g == ZERO_F16 ? grad_stats_quad_kernel<__half, true, B, U, NT>
+                             : grad_stats_quad_kernel<__nv_bfloat16, true, B, U, NT>;
+    return g == ZERO_F16 ? grad_stats_quad_kernel<__half, false, B, U, NT>
+                         : grad_stats_quad_kernel<__nv_bfloat16, false, B, U, NT>;
+}
+
+// The quad statistics kernel for N replicas (N <= kQuadMaxWorld), its threads
+// per block and quads per thread and iteration.
+inline StatsKernelFn pick_stats_quad_kernel(zero_dtype_t g, bool write, int world, int* nt, int* u) {
+    if (world <= 1) { *nt = StatsQuadShape<1>::NT; *u = StatsQuadShape<1>::U; return pick_stats_quad_b<1>(g, write); }
+    if (world <= 2) { *nt = StatsQuadShape<2>::NT; *u = StatsQuadShape<2>::U; return pick_stats_quad_b<2>(g, write); }
+    if (world <= 4) { *nt = StatsQuadShape<4>::NT; *u = StatsQuadShape<4>::U; return pick_stats_quad_b<4>(g, write); }
+    if (world <= 8) { *nt = StatsQuadShape<8>::NT; *u = StatsQuadShape<8>::U; return pick_stats_quad_b<8>(g, write); }
+    *nt = StatsQuadShape<16>::NT;
+    *u = StatsQuadShape<16>::U;
+    return pick_stats_quad_b<16>(g, write);
 }
 
 inline KernelFn pick_pipe_kernel(zero_dtype_t g, zero_dtype_t pd) {
@@ -482,28 +506,64 @@ inline int prepare_stats(const char* fn, const void* const* grad_bufs, int32_t w
         prm.nvec = (count - h) / kVec;
     }
     prm.tile = 0;
-    // pipeline kernel: as for the step, only when every gradient buffer is
-    // this GPU's memory
-    int64_t blocks = 0;
-    const int tile = h >= 0 ? stats_pipe_tile(world) : 0;
-    if (tile > 0) {
-        int sms = 0;
-        if (int rc = stats_pipe_setup(grad_dtype, reduced != nullptr, &sms)) return rc;
-        const int64_t ntiles = (count - h) / tile;
-        // from two tiles per SM (unlike the step and the staged update: with
-        // gradients alone, the register kernel keeps too few bytes in flight
-        // at small N; measured on B200, 16M x N = 4: 0.85 pipeline against
-        // 0.71 register for the reduce-scatter, 64M x N = 8: 1.05 against 1.03)
-        const int force = step_kernel_override();
-        const bool want = force == kKindPipe ? ntiles >= 1
-                                             : force != kKindRegister && ntiles >= 2 * static_cast<int64_t>(sms);
-        if (want && all_local_device_memory(grad_bufs, world)) {
-            prm.tile = tile;
-            prm.nvec = ntiles * tile / kVec;
-            blocks = sms;
-        }
+    prm.kind = kKindRegister;
+    // Kernel choice (measured on B200 against a measured copy rate of
+    // 6.43 TB/s, inputs larger than 4x L2):
+    //  - statistics only (2N bytes per element, all reads): the quad kernel
+    //    for N <= 16 (256M elements, N = 2..16: 0.90-1.14 against 0.64-1.10
+    //    for the pipeline kernel);
+    //  - with the fp32 store of the staged reduce-scatter: the pipeline
+    //    kernel for 3 <= N <= 8 from kStatsPipeMinTilesPerSm tiles per SM when
+    //    every gradient buffer is this GPU's memory (256M, N = 4 / 8: 1.04 /
+    //    1.09 against 1.02 / 1.06), the quad kernel for the rest of N <= 16
+    //    (256M, N = 16: 1.06 against 1.02; 64M, N = 2: 0.93 against 0.85);
+    //  - 17 <= N <= 20: the pipeline kernel from two tiles per SM when the
+    //    gradients are local, else the register kernel; unaligned calls and
+    //    N > 20: the register kernel.
+    // zero_test_force_step_kernel overrides the choice where the forced
+    // kernel can run the call.
+    int sms = 0;
+    {
+        std::lock_guard<std::mutex> lk(g_dev_mu);
+        DeviceInfo* d = nullptr;
+        if (int rc = device_info(&d)) return rc;
+        sms = d->sms;
     }
-    if (prm.tile == 0) {
+    const int force = step_kernel_override();
+    const int tile = h >= 0 ? stats_pipe_tile(world) : 0;
+    const int64_t ntiles = tile > 0 ? (count - h) / tile : 0;
+    const bool vec = prm.nvec > 0;
+    const bool quad_ok = vec && world <= kQuadMaxWorld;
+    const bool pipe_big = reduced != nullptr && world >= 3 && world <= kStatsPipeMaxWorldWrite &&
+                          ntiles >= kStatsPipeMinTilesPerSm * static_cast<int64_t>(sms);
+    int kind = kKindRegister;
+    if (quad_ok && !pipe_big) {
+        kind = kKindQuad;
+    } else if (tile > 0 && ntiles >= 2 * static_cast<int64_t>(sms) && all_local_device_memory(grad_bufs, world)) {
+        kind = kKindPipe;
+    } else if (quad_ok) {
+        kind = kKindQuad;
+    }
+    if (force == kKindRegister) kind = kKindRegister;
+    if (force == kKindQuad && quad_ok) kind = kKindQuad;
+    if (force == kKindPipe && tile > 0 && ntiles >= 1 && all_local_device_memory(grad_bufs, world)) kind = kKindPipe;
+    int64_t blocks = 0;
+    if (kind == kKindPipe) {
+        if (int rc = stats_pipe_setup(grad_dtype, reduced != nullptr, &sms)) return rc;
+        prm.tile = tile;
+        prm.nvec = ntiles * tile / kVec;
+        prm.kind = kKindPipe;
+        blocks = sms;
+    } else if (kind == kKindQuad) {
+        prm.kind = kKindQuad;
+        int nt = 0, u = 0;
+        (void)pick_stats_quad_kernel(grad_dtype, reduced != nullptr, world, &nt, &u);
+        const int64_t per_block = static_cast<int64_t>(nt) * u;
+        blocks = (2 * prm.nvec + per_block - 1) / per_block;
+        const int64_t cap = static_cast<int64_t>(sms) * kQuadBlocksPerSm;
+        if (blocks > cap) blocks = cap;
+        if (blocks < 1) blocks = 1;
+    } else {
         int limit = 0;
         if (int rc = stats_grid_limit(grad_dtype, reduced != nullptr, &limit)) return rc;
         const int64_t work = prm.nvec > 0 ? prm.nvec : count;
@@ -523,9 +583,13 @@ inline int launch_stats(const char* fn, const StepParams& prm, int64_t blocks, z
     if (blocks == 0) return ok();
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool write = reduced != nullptr;
-    if (prm.tile > 0) {
+    if (prm.kind == kKindPipe) {
         pick_stats_pipe_kernel(grad_dtype, write)<<<static_cast<unsigned int>(blocks), kPipeThreads,
                                                     stats_pipe_smem_bytes(prm.world, prm.tile), s>>>(prm, reduced);
+    } else if (prm.kind == kKindQuad) {
+        int nt = 0, u = 0;
+        StatsKernelFn k = pick_stats_quad_kernel(grad_dtype, write, prm.world, &nt, &u);
+        k<<<static_cast<unsigned int>(blocks), nt, 0, s>>>(prm, reduced);
     } else {
         pick_stats_kernel(grad_dtype, write)<<<static_cast<unsigned int>(blocks), kThreads, 0, s>>>(prm, reduced);
     }
