@@ -399,7 +399,8 @@ inline int prepare_step(const char* fn, const void* const* grad_bufs, int32_t wo
         const int64_t per_block = static_cast<int64_t>(nt) * u;
         const int64_t work = prm.nvec > 0 ? 2 * prm.nvec : count;
         blocks = (work + per_block - 1) / per_block;
-        const int64_t cap = static_cast<int64_t>(sms) * kQuadBlocksPerSm;
+        int64_t cap = static_cast<int64_t>(sms) * kQuadBlocksPerSm;
+        if (cap > kMaxBlocks) cap = kMaxBlocks;   // one norm partial per block in the workspace
         if (blocks > cap) blocks = cap;
         if (blocks < 1) blocks = 1;
     } else {
@@ -560,7 +561,8 @@ inline int prepare_stats(const char* fn, const void* const* grad_bufs, int32_t w
         (void)pick_stats_quad_kernel(grad_dtype, reduced != nullptr, world, &nt, &u);
         const int64_t per_block = static_cast<int64_t>(nt) * u;
         blocks = (2 * prm.nvec + per_block - 1) / per_block;
-        const int64_t cap = static_cast<int64_t>(sms) * kQuadBlocksPerSm;
+        int64_t cap = static_cast<int64_t>(sms) * kQuadBlocksPerSm;
+        if (cap > kMaxBlocks) cap = kMaxBlocks;   // one norm partial per block in the workspace
         if (blocks > cap) blocks = cap;
         if (blocks < 1) blocks = 1;
     } else {
