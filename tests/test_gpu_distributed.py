@@ -1,9 +1,10 @@
 """Multi-process ZeRO-2: one process per rank, peers' buffers through CUDA IPC.
 
 Layouts: 2 ranks with buckets padded to a multiple of 8N (every partition
-16-byte aligned; the 3.1M-element bucket takes the pipeline kernel reading
-peers' memory with bulk copies), 3 ranks padded to a multiple of N only
-(partitions off the 16-byte phase: register and scalar paths).
+16-byte aligned: the quad kernel at these sizes; gradient buffers on another
+GPU always take plain loads, since the pipeline kernel's bulk copies read only
+this GPU's memory), 3 ranks padded to a multiple of N only (partitions off the
+16-byte phase: register and scalar paths).
 
 2 and 3 ranks run as separate processes (on the one GPU of this machine, each
 with its own context; host barriers over gloo order them, no kernel waits on

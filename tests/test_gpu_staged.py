@@ -88,7 +88,7 @@ CASES = [
     (4, 4 * 20_011, oracle.F16, -1, 3, 0),
     (4, 4 * 20_011, oracle.F16, -1, 0, 1),
     (64, 64 * 4099, oracle.F16, -1, 0, 0),
-    # >= 2 x 148 update tiles of 6144: the update's pipeline kernel
+    # about 4 update tiles of 4096 per SM: the update's pipeline kernel when forced
     (4, 4 * 600_007, oracle.F16, -1, 0, 0),
     (2, 2 * 1_000_003, oracle.BF16, -1, 0, 0),
     (2, 2 * 1_900_003, oracle.F16, 1, 0, 0),

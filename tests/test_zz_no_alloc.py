@@ -10,9 +10,11 @@ libzero instead.  The GPU test calls it through the C ABI twice in a row (the
 second call reuses the scratch the first one left behind) and checks every
 output against the regular entry point (same tolerance as the other parity
 tests, and in fact bit for bit, the norm included) and against the oracle.
-The cases reach both step kernels: the register kernel (a ragged size) and
-the shared-memory pipeline kernel (at least two tiles per SM), plus a call on
-a single partition.
+The cases reach all three step kernels, each forced with
+zero_test_force_step_kernel on both entry points: the register kernel and the
+quad kernel (the automatic choice at this size) on a ragged size, the
+shared-memory pipeline kernel on at least two tiles per SM; plus a call on a
+single partition with the automatic choice.
 
 The file is named so that pytest collects it last.
 """
@@ -71,13 +73,23 @@ def _run(entry, grads, state_in, t, padded, partition, count, use_ws):
     return out, params, int(flag.item()), float(norm.item())
 
 
+@pytest.fixture
+def kernel_kind(request):
+    Z.zero_test_force_step_kernel(request.param)
+    try:
+        yield request.param
+    finally:
+        Z.zero_test_force_step_kernel(Z.STEP_KERNEL_AUTO)
+
+
 @pytest.mark.gpu
-@pytest.mark.parametrize("world,padded,partition", [
-    (8, 8 * 100_003 + 8, Z.ZERO_ALL_PARTITIONS),              # register kernel, ragged vector tail
-    (8, 8 * (2 * 148 * 3072 + 1000), Z.ZERO_ALL_PARTITIONS),  # pipeline kernel: >= 2 tiles of 3072 per SM
-    (8, 8 * 100_003 + 8, 3),                                   # one rank's partition
-])
-def test_noalloc_matches_regular_entry_and_oracle_on_two_calls_in_a_row(world, padded, partition):
+@pytest.mark.parametrize("world,padded,partition,kernel_kind", [
+    (8, 8 * 100_003 + 8, Z.ZERO_ALL_PARTITIONS, Z.STEP_KERNEL_REGISTER),   # ragged vector tail
+    (8, 8 * 100_003 + 8, Z.ZERO_ALL_PARTITIONS, Z.STEP_KERNEL_QUAD),
+    (8, 8 * (2 * 148 * 3072 + 1000), Z.ZERO_ALL_PARTITIONS, Z.STEP_KERNEL_PIPE),  # >= 2 tiles of 3072 per SM
+    (8, 8 * 100_003 + 8, 3, Z.STEP_KERNEL_AUTO),                             # one rank's partition
+], indirect=["kernel_kind"])
+def test_noalloc_matches_regular_entry_and_oracle_on_two_calls_in_a_row(world, padded, partition, kernel_kind):
     P = padded // world
     begin = 0 if partition < 0 else partition * P
     count = padded if partition < 0 else P
