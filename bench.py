@@ -493,7 +493,7 @@ def run_gpu(args):
                    else None)
     if kinds:
         names = {Z.STEP_KERNEL_REGISTER: "register-streaming", Z.STEP_KERNEL_PIPE: "shared-memory pipeline",
-                 Z.STEP_KERNEL_QUAD: "quad-streaming"}
+                 Z.STEP_KERNEL_QUAD: "quad-streaming", Z.STEP_KERNEL_OCT: "oct-streaming"}
         fused_label = "fused_step per bucket: " + ", ".join(
             f"{kinds.count(k)} x {names[k]} kernel" for k in sorted(set(kinds)))
     else:
@@ -564,6 +564,29 @@ def run_sweep(args):
     import zero_sharded_optimizer_reduce_b200 as Z
     torch.cuda.set_device(0)
     peak, peak_kind = peaks()
+    # this box's own copy rate, for reference beside the fixed peak: a
+    # device-to-device copy of 4 GiB (8 GiB moved), timed like the points
+    src = torch.empty(4 << 30, dtype=torch.uint8, device="cuda").fill_(1)
+    dst = torch.empty_like(src)
+    ctimes = []
+    for i in range(23):
+        torch.cuda._sleep(200_000)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        dst.copy_(src)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            ctimes.append(e0.elapsed_time(e1))
+    copy_gbs = 2 * src.numel() / (statistics.median(ctimes) * 1e-3) / 1e9
+    del src, dst
+    torch.cuda.empty_cache()
+    print(json.dumps({"sweep": True, "copy_reference": True, "bytes_moved": 2 * (4 << 30), "reps": 20,
+                      "gbs": copy_gbs, "what": "torch copy_ of a 4 GiB device buffer (a device-to-device "
+                                               "cudaMemcpy): this box's copy rate, median of 20"}), flush=True)
+    names = {Z.STEP_KERNEL_REGISTER: "register", Z.STEP_KERNEL_PIPE: "pipeline", Z.STEP_KERNEL_QUAD: "quad",
+             Z.STEP_KERNEL_OCT: "oct"}
     free_gb = torch.cuda.mem_get_info()[0] / 1e9
     flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
     dtypes = [args.grad_dtype] if args.sweep_dtype_only else ["f16", "bf16"]
@@ -616,9 +639,13 @@ def run_sweep(args):
             assert int(opt.flag.item()) == 0
             ms = statistics.median(times)
             gbs = psi * bpe / (ms * 1e-3) / 1e9
-            print(json.dumps({"sweep": True, "psi": psi, "world": N, "grad_dtype": dt,
+            # the runner of this one-bucket optimizer prepares the same call
+            # (bank 0 -> 1), so it names the kernel the timed calls ran
+            kind = opt.bucket_kernels()[0]
+            print(json.dumps({"sweep": True, "psi": psi, "world": N, "grad_dtype": dt, "kernel": names[kind],
                               "kernel_ms_median": ms, "reps": reps, "gparams_s": psi / (ms * 1e-3) / 1e9, "gbs": gbs,
-                              "frac_measured": gbs / peak, "frac_nominal_8tbs": gbs / 8000.0,
+                              "frac_measured": gbs / peak, "frac_copy_this_run": gbs / copy_gbs,
+                              "frac_nominal_8tbs": gbs / 8000.0,
                               "l2": "L2-influenced (footprint < 4x L2, flushed between steps)" if small
                               else "footprint > 4x L2"}), flush=True)
             del opt

@@ -389,15 +389,17 @@ def test_staged_runner_rejects_bad_arguments():
 
 
 def test_step_kernel_hook_validates_and_resets():
-    """zero_test_force_step_kernel: host only, -1..2 accepted, anything else
+    """zero_test_force_step_kernel: host only, -1..3 accepted, anything else
     ZERO_ERR_ARG; the binding's names match the C values."""
     L = Z.lib
-    for kind in (Z.STEP_KERNEL_REGISTER, Z.STEP_KERNEL_PIPE, Z.STEP_KERNEL_QUAD, Z.STEP_KERNEL_AUTO):
+    for kind in (Z.STEP_KERNEL_REGISTER, Z.STEP_KERNEL_PIPE, Z.STEP_KERNEL_QUAD, Z.STEP_KERNEL_OCT,
+                 Z.STEP_KERNEL_AUTO):
         assert L.zero_test_force_step_kernel(kind) == 0
-    assert L.zero_test_force_step_kernel(3) == -1
+    assert L.zero_test_force_step_kernel(4) == -1
     assert L.zero_test_force_step_kernel(-2) == -1
     assert b"kind" in L.zero_last_error()
-    assert (Z.STEP_KERNEL_AUTO, Z.STEP_KERNEL_REGISTER, Z.STEP_KERNEL_PIPE, Z.STEP_KERNEL_QUAD) == (-1, 0, 1, 2)
+    assert (Z.STEP_KERNEL_AUTO, Z.STEP_KERNEL_REGISTER, Z.STEP_KERNEL_PIPE, Z.STEP_KERNEL_QUAD,
+            Z.STEP_KERNEL_OCT) == (-1, 0, 1, 2, 3)
     Z.zero_test_force_step_kernel(Z.STEP_KERNEL_AUTO)
 
 

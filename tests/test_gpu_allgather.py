@@ -1,16 +1,18 @@
 """All-gather reconstruct (zero_allgather_params) against the oracle's gather.
 
-The copy takes one of three routes by the slices' alignment: whole 16-byte
-blocks through the bulk-copy kernel when source and destination share their
-16-byte phase, realigned blocks through the register kernel when they do not,
-and element copies for the sub-16-byte edges.  These cases pin every route
-bit for bit (ZeRO explainer, "Stage 3 - Parameter Partitioning (P_os+g+p)":
-the gathered layer is exactly the concatenation of the ranks' slices):
+The copy kernel writes whole 32-byte aligned destination blocks; each is two
+aligned 16-byte source blocks when source and destination share their 16-byte
+phase, or three realigned ones when they do not, and the edges before the
+first and after the last whole block are copied element by element.  These
+cases pin every route bit for bit (ZeRO explainer, "Stage 3 - Parameter
+Partitioning (P_os+g+p)": the gathered layer is exactly the concatenation of
+the ranks' slices):
 
-- every pair of source and destination element phases, at sizes below, at and
-  above one block, so that each realignment shift, head and tail occurs;
-- slices large enough that every CTA of the bulk kernel takes several chunks
-  and chunks end at slice boundaries;
+- every source element phase below 16 bytes against every destination phase
+  below 32 bytes, at sizes below, at and above one block, so that each
+  realignment shift, head and tail occurs;
+- slices large enough that every block of the grid takes several iterations
+  and the iterations end at slice boundaries;
 - a Stage-1/2 gather of an odd partition size (every rank but the first off
   the destination's phase), scaled past L2;
 - guard bytes around the destination and a status word that stays 0.
@@ -69,22 +71,23 @@ def _gather_and_check(dev, host, offset, part, dtype, dst_elem_offset=0):
 @pytest.mark.parametrize("dtype", [torch.float16, torch.float32])
 @pytest.mark.parametrize("part", [1, 7, 8, 9, 130, 3001])
 def test_every_phase_pair(dtype, part):
-    """Source slice at element offset a, destination at element offset b, for
-    every a, b below 16 bytes: all realignment shifts, heads and tails."""
+    """Source slice at element offset a (below 16 bytes), destination at
+    element offset b (below 32 bytes): all realignment shifts, heads and
+    tails."""
     es = torch.empty((), dtype=dtype).element_size()
-    phases = 16 // es
-    for a in range(phases):
+    for a in range(16 // es):
         dev, host, keep = _shards(3, a + part + 5, dtype, seed=100 * part + a)
-        for b in range(phases):
+        for b in range(32 // es):
             _gather_and_check(dev, host, a, part, dtype, dst_elem_offset=b)
 
 
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("world,part,src_off,dst_off", [
-    (8, 3_000_000, 0, 0),          # aligned: bulk kernel, several chunks per CTA
-    (8, 3_000_003, 0, 0),          # ranks off the phase: realigned register kernel
+    (8, 3_000_000, 0, 0),          # aligned: several iterations per thread
+    (8, 3_000_000, 0, 8),          # 16-byte phase shared, 32-byte heads of 16 bytes (fp16)
+    (8, 3_000_003, 0, 0),          # ranks off the phase: realigned blocks
     (5, 1_234_567, 3, 1),          # everything off the phase, odd world
-    (2, 49_152, 0, 0),             # chunk boundaries at slice ends
+    (2, 49_152, 0, 0),             # iterations ending at slice ends
     (16, 65_536 + 8, 8, 0),        # aligned with a shard offset
 ])
 def test_large_gathers(dtype, world, part, src_off, dst_off):

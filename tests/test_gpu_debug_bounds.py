@@ -46,7 +46,8 @@ def _pipe_T(world):
     return min(8192, (180 * 1024 // (2 * (2 * world + 12))) // 512 * 512)
 
 
-@pytest.mark.parametrize("kind", [Z.STEP_KERNEL_AUTO, Z.STEP_KERNEL_REGISTER, Z.STEP_KERNEL_PIPE, Z.STEP_KERNEL_QUAD])
+@pytest.mark.parametrize("kind", [Z.STEP_KERNEL_AUTO, Z.STEP_KERNEL_REGISTER, Z.STEP_KERNEL_PIPE, Z.STEP_KERNEL_QUAD,
+                                  Z.STEP_KERNEL_OCT])
 @pytest.mark.parametrize("world,padded,part,offs", [
     (3, 3 * 50_001, -1, (0, 0, 0)),                                  # ragged
     (4, 4 * 20_011, -1, (3, 5, 1)),                                  # scalar path (phases differ)
@@ -120,6 +121,8 @@ def test_broadcast_update_in_bounds():
     (4, 250_001, 0, 0),          # ranks 1-3 realigned (odd partition)
     (5, 123_457, 3, 1),          # everything off the phase, heads and tails
     (3, 5, 1, 2),                # slices shorter than one 16-byte block
+    (8, 300_000, 0, 8),          # 16-byte phase shared, destinations 16 bytes off 32 (fp16)
+    (3, 13, 0, 3),               # slices between one 16- and one 32-byte block
 ])
 def test_allgather_in_bounds(dtype, world, part, src_off, dst_off):
     """Both copy kernels (phase-matched and realigned) with their element

@@ -20,11 +20,14 @@ from test_gpu_step import Case, _adam
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture
-def quad():
-    Z.zero_test_force_step_kernel(Z.STEP_KERNEL_QUAD)
+@pytest.fixture(params=["quad", "oct"])
+def quad(request):
+    """The quad kernel, then the oct kernel (8 elements per thread, 32-byte
+    state stores; it runs where the fp32 outputs are 32-byte aligned at the
+    vector region, elsewhere the call keeps its automatic choice)."""
+    Z.zero_test_force_step_kernel(Z.STEP_KERNEL_QUAD if request.param == "quad" else Z.STEP_KERNEL_OCT)
     try:
-        yield
+        yield request.param
     finally:
         Z.zero_test_force_step_kernel(Z.STEP_KERNEL_AUTO)
 
@@ -91,19 +94,21 @@ def test_automatic_choice_mid_size(world):
 def test_runner_reports_the_kernel_choice():
     """zero_runner_bucket_kernel names the kernel the next launch runs: the
     pipeline kernel for a 64M-element bucket at N = 8 (147 tiles per SM), the
-    quad kernel for a 1M-element bucket, the register kernel above N = 20,
-    and whatever the override forces."""
+    oct kernel for a 1M-element bucket (the optimizer's buffers are 32-byte
+    aligned), the register kernel above N = 20, and whatever the override
+    forces."""
     from zero_sharded_optimizer_reduce_b200.optimizer import ZeroAdam
     opt = ZeroAdam([64 << 20, 1 << 20], world=8, bucket_elems=64 << 20)
     assert opt.layout.n_buckets == 2
-    assert opt.bucket_kernels() == [Z.STEP_KERNEL_PIPE, Z.STEP_KERNEL_QUAD]
-    Z.zero_test_force_step_kernel(Z.STEP_KERNEL_REGISTER)
-    try:
-        assert opt.bucket_kernels() == [Z.STEP_KERNEL_REGISTER, Z.STEP_KERNEL_REGISTER]
-    finally:
-        Z.zero_test_force_step_kernel(Z.STEP_KERNEL_AUTO)
+    assert opt.bucket_kernels() == [Z.STEP_KERNEL_PIPE, Z.STEP_KERNEL_OCT]
+    for kind in (Z.STEP_KERNEL_REGISTER, Z.STEP_KERNEL_QUAD):
+        Z.zero_test_force_step_kernel(kind)
+        try:
+            assert opt.bucket_kernels() == [kind, kind]
+        finally:
+            Z.zero_test_force_step_kernel(Z.STEP_KERNEL_AUTO)
     del opt
     assert ZeroAdam([240_000], world=24).bucket_kernels() == [Z.STEP_KERNEL_REGISTER]
-    assert ZeroAdam([240_000], world=2).bucket_kernels() == [Z.STEP_KERNEL_QUAD]
+    assert ZeroAdam([240_000], world=2).bucket_kernels() == [Z.STEP_KERNEL_OCT]
     assert ZeroAdam([240_000], world=4, mode="staged").bucket_kernels() is None
     torch.cuda.empty_cache()

@@ -530,7 +530,7 @@ class Runner:
 
     def bucket_kernel(self, bucket: int) -> int:
         """The fused-step kernel the next launch runs for `bucket`:
-        STEP_KERNEL_REGISTER, STEP_KERNEL_PIPE or STEP_KERNEL_QUAD."""
+        STEP_KERNEL_REGISTER, STEP_KERNEL_PIPE, STEP_KERNEL_QUAD or STEP_KERNEL_OCT."""
         kind = ctypes.c_int32()
         _check(lib.zero_runner_bucket_kernel(self._h, bucket, ctypes.byref(kind)))
         return kind.value
@@ -551,7 +551,7 @@ def zero_test_wait_timeout(status, limit_ns: int, stream=None) -> None:
     _check(lib.zero_test_wait_timeout(_dev(status, 1, "status", torch.int32), int(limit_ns), _stream(stream)))
 
 
-STEP_KERNEL_AUTO, STEP_KERNEL_REGISTER, STEP_KERNEL_PIPE, STEP_KERNEL_QUAD = -1, 0, 1, 2
+STEP_KERNEL_AUTO, STEP_KERNEL_REGISTER, STEP_KERNEL_PIPE, STEP_KERNEL_QUAD, STEP_KERNEL_OCT = -1, 0, 1, 2, 3
 
 
 def zero_test_force_step_kernel(kind: int) -> None:

@@ -10,22 +10,25 @@
 //
 // One kernel, two bodies.  The grid is (blocks per segment) x (segments):
 // every segment is copied by its own column of blocks at the same time, each
-// thread moving several aligned 16-byte destination blocks per iteration with
-// plain loads and stores (no streaming or L1 no-allocate hints: on B200 they
-// cost 3-17 % in this copy), with a grid of several waves.
-//  - source and destination share their 16-byte
-//    phase (the usual case: every slice of a Stage-3 unit, every bucket whose
-//    partition is a multiple of 8 elements): 8 blocks per thread in flight;
-//  - the phases differ (an odd partition size puts
-//    every rank but the first off its destination's phase): each thread loads
-//    the two aligned source blocks that its destination block straddles (the
-//    second is the next thread's first, read again from L1) and realigns them
-//    with funnel shifts, so loads and stores stay 16-byte and coalesced.
-// The sub-16-byte edges of each segment (before its first aligned
-// destination byte, after its last whole block) are copied element by
-// element by the segment's first block.  A source block read this way always
-// holds at least one byte of the segment, so it never reaches a page the
-// segment does not touch; bytes outside the segment are never written.
+// thread moving several aligned 32-byte destination blocks per iteration with
+// plain 16-byte loads and one 32-byte store per block (no streaming or L1
+// no-allocate hints: on B200 they cost 3-17 % in this copy), with a grid of
+// several waves.  The store width is what sets the rate of a 1:1 copy: on
+// B200, 16-byte stores reach 0.96 of a device-to-device cudaMemcpy and 32-byte
+// stores 0.99-1.00, whatever the load width.
+//  - source and destination share their 16-byte phase (the usual case: every
+//    slice of a Stage-3 unit, every bucket whose partition is a multiple of 8
+//    elements): each destination block is two aligned source blocks;
+//  - the phases differ (an odd partition size puts every rank but the first
+//    off its destination's phase): each thread loads the three aligned
+//    source blocks that its destination block straddles (the third is the
+//    next thread's first, read again from L1) and realigns them with funnel
+//    shifts, so loads and stores stay aligned and coalesced.
+// The edges of each segment (before its first 32-byte aligned destination
+// byte, after its last whole block) are copied element by element by the
+// segment's first block.  A source block read this way always holds at least
+// one byte of the segment, so it never reaches a page the segment does not
+// touch; bytes outside the segment are never written.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -41,12 +44,11 @@ namespace {
 
 constexpr int kMaxSegs = 64;          // segments per launch
 constexpr int kCopyThreads = 256;
-// Destination blocks per thread per iteration, and blocks of the whole grid
-// per SM (several waves), for the phase-matched and the realigning body.
-// Measured on B200 (8 x 25M fp16 slices, L2 flushed): 0.995 and 0.980 of the
-// measured B200 copy rate (6.43 TB/s); 512-thread blocks, other depths and
-// one-wave grids 0.91-0.98.
-constexpr int kKMatched = 8, kKShifted = 4;
+constexpr int kBlk = 32;              // bytes per destination block (one 32-byte store)
+// Destination blocks per thread per iteration (128 and 64 bytes stored), and
+// blocks of the whole grid per SM (several waves), for the phase-matched and
+// the realigning body.
+constexpr int kKMatched = 4, kKShifted = 2;
 constexpr int kBlocksPerSmMatched = 64, kBlocksPerSmShifted = 32;
 constexpr int32_t kStatusBounds = 4;  // debug builds: an index check failed, access skipped
 
@@ -71,8 +73,8 @@ struct CopySeg {
     char* dst;            // first destination byte
     const char* src_al;   // aligned source block holding the byte copied to dst + head
     int64_t bytes;        // segment length
-    int64_t head;         // bytes before the first 16-byte aligned destination byte
-    int64_t nblk;         // whole aligned 16-byte destination blocks after the head
+    int64_t head;         // bytes before the first 32-byte aligned destination byte
+    int64_t nblk;         // whole aligned 32-byte destination blocks after the head
     int32_t shift;        // (src + head) - src_al; 0 when the 16-byte phases agree
 };
 
@@ -83,7 +85,13 @@ struct CopyParams {
 };
 
 __device__ __forceinline__ uint4 ld16(const char* p) { return *reinterpret_cast<const uint4*>(p); }
-__device__ __forceinline__ void st16(char* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
+
+// One 32-byte store (a 32-byte aligned address): lo then hi.
+__device__ __forceinline__ void st32(char* p, const uint4& lo, const uint4& hi) {
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(lo.x), "r"(lo.y), "r"(lo.z),
+                 "r"(lo.w), "r"(hi.x), "r"(hi.y), "r"(hi.z), "r"(hi.w)
+                 : "memory");
+}
 
 // Bytes [4Q + sh/8, 4Q + sh/8 + 16) of the 32-byte concatenation a:b.
 template <int Q>
@@ -122,55 +130,65 @@ __global__ void __launch_bounds__(kCopyThreads) copy_grid_kernel(const __grid_co
     const int es = p.esize;
     if (blockIdx.x == 0) {
         for (int64_t i = threadIdx.x; i < sg.head / es; i += kCopyThreads) copy_elem(sg, i * es, es, p.status);
-        const int64_t tail0 = sg.head + 16 * sg.nblk;
+        const int64_t tail0 = sg.head + kBlk * sg.nblk;
         for (int64_t i = threadIdx.x; i < (sg.bytes - tail0) / es; i += kCopyThreads)
             copy_elem(sg, tail0 + i * es, es, p.status);
     }
     char* const dst_al = sg.dst + sg.head;
     const int64_t n = sg.nblk;
     const int64_t nt = static_cast<int64_t>(gridDim.x) * kCopyThreads;
+    const int64_t body = sg.bytes - sg.head;   // bytes from the first aligned destination byte
     int64_t i = static_cast<int64_t>(blockIdx.x) * kCopyThreads + threadIdx.x;
     if (sg.shift == 0) {
         constexpr int kCopyK = kKMatched;
         for (; i + (kCopyK - 1) * nt < n; i += kCopyK * nt) {
-            uint4 r[kCopyK];
-#pragma unroll
-            for (int k = 0; k < kCopyK; ++k) r[k] = ld16(sg.src_al + 16 * (i + k * nt));
+            uint4 r[kCopyK][2];
 #pragma unroll
             for (int k = 0; k < kCopyK; ++k) {
-                if (out_of_bounds(16 * (i + k * nt) + 16 <= sg.bytes - sg.head, p.status)) continue;
-                st16(dst_al + 16 * (i + k * nt), r[k]);
+                const char* s0 = sg.src_al + kBlk * (i + k * nt);
+                r[k][0] = ld16(s0);
+                r[k][1] = ld16(s0 + 16);
+            }
+#pragma unroll
+            for (int k = 0; k < kCopyK; ++k) {
+                if (out_of_bounds(kBlk * (i + k * nt) + kBlk <= body, p.status)) continue;
+                st32(dst_al + kBlk * (i + k * nt), r[k][0], r[k][1]);
             }
         }
         for (; i < n; i += nt) {
-            if (out_of_bounds(16 * i + 16 <= sg.bytes - sg.head, p.status)) continue;
-            st16(dst_al + 16 * i, ld16(sg.src_al + 16 * i));
+            if (out_of_bounds(kBlk * i + kBlk <= body, p.status)) continue;
+            const char* s0 = sg.src_al + kBlk * i;
+            st32(dst_al + kBlk * i, ld16(s0), ld16(s0 + 16));
         }
     } else {
-        // destination block j straddles source blocks j and j + 1; the last one
-        // needed is block n, which still holds segment bytes (shift > 0)
+        // destination block j straddles source blocks 2j, 2j + 1 and 2j + 2;
+        // the last one needed, 2n, still holds segment bytes (shift > 0)
         constexpr int kCopyK = kKShifted;
         const int shift = sg.shift;
         for (; i + (kCopyK - 1) * nt < n; i += kCopyK * nt) {
-            uint4 a[kCopyK], b[kCopyK];
+            uint4 a[kCopyK], b[kCopyK], c[kCopyK];
 #pragma unroll
             for (int k = 0; k < kCopyK; ++k) {
-                const char* s0 = sg.src_al + 16 * (i + k * nt);
-                a[k] = out_of_bounds(src_block_ok(sg, s0), p.status) ? make_uint4(0u, 0u, 0u, 0u) : ld16(s0);
-                b[k] = out_of_bounds(src_block_ok(sg, s0 + 16), p.status) ? make_uint4(0u, 0u, 0u, 0u) : ld16(s0 + 16);
+                const char* s0 = sg.src_al + kBlk * (i + k * nt);
+                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                a[k] = out_of_bounds(src_block_ok(sg, s0), p.status) ? z : ld16(s0);
+                b[k] = out_of_bounds(src_block_ok(sg, s0 + 16), p.status) ? z : ld16(s0 + 16);
+                c[k] = out_of_bounds(src_block_ok(sg, s0 + 32), p.status) ? z : ld16(s0 + 32);
             }
 #pragma unroll
             for (int k = 0; k < kCopyK; ++k) {
-                if (out_of_bounds(16 * (i + k * nt) + 16 <= sg.bytes - sg.head, p.status)) continue;
-                st16(dst_al + 16 * (i + k * nt), realign_rt(a[k], b[k], shift));
+                if (out_of_bounds(kBlk * (i + k * nt) + kBlk <= body, p.status)) continue;
+                st32(dst_al + kBlk * (i + k * nt), realign_rt(a[k], b[k], shift), realign_rt(b[k], c[k], shift));
             }
         }
         for (; i < n; i += nt) {
-            const char* s0 = sg.src_al + 16 * i;
-            if (out_of_bounds(src_block_ok(sg, s0) && src_block_ok(sg, s0 + 16) && 16 * i + 16 <= sg.bytes - sg.head,
+            const char* s0 = sg.src_al + kBlk * i;
+            if (out_of_bounds(src_block_ok(sg, s0) && src_block_ok(sg, s0 + 16) && src_block_ok(sg, s0 + 32) &&
+                                  kBlk * i + kBlk <= body,
                               p.status))
                 continue;
-            st16(dst_al + 16 * i, realign_rt(ld16(s0), ld16(s0 + 16), shift));
+            const uint4 b = ld16(s0 + 16);
+            st32(dst_al + kBlk * i, realign_rt(ld16(s0), b, shift), realign_rt(b, ld16(s0 + 32), shift));
         }
     }
 }
@@ -205,9 +223,9 @@ CopySeg make_seg(const Seg& g) {
     r.src = g.src;
     r.dst = g.dst;
     r.bytes = g.bytes;
-    r.head = static_cast<int64_t>((16u - (reinterpret_cast<uintptr_t>(g.dst) & 15u)) & 15u);
+    r.head = static_cast<int64_t>((32u - (reinterpret_cast<uintptr_t>(g.dst) & 31u)) & 31u);
     if (r.head > g.bytes) r.head = g.bytes;
-    r.nblk = (g.bytes - r.head) / 16;
+    r.nblk = (g.bytes - r.head) / kBlk;
     const uintptr_t a = reinterpret_cast<uintptr_t>(g.src + r.head);
     r.src_al = reinterpret_cast<const char*>(a & ~static_cast<uintptr_t>(15));
     r.shift = r.nblk > 0 ? static_cast<int32_t>(a & 15u) : 0;

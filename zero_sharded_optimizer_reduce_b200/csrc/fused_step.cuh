@@ -39,6 +39,7 @@ struct Consts {
 constexpr int32_t kKindRegister = 0;  // fused_step_kernel: 8 elements per thread
 constexpr int32_t kKindPipe = 1;      // fused_step_pipe_kernel: bulk-copy tiles through shared memory
 constexpr int32_t kKindQuad = 2;      // fused_step_quad_kernel: 4 elements per thread, plain loads (N <= 16)
+constexpr int32_t kKindOct = 3;       // fused_step_oct_kernel: 8 elements per thread, 32-byte state stores
 
 struct StepParams {
     const void* grads[ZERO_MAX_WORLD];  // already offset to the call's first element
@@ -47,7 +48,8 @@ struct StepParams {
     int64_t head;   // elements [0, head) take the scalar path
     int64_t nvec;   // vectors of kVec elements starting at `head`
     int32_t tile;   // elements per pipeline tile (pipeline kernels only)
-    int32_t kind;   // which step kernel the host launches: kKindRegister / kKindPipe / kKindQuad
+    int32_t kind;   // which step kernel the host launches: kKindRegister / kKindPipe / kKindQuad / kKindOct
+    int32_t st32;   // 1: the fp32 outputs are 32-byte aligned at `head` (32-byte state stores)
     const float* master_in;
     const float* m_in;
     const float* v_in;
@@ -88,6 +90,15 @@ __device__ __forceinline__ float4 ld_state16(const float* p) {
 
 __device__ __forceinline__ void st_state16(float* p, float a, float b, float c, float d) {
     asm volatile("st.global.v4.f32 [%0], {%1,%2,%3,%4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
+// One 32-byte store of 8 fp32 values (a 32-byte aligned address).  On B200
+// the store width sets the rate of write-heavy streams: a 1:1 copy with
+// 32-byte stores runs 3-4 % faster than with 16-byte stores.
+__device__ __forceinline__ void st_state32(float* p, const float* w) {
+    asm volatile("st.global.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "f"(w[0]), "f"(w[1]), "f"(w[2]),
+                 "f"(w[3]), "f"(w[4]), "f"(w[5]), "f"(w[6]), "f"(w[7])
                  : "memory");
 }
 
@@ -424,6 +435,68 @@ __global__ void __launch_bounds__(NT, NT >= 512 ? 2 : 3) fused_step_quad_kernel(
     scalar_elements<GT, PT>(p, c, tid, nthreads, bad, sq);
     finish_block<NT>(p, bad, sq);
 }
+
+// Oct-streaming kernel for N <= B replicas: thread t updates octs (8
+// consecutive elements) t, t + T, ..., issuing every load of an oct (N
+// 16-byte gradient loads, 6 16-byte state loads) before using any, then one
+// 32-byte store per state array and one 16-byte parameter store; a grid of
+// several waves.  It needs the fp32 outputs 32-byte aligned at the vector
+// region's start (StepParams::st32, set by the host).
+template <typename GT, typename PT, int B, int NT, int MINB>
+__global__ void __launch_bounds__(NT, MINB) fused_step_oct_kernel(const __grid_constant__ StepParams p) {
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * NT + threadIdx.x;
+    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * NT;
+    const int world = p.world;
+    Consts c = p.c;
+    if (!step_prologue(p, c)) return;
+    bool bad = false;
+    double sq = 0.0;
+    for (int64_t vi = tid; vi < p.nvec; vi += nthreads) {
+        const int64_t e0 = p.head + vi * kVec;
+        if (out_of_bounds(e0 + kVec <= p.count, p.overflow)) continue;
+        uint4 r[B];
+#pragma unroll
+        for (int k = 0; k < B; ++k)
+            if (k < world) r[k] = ld_grad16(static_cast<const uint16_t*>(p.grads[k]) + e0);
+        const float4 p0 = ld_f4(p.master_in + e0), p1 = ld_f4(p.master_in + e0 + 4);
+        const float4 m0 = ld_f4(p.m_in + e0), m1 = ld_f4(p.m_in + e0 + 4);
+        const float4 v0 = ld_f4(p.v_in + e0), v1 = ld_f4(p.v_in + e0 + 4);
+        // rank-order fp32 sum
+        float s[kVec];
+        cvt8<GT>(r[0], s);
+#pragma unroll
+        for (int k = 1; k < B; ++k)
+            if (k < world) add8<GT>(r[k], s);
+        float pw[kVec] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+        float mw[kVec] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+        float vw[kVec] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+        for (int e = 0; e < kVec; ++e) {
+            bad |= !isfinite(s[e]);
+            const float g = adam(s[e], pw[e], mw[e], vw[e], c);
+            if (p.sqnorm) sq = fma(static_cast<double>(g), static_cast<double>(g), sq);
+        }
+        st_state32(p.master_out + e0, pw);
+        st_state32(p.m_out + e0, mw);
+        st_state32(p.v_out + e0, vw);
+        uint4 q;
+        q.x = Fmt<PT>::pack(pw[0], pw[1]);
+        q.y = Fmt<PT>::pack(pw[2], pw[3]);
+        q.z = Fmt<PT>::pack(pw[4], pw[5]);
+        q.w = Fmt<PT>::pack(pw[6], pw[7]);
+        st_u16x8(static_cast<uint16_t*>(p.param_out) + e0, q);
+    }
+    scalar_elements<GT, PT>(p, c, tid, nthreads, bad, sq);
+    finish_block<NT>(p, bad, sq);
+}
+
+// Shapes of the oct kernel by replica count: NT threads per block and the
+// blocks per SM its registers are sized for (no spills).
+template <int B> struct OctShape;
+template <> struct OctShape<2> { static constexpr int NT = 512, MINB = 2; };
+template <> struct OctShape<4> { static constexpr int NT = 256, MINB = 3; };
+template <> struct OctShape<8> { static constexpr int NT = 256, MINB = 2; };
+template <> struct OctShape<16> { static constexpr int NT = 256, MINB = 2; };
 
 // Shapes of the quad kernel by replica count: B replicas' loads and U quads
 // in flight per thread, NT threads per block (two or three blocks per SM at

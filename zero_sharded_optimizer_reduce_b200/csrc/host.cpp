@@ -39,7 +39,7 @@ extern "C" {
 const char* zero_last_error(void) { return zero::g_last_error; }
 
 int zero_test_force_step_kernel(int32_t kind) {
-    if (kind < -1 || kind > 2) return fail(ZERO_ERR_ARG, "zero_test_force_step_kernel: kind %d outside -1..2", kind);
+    if (kind < -1 || kind > 3) return fail(ZERO_ERR_ARG, "zero_test_force_step_kernel: kind %d outside -1..3", kind);
     zero::g_step_kernel_override.store(kind, std::memory_order_relaxed);
     return zero::ok();
 }

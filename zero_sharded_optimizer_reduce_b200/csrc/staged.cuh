@@ -81,12 +81,18 @@ __global__ void __launch_bounds__(kThreads) adam_reduced_kernel(const __grid_con
         float vw[kVec] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
         for (int e = 0; e < kVec; ++e) adam(g[e], pw[e], mw[e], vw[e], c);
-        st_state16(p.master_out + e0, pw[0], pw[1], pw[2], pw[3]);
-        st_state16(p.master_out + e0 + 4, pw[4], pw[5], pw[6], pw[7]);
-        st_state16(p.m_out + e0, mw[0], mw[1], mw[2], mw[3]);
-        st_state16(p.m_out + e0 + 4, mw[4], mw[5], mw[6], mw[7]);
-        st_state16(p.v_out + e0, vw[0], vw[1], vw[2], vw[3]);
-        st_state16(p.v_out + e0 + 4, vw[4], vw[5], vw[6], vw[7]);
+        if (p.st32) {   // uniform over the grid
+            st_state32(p.master_out + e0, pw);
+            st_state32(p.m_out + e0, mw);
+            st_state32(p.v_out + e0, vw);
+        } else {
+            st_state16(p.master_out + e0, pw[0], pw[1], pw[2], pw[3]);
+            st_state16(p.master_out + e0 + 4, pw[4], pw[5], pw[6], pw[7]);
+            st_state16(p.m_out + e0, mw[0], mw[1], mw[2], mw[3]);
+            st_state16(p.m_out + e0 + 4, mw[4], mw[5], mw[6], mw[7]);
+            st_state16(p.v_out + e0, vw[0], vw[1], vw[2], vw[3]);
+            st_state16(p.v_out + e0 + 4, vw[4], vw[5], vw[6], vw[7]);
+        }
         uint4 q;
         q.x = Fmt<PT>::pack(pw[0], pw[1]);
         q.y = Fmt<PT>::pack(pw[2], pw[3]);

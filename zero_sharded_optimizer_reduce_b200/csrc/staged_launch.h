@@ -138,18 +138,27 @@ inline int prepare_reduced(const char* fn, const float* reduced, int64_t count, 
         prm.head = h;
         prm.nvec = (count - h) / kVec;
     }
+    // 32-byte state stores when the fp32 outputs are 32-byte aligned at head
+    prm.st32 = 0;
+    if (prm.nvec > 0) {
+        bool al = true;
+        for (const float* a : {master_out, m_out, v_out})
+            al = al && ((reinterpret_cast<uintptr_t>(a) + 4 * static_cast<uintptr_t>(h)) % 32) == 0;
+        prm.st32 = al ? 1 : 0;
+    }
     prm.tile = 0;
     *prm_out = prm;
     *work_out = prm.nvec > 0 ? prm.nvec : count;
     return ZERO_OK;
 }
 
-// Enqueue the update prepared by prepare_reduced: the pipeline kernel when
-// the aligned part gives every SM at least kPipeMinTilesPerSm tiles, else
-// the register kernel (plain loads, a grid of kRegWaves waves).  Measured on
-// B200 (fp32 reduced gradients in, 30 bytes per element): 16M elements 0.93
-// register against 0.88 pipeline, 64M 0.98 against 0.96, 256M both 0.97-0.98
-// of a measured B200 copy rate (6.43 TB/s).  `work` as returned by prepare_reduced (> 0).
+// Enqueue the update prepared by prepare_reduced: the register kernel (plain
+// loads, 32-byte state stores where the outputs allow them, a grid of
+// kRegWaves waves); the pipeline kernel only when zero_test_force_step_kernel
+// asks for it.  Measured on B200 (fp32 reduced gradients in, 30 bytes per
+// element, against a measured copy rate of 6.43 TB/s): 16M elements 0.93-0.96
+// register against 0.87 pipeline, 64M 0.99 against 0.95, 256M-492M
+// 0.99 against 0.98.  `work` as returned by prepare_reduced (> 0).
 inline int launch_reduced(const char* fn, StepParams prm, const ParamDsts& d, int64_t work, zero_dtype_t pd,
                           bool bcast, zero_stream_t stream) {
     ReducedDevice* dev = nullptr;
@@ -157,9 +166,7 @@ inline int launch_reduced(const char* fn, StepParams prm, const ParamDsts& d, in
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int64_t ntiles = prm.nvec > 0 ? (prm.count - prm.head) / kReducedTile : 0;
     const int force = step_kernel_override();
-    const bool pipe = force == kKindPipe ? ntiles >= 1
-                                         : force != kKindRegister &&
-                                               ntiles >= kPipeMinTilesPerSm * static_cast<int64_t>(dev->sms);
+    const bool pipe = force == kKindPipe && ntiles >= 1;
     if (pipe) {
         // the pipeline kernel takes the whole tiles; the rest goes through
         // its scalar path

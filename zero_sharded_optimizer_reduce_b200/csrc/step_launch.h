@@ -16,7 +16,8 @@ constexpr uint32_t kPipeSmemTarget = 180u * 1024u;  // shared memory of both sta
 constexpr uint32_t kPipeMinTile = 1536;             // elements: 3/4 of 4 x consumer threads
 constexpr uint32_t kPipeSmemMax = 220u * 1024u;     // dynamic shared memory cap
 constexpr int kPipeMaxWorld = 20;                   // largest N measured to gain from the pipeline
-constexpr int64_t kPipeMinTilesPerSm = 128;         // calls with fewer tiles per SM take the quad kernel
+constexpr int64_t kPipeMinTilesPerSm = 128;         // calls with fewer tiles per SM take the oct / quad kernel
+constexpr int kOctMaxWorldAtAnySize = 4;            // N up to this takes the oct kernel at every size
 constexpr int64_t kStatsPipeMinTilesPerSm = 128;    // the same for the staged reduce-scatter
 constexpr int kStatsPipeMaxWorldWrite = 8;          // largest N whose reduce-scatter takes that pipeline
 
@@ -83,6 +84,25 @@ inline StatsKernelFn pick_stats_quad_kernel(zero_dtype_t g, bool write, int worl
     *nt = StatsQuadShape<16>::NT;
     *u = StatsQuadShape<16>::U;
     return pick_stats_quad_b<16>(g, write);
+}
+
+template <int B>
+inline KernelFn pick_oct_b(zero_dtype_t g, zero_dtype_t pd) {
+    constexpr int NT = OctShape<B>::NT, M = OctShape<B>::MINB;
+    if (g == ZERO_F16 && pd == ZERO_F16) return fused_step_oct_kernel<__half, __half, B, NT, M>;
+    if (g == ZERO_F16 && pd == ZERO_BF16) return fused_step_oct_kernel<__half, __nv_bfloat16, B, NT, M>;
+    if (g == ZERO_BF16 && pd == ZERO_F16) return fused_step_oct_kernel<__nv_bfloat16, __half, B, NT, M>;
+    return fused_step_oct_kernel<__nv_bfloat16, __nv_bfloat16, B, NT, M>;
+}
+
+// The oct-kernel instance for N replicas (N <= kQuadMaxWorld) and its threads
+// per block.
+inline KernelFn pick_oct_kernel(zero_dtype_t g, zero_dtype_t pd, int world, int* nt) {
+    if (world <= 2) { *nt = OctShape<2>::NT; return pick_oct_b<2>(g, pd); }
+    if (world <= 4) { *nt = OctShape<4>::NT; return pick_oct_b<4>(g, pd); }
+    if (world <= 8) { *nt = OctShape<8>::NT; return pick_oct_b<8>(g, pd); }
+    *nt = OctShape<16>::NT;
+    return pick_oct_b<16>(g, pd);
 }
 
 inline KernelFn pick_pipe_kernel(zero_dtype_t g, zero_dtype_t pd) {
@@ -343,18 +363,33 @@ inline int prepare_step(const char* fn, const void* const* grad_bufs, int32_t wo
     }
     prm.tile = 0;
     prm.kind = kKindRegister;
+    // 32-byte state stores need the fp32 outputs 32-byte aligned where the
+    // vector region starts
+    prm.st32 = 0;
+    if (prm.nvec > 0) {
+        bool al = true;
+        for (const float* a : {master_out, m_out, v_out})
+            al = al && ((reinterpret_cast<uintptr_t>(a) + 4 * static_cast<uintptr_t>(h)) % 32) == 0;
+        prm.st32 = al ? 1 : 0;
+    }
 
-    // Kernel choice (measured on B200 against the copy rate, L2 cold):
+    // Kernel choice (measured on B200 against a measured copy rate of
+    // 6.43 TB/s, L2 cold):
     //  - arrays whose 16-byte phases never coincide, or N > kPipeMaxWorld: the
     //    register kernel (its scalar path when unaligned; at N = 64 it runs at
     //    the copy rate);
-    //  - N >= 3 with at least kPipeMinTilesPerSm tiles per SM and every
-    //    gradient buffer in this GPU's memory: the pipeline kernel (its bulk
-    //    copies never read another GPU's memory; 1.05 of the copy rate at
-    //    N = 4..16, 1B elements, against 0.99-1.05 for the quad kernel);
-    //  - N <= 16 otherwise: the quad kernel (N <= 2, where half of the bytes
-    //    are writes: 0.98 against 0.97; 16M elements at N = 1..16: 0.95-1.06
-    //    against 0.84-1.03, no pipeline to fill and drain; peer memory);
+    //  - N <= 16 streams: the oct kernel when the fp32 outputs are 32-byte
+    //    aligned at the vector region (its 32-byte stores: N = 1 / 2 at 256M
+    //    and 1B elements 1.00-1.02 against 0.98-0.99 for the quad kernel;
+    //    N = 4 at 256M 1.01 against 0.99 for the pipeline), else the quad
+    //    kernel; they take N <= kOctMaxWorldAtAnySize (2 for the quad kernel)
+    //    at every size, calls below kPipeMinTilesPerSm tiles per SM (no
+    //    pipeline to fill and drain: 16M elements at N = 1..16, 0.97-1.04
+    //    against 0.82-1.04) and gradients in another GPU's memory;
+    //  - otherwise, with every gradient buffer in this GPU's memory, the
+    //    pipeline kernel (its bulk copies never read another GPU's memory;
+    //    N = 8 / 16 at 256M: 1.05 / 1.09-1.10 against 1.04 / 1.08 for the oct
+    //    kernel);
     //  - 17 <= N <= 20 calls below the pipeline threshold: the pipeline kernel
     //    when the gradients are local and every SM gets two tiles, else the
     //    register kernel.
@@ -375,18 +410,30 @@ inline int prepare_step(const char* fn, const void* const* grad_bufs, int32_t wo
     if (h >= 0 && world <= kPipeMaxWorld) {
         const bool quad_ok = world <= kQuadMaxWorld;
         const bool big = ntiles >= kPipeMinTilesPerSm * static_cast<int64_t>(sms);
-        if (quad_ok && (world <= 2 || !big)) {
-            kind = kKindQuad;
+        const int stream_kind = prm.st32 ? kKindOct : kKindQuad;
+        const bool small_n = world <= (prm.st32 ? kOctMaxWorldAtAnySize : 2);
+        if (quad_ok && (small_n || !big)) {
+            kind = stream_kind;
         } else if (all_local_device_memory(grad_bufs, world)) {   // queried only where it decides
             if (big || ntiles >= 2 * static_cast<int64_t>(sms)) kind = kKindPipe;
         } else if (quad_ok) {
-            kind = kKindQuad;
+            kind = stream_kind;
         }
     }
     if (force == kKindRegister) kind = kKindRegister;
     if (force == kKindQuad && h >= 0 && world <= kQuadMaxWorld) kind = kKindQuad;
     if (force == kKindPipe && tile > 0 && ntiles >= 1 && all_local_device_memory(grad_bufs, world)) kind = kKindPipe;
-    if (kind == kKindPipe) {
+    if (force == kKindOct && h >= 0 && world <= kQuadMaxWorld && prm.st32) kind = kKindOct;
+    if (kind == kKindOct) {
+        prm.kind = kKindOct;
+        int nt = 0;
+        (void)pick_oct_kernel(grad_dtype, param_dtype, world, &nt);
+        blocks = (prm.nvec + nt - 1) / nt;
+        int64_t cap = static_cast<int64_t>(sms) * kQuadBlocksPerSm;
+        if (cap > kMaxBlocks) cap = kMaxBlocks;   // one norm partial per block in the workspace
+        if (blocks > cap) blocks = cap;
+        if (blocks < 1) blocks = 1;
+    } else if (kind == kKindPipe) {
         if (int rc = pipe_setup(grad_dtype, param_dtype, &sms)) return rc;
         prm.tile = tile;
         prm.nvec = ntiles * tile / kVec;
@@ -628,6 +675,10 @@ inline int launch_step(const char* fn, const StepParams& prm, int64_t blocks, ze
     } else if (prm.kind == kKindQuad) {
         int nt = 0, u = 0;
         KernelFn k = pick_quad_kernel(grad_dtype, param_dtype, prm.world, &nt, &u);
+        k<<<static_cast<unsigned int>(blocks), nt, 0, s>>>(prm);
+    } else if (prm.kind == kKindOct) {
+        int nt = 0;
+        KernelFn k = pick_oct_kernel(grad_dtype, param_dtype, prm.world, &nt);
         k<<<static_cast<unsigned int>(blocks), nt, 0, s>>>(prm);
     } else {
         pick_kernel(grad_dtype, param_dtype)<<<static_cast<unsigned int>(blocks), kThreads, 0, s>>>(prm);
