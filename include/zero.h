@@ -475,18 +475,21 @@ int zero_test_wait_timeout(int32_t* status, int64_t limit_ns, zero_stream_t stre
  *
  * The paper has no counterpart: a test hook of this library.  Every fused
  * step call (zero_reduce_scatter_adam_step, its gated and no-alloc variants,
- * the runner) normally picks one of three kernels that compute the same bits:
- * the shared-memory pipeline kernel for large calls with N >= 3, the
- * quad-streaming kernel for N <= 2, mid-size calls and peer memory, the
+ * the runner) normally picks one of four kernels that compute the same bits:
+ * the shared-memory pipeline kernel for large calls with N >= 5, the
+ * oct-streaming kernel (32-byte state stores) for N <= 4, mid-size calls and
+ * peer memory when the fp32 outputs are 32-byte aligned where the vector
+ * region starts, the quad-streaming kernel for those calls otherwise, the
  * register kernel for N > 20 or arrays off a common 16-byte phase.  This call
  * makes the process's later calls take `kind` instead wherever that kernel
  * can run the call (the pipeline kernel needs a common phase, N <= 20, one
  * whole tile and gradients in this GPU's memory; the quad kernel a common
- * phase and N <= 16), so that tests reach each kernel at small sizes.  The
- * statistics pass, the staged reduce-scatter and the staged update follow it
- * too: 1 forces their pipeline kernels, 0 their register kernels (2 leaves
- * their automatic choice).
- * kind  -1 automatic (the default), 0 register, 1 pipeline, 2 quad
+ * phase and N <= 16; the oct kernel that and the 32-byte alignment), so that
+ * tests reach each kernel at small sizes.  The statistics pass, the staged
+ * reduce-scatter and the staged update follow it too: 1 forces their
+ * pipeline kernels, 0 their register kernels, 2 the statistics' quad kernel
+ * (3 leaves their automatic choice).
+ * kind  -1 automatic (the default), 0 register, 1 pipeline, 2 quad, 3 oct
  * Errors: ZERO_ERR_ARG.  Host only, no CUDA call.
  */
 int zero_test_force_step_kernel(int32_t kind);
@@ -589,7 +592,8 @@ void zero_runner_destroy(zero_runner_t* runner);
  * zero_runner_bucket_kernel - which fused-step kernel the next
  * zero_runner_launch runs for bucket `bucket` of a two-bank runner: 0 the
  * register-streaming kernel, 1 the shared-memory pipeline kernel, 2 the
- * quad-streaming kernel (the numbering of zero_test_force_step_kernel).  It
+ * quad-streaming kernel, 3 the oct-streaming kernel (the numbering of
+ * zero_test_force_step_kernel).  It
  * makes the launch's own preparation (bank cur, the current t and loss
  * scale, the kernel override in force) without enqueueing anything; the
  * choice depends on the bucket's size, N, the buffers' 16-byte phase and
