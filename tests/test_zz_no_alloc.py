@@ -10,11 +10,11 @@ libzero instead.  The GPU test calls it through the C ABI twice in a row (the
 second call reuses the scratch the first one left behind) and checks every
 output against the regular entry point (same tolerance as the other parity
 tests, and in fact bit for bit, the norm included) and against the oracle.
-The cases reach all three step kernels, each forced with
-zero_test_force_step_kernel on both entry points: the register kernel and the
-quad kernel (the automatic choice at this size) on a ragged size, the
-shared-memory pipeline kernel on at least two tiles per SM; plus a call on a
-single partition with the automatic choice.
+The cases reach all four step kernels, each forced with
+zero_test_force_step_kernel on both entry points: the register, quad and oct
+kernels (the oct kernel is the automatic choice at this size) on a ragged
+size, the shared-memory pipeline kernel on at least two tiles per SM; plus a
+call on a single partition with the automatic choice.
 
 The file is named so that pytest collects it last.
 """
@@ -86,6 +86,7 @@ def kernel_kind(request):
 @pytest.mark.parametrize("world,padded,partition,kernel_kind", [
     (8, 8 * 100_003 + 8, Z.ZERO_ALL_PARTITIONS, Z.STEP_KERNEL_REGISTER),   # ragged vector tail
     (8, 8 * 100_003 + 8, Z.ZERO_ALL_PARTITIONS, Z.STEP_KERNEL_QUAD),
+    (8, 8 * 100_003 + 8, Z.ZERO_ALL_PARTITIONS, Z.STEP_KERNEL_OCT),     # the automatic choice at this size
     (8, 8 * (2 * 148 * 3072 + 1000), Z.ZERO_ALL_PARTITIONS, Z.STEP_KERNEL_PIPE),  # >= 2 tiles of 3072 per SM
     (8, 8 * 100_003 + 8, 3, Z.STEP_KERNEL_AUTO),                             # one rank's partition
 ], indirect=["kernel_kind"])
