@@ -680,12 +680,19 @@ def run_stage3(args):
         for _ in range(args.warmup):
             s3.step()
         torch.cuda.synchronize()
+        # ncu --profile-from-start off captures the timed steps of the value's
+        # configuration (no prefetch, staged update) only
+        headline = not prefetch and update == "staged"
+        if headline:
+            torch.cuda.profiler.start()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(args.steps):
             s3.step()
         e1.record()
         torch.cuda.synchronize()
+        if headline:
+            torch.cuda.profiler.stop()
         out[(prefetch, update)] = e0.elapsed_time(e1) / args.steps
         if prefetch and update == "staged":
             # the all-gather alone: unit 0 from the 8 shards into a layer buffer
