@@ -23,15 +23,22 @@ def test_layout_matches_oracle(numels, world, cap, align):
     assert list(a.tensor_bucket) == b.tensor_bucket and list(a.tensor_offset) == b.tensor_offset
 
 
+KINDS = [-1, 0, 1, 2, 3]   # automatic, register, pipeline, quad, oct (zero_test_force_step_kernel)
+
+
 @pytest.mark.gpu
-@settings(max_examples=40, deadline=None, derandomize=True)
+@settings(max_examples=80, deadline=None, derandomize=True)
 @given(world=st.integers(1, 17), per_rank=st.integers(1, 5000),
        dtypes=st.sampled_from([(oracle.F16, oracle.F16), (oracle.BF16, oracle.BF16), (oracle.F16, oracle.BF16),
                                (oracle.BF16, oracle.F16)]),
        offs=st.tuples(st.integers(0, 7), st.integers(0, 7), st.integers(0, 7)),
        part=st.integers(-1, 16), inplace=st.booleans(), wd=st.sampled_from([0.0, 0.01, 0.1]),
-       t=st.integers(1, 50), seed=st.integers(0, 10_000))
-def test_step_matches_oracle(world, per_rank, dtypes, offs, part, inplace, wd, t, seed):
+       t=st.integers(1, 50), seed=st.integers(0, 10_000), kind=st.sampled_from(KINDS))
+def test_step_matches_oracle(world, per_rank, dtypes, offs, part, inplace, wd, t, seed, kind):
+    """Random sizes, offsets (state offsets of 0-7 fp32 elements put the
+    outputs on and off a 32-byte boundary), partitions, dtypes and a forced
+    kernel (it runs where it can, else the automatic choice)."""
+    import zero_sharded_optimizer_reduce_b200 as Z
     from test_gpu_step import Case
     gd, pd = dtypes
     partition = part if part < world else -1
@@ -39,7 +46,11 @@ def test_step_matches_oracle(world, per_rank, dtypes, offs, part, inplace, wd, t
              soff=offs[1], poff=offs[2], inplace=inplace)
     adam = workloads.AdamConfig(weight_decay=wd)
     ref, ovf, _ = c.expect(adam, t=t)
-    c.run(adam, t=t)
+    Z.zero_test_force_step_kernel(kind)
+    try:
+        c.run(adam, t=t)
+    finally:
+        Z.zero_test_force_step_kernel(Z.STEP_KERNEL_AUTO)
     assert int(c.flag.item()) == ovf == 0
     assert c.compare(ref) == [0, 0, 0, 0]
 
@@ -50,8 +61,9 @@ def test_step_matches_oracle(world, per_rank, dtypes, offs, part, inplace, wd, t
        dtypes=st.sampled_from([(oracle.F16, oracle.F16), (oracle.BF16, oracle.BF16), (oracle.F16, oracle.BF16)]),
        offs=st.tuples(st.integers(0, 7), st.integers(0, 7), st.integers(0, 7), st.integers(0, 7)),
        part=st.integers(-1, 16), inplace=st.booleans(), wd=st.sampled_from([0.0, 0.01]),
-       t=st.integers(1, 50), seed=st.integers(0, 10_000))
-def test_staged_step_matches_oracle(world, per_rank, dtypes, offs, part, inplace, wd, t, seed):
+       t=st.integers(1, 50), seed=st.integers(0, 10_000), kind=st.sampled_from(KINDS[:4]))
+def test_staged_step_matches_oracle(world, per_rank, dtypes, offs, part, inplace, wd, t, seed, kind):
+    import zero_sharded_optimizer_reduce_b200 as Z
     from test_gpu_staged import Staged
     gd, pd = dtypes
     partition = part if part < world else -1
@@ -59,10 +71,14 @@ def test_staged_step_matches_oracle(world, per_rank, dtypes, offs, part, inplace
                soff=offs[1], poff=offs[2], roff=offs[3], inplace=inplace, scale=1024.0)
     adam = workloads.AdamConfig(weight_decay=wd)
     ref, ovf, _ = c.expect(adam, t=t)
-    c.reduce_scatter()
-    s, inv, g = c.oracle_reduced()
-    assert np.array_equal(host_reduced(c), g.view(np.uint32))
-    c.update(adam, t=t, gate=c.flag)
+    Z.zero_test_force_step_kernel(kind)
+    try:
+        c.reduce_scatter()
+        s, inv, g = c.oracle_reduced()
+        assert np.array_equal(host_reduced(c), g.view(np.uint32))
+        c.update(adam, t=t, gate=c.flag)
+    finally:
+        Z.zero_test_force_step_kernel(Z.STEP_KERNEL_AUTO)
     assert int(c.flag.item()) == ovf == 0
     assert c.compare(ref) == [0, 0, 0, 0]
 
