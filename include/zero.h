@@ -487,8 +487,9 @@ int zero_test_wait_timeout(int32_t* status, int64_t limit_ns, zero_stream_t stre
  * phase and N <= 16; the oct kernel that and the 32-byte alignment), so that
  * tests reach each kernel at small sizes.  The statistics pass, the staged
  * reduce-scatter and the staged update follow it too: 1 forces their
- * pipeline kernels, 0 their register kernels, 2 the statistics' quad kernel
- * (3 leaves their automatic choice).
+ * pipeline kernels, 0 their register kernels, 2 the statistics' quad kernel,
+ * 3 the reduce-scatter's oct kernel (N <= 2, `reduced` 32-byte aligned; the
+ * staged update keeps its automatic choice).
  * kind  -1 automatic (the default), 0 register, 1 pipeline, 2 quad, 3 oct
  * Errors: ZERO_ERR_ARG.  Host only, no CUDA call.
  */

@@ -72,9 +72,9 @@ def test_fused_step_in_bounds(world, padded, part, offs, kind):
 
 
 @pytest.mark.parametrize("kind", [Z.STEP_KERNEL_AUTO, Z.STEP_KERNEL_REGISTER, Z.STEP_KERNEL_PIPE,
-                                  Z.STEP_KERNEL_QUAD])
+                                  Z.STEP_KERNEL_QUAD, Z.STEP_KERNEL_OCT])
 @pytest.mark.parametrize("world,padded,part", [(8, 8 * 250_003, -1), (16, 16 * 60_001, -1), (3, 3 * 7_001, 2),
-                                                (2, 2 * 1_900_003, 1)])
+                                                (2, 2 * 1_900_003, 1), (1, 1_000_003, -1)])
 def test_staged_route_and_statistics_in_bounds(world, padded, part, kind):
     Z.zero_test_force_step_kernel(kind)
     try:

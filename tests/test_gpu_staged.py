@@ -27,15 +27,17 @@ pytestmark = pytest.mark.gpu
 SMS = 148
 
 
-_KINDS = {"auto": Z.STEP_KERNEL_AUTO, "pipeline": Z.STEP_KERNEL_PIPE, "register": Z.STEP_KERNEL_REGISTER}
+_KINDS = {"auto": Z.STEP_KERNEL_AUTO, "pipeline": Z.STEP_KERNEL_PIPE, "register": Z.STEP_KERNEL_REGISTER,
+          "quad": Z.STEP_KERNEL_QUAD}
 
 
 @pytest.fixture(autouse=True, params=list(_KINDS))
 def kernel_choice(request):
-    """Every case three times: the automatic choice (at these sizes the
-    reduce-scatter takes the quad kernel up to N = 16 and the update the
-    register kernel), the pipeline kernels forced wherever they can run, and
-    the register kernels forced."""
+    """Every case four times: the automatic choice (at these sizes the
+    reduce-scatter takes the oct kernel at N <= 2 with `reduced` 32-byte
+    aligned, else the quad kernel up to N = 16, and the update the register
+    kernel), the pipeline kernels forced wherever they can run, the register
+    kernels forced, and the quad reduce-scatter forced."""
     Z.zero_test_force_step_kernel(_KINDS[request.param])
     try:
         yield request.param

@@ -166,6 +166,60 @@ template <> struct StatsQuadShape<4> { static constexpr int U = 4, NT = 512; };
 template <> struct StatsQuadShape<8> { static constexpr int U = 2, NT = 512; };
 template <> struct StatsQuadShape<16> { static constexpr int U = 1, NT = 512; };
 
+// Oct-streaming staged reduce-scatter for N <= B replicas (B = 1, 2: the
+// write-heavy cases, 4 bytes written per 2N read): thread t reduces octs (8
+// consecutive elements) t, t + T, ..., U of them per iteration, every
+// replica's 16-byte load of those U octs issued before the first add, then
+// one 32-byte store of the 8 unscaled gradients per oct.  Needs `reduced`
+// 32-byte aligned at the vector region's start (the host checks).
+template <typename GT, int B, int U, int NT>
+__global__ void __launch_bounds__(NT, 2) grad_rs_oct_kernel(const __grid_constant__ StepParams p,
+                                                           float* __restrict__ reduced) {
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * NT + threadIdx.x;
+    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * NT;
+    const int world = p.world;
+    const float inv = p.c.inv;
+    const bool want_sq = p.sqnorm != nullptr;
+    bool bad = false;
+    double sq = 0.0;
+    for (int64_t v0 = tid; v0 < p.nvec; v0 += U * nthreads) {
+        uint4 r[U][B];
+        bool live[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t e0 = p.head + kVec * (v0 + u * nthreads);
+            live[u] = v0 + u * nthreads < p.nvec && !out_of_bounds(e0 + kVec <= p.count, p.overflow);
+            if (!live[u]) continue;
+#pragma unroll
+            for (int k = 0; k < B; ++k)
+                if (k < world) r[u][k] = ld_grad16(static_cast<const uint16_t*>(p.grads[k]) + e0);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (!live[u]) continue;
+            const int64_t e0 = p.head + kVec * (v0 + u * nthreads);
+            float g[kVec];
+            cvt8<GT>(r[u][0], g);   // rank-order fp32 sum
+#pragma unroll
+            for (int k = 1; k < B; ++k)
+                if (k < world) add8<GT>(r[u][k], g);
+#pragma unroll
+            for (int e = 0; e < kVec; ++e) {
+                bad |= !isfinite(g[e]);
+                g[e] = __fmul_rn(g[e], inv);
+                if (want_sq) sq = fma(static_cast<double>(g[e]), static_cast<double>(g[e]), sq);
+            }
+            st_state32(reduced + e0, g);
+        }
+    }
+    stats_scalar_elements<GT, true>(p, reduced, tid, nthreads, bad, sq);
+    finish_block<NT>(p, bad, sq);
+}
+
+template <int B> struct RsOctShape;
+template <> struct RsOctShape<1> { static constexpr int U = 4, NT = 512; };
+template <> struct RsOctShape<2> { static constexpr int U = 4, NT = 512; };
+
 // Pipeline statistics kernel: the producer warp streams tiles of the N
 // gradient slices into two shared-memory stages with 1-D bulk copies (no
 // multicast, this CTA's own shared memory); 16 consumer warps sum each

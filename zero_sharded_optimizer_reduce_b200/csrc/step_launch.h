@@ -105,6 +105,21 @@ inline KernelFn pick_oct_kernel(zero_dtype_t g, zero_dtype_t pd, int world, int*
     return pick_oct_b<16>(g, pd);
 }
 
+// The oct reduce-scatter for N <= 2, its threads per block and octs per
+// thread and iteration.
+inline StatsKernelFn pick_rs_oct_kernel(zero_dtype_t g, int world, int* nt, int* u) {
+    if (world <= 1) {
+        *nt = RsOctShape<1>::NT;
+        *u = RsOctShape<1>::U;
+        return g == ZERO_F16 ? grad_rs_oct_kernel<__half, 1, RsOctShape<1>::U, RsOctShape<1>::NT>
+                             : grad_rs_oct_kernel<__nv_bfloat16, 1, RsOctShape<1>::U, RsOctShape<1>::NT>;
+    }
+    *nt = RsOctShape<2>::NT;
+    *u = RsOctShape<2>::U;
+    return g == ZERO_F16 ? grad_rs_oct_kernel<__half, 2, RsOctShape<2>::U, RsOctShape<2>::NT>
+                         : grad_rs_oct_kernel<__nv_bfloat16, 2, RsOctShape<2>::U, RsOctShape<2>::NT>;
+}
+
 inline KernelFn pick_pipe_kernel(zero_dtype_t g, zero_dtype_t pd) {
     if (g == ZERO_F16 && pd == ZERO_F16) return fused_step_pipe_kernel<__half, __half>;
     if (g == ZERO_F16 && pd == ZERO_BF16) return fused_step_pipe_kernel<__half, __nv_bfloat16>;
@@ -592,11 +607,27 @@ inline int prepare_stats(const char* fn, const void* const* grad_bufs, int32_t w
     } else if (quad_ok) {
         kind = kKindQuad;
     }
+    // the write-heavy reduce-scatter at N <= 2: 32-byte stores of the reduced
+    // gradients (the oct version) where `reduced` is 32-byte aligned at h
+    const bool rs_oct_ok = quad_ok && reduced != nullptr && world <= 2 &&
+                           ((reinterpret_cast<uintptr_t>(reduced) + 4 * static_cast<uintptr_t>(h)) % 32) == 0;
+    if (kind == kKindQuad && rs_oct_ok) kind = kKindOct;
     if (force == kKindRegister) kind = kKindRegister;
     if (force == kKindQuad && quad_ok) kind = kKindQuad;
+    if (force == kKindOct && rs_oct_ok) kind = kKindOct;
     if (force == kKindPipe && tile > 0 && ntiles >= 1 && all_local_device_memory(grad_bufs, world)) kind = kKindPipe;
     int64_t blocks = 0;
-    if (kind == kKindPipe) {
+    if (kind == kKindOct) {
+        prm.kind = kKindOct;
+        int nt = 0, u = 0;
+        (void)pick_rs_oct_kernel(grad_dtype, world, &nt, &u);
+        const int64_t per_block = static_cast<int64_t>(nt) * u;
+        blocks = (prm.nvec + per_block - 1) / per_block;
+        int64_t cap = static_cast<int64_t>(sms) * kQuadBlocksPerSm;
+        if (cap > kMaxBlocks) cap = kMaxBlocks;   // one norm partial per block in the workspace
+        if (blocks > cap) blocks = cap;
+        if (blocks < 1) blocks = 1;
+    } else if (kind == kKindPipe) {
         if (int rc = stats_pipe_setup(grad_dtype, reduced != nullptr, &sms)) return rc;
         prm.tile = tile;
         prm.nvec = ntiles * tile / kVec;
@@ -638,6 +669,10 @@ inline int launch_stats(const char* fn, const StepParams& prm, int64_t blocks, z
     } else if (prm.kind == kKindQuad) {
         int nt = 0, u = 0;
         StatsKernelFn k = pick_stats_quad_kernel(grad_dtype, write, prm.world, &nt, &u);
+        k<<<static_cast<unsigned int>(blocks), nt, 0, s>>>(prm, reduced);
+    } else if (prm.kind == kKindOct) {
+        int nt = 0, u = 0;
+        StatsKernelFn k = pick_rs_oct_kernel(grad_dtype, prm.world, &nt, &u);
         k<<<static_cast<unsigned int>(blocks), nt, 0, s>>>(prm, reduced);
     } else {
         pick_stats_kernel(grad_dtype, write)<<<static_cast<unsigned int>(blocks), kThreads, 0, s>>>(prm, reduced);
