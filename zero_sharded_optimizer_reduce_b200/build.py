@@ -29,7 +29,7 @@ LIB_DEBUG = os.path.join(PKG, "libzero_debug.so")
 
 SOURCES = ["step.cu", "step_static.cu", "stats.cu", "staged.cu", "selftest.cu", "runner.cu", "copy.cu", "host.cpp",
            "ipc.cpp"]
-HEADERS = [os.path.join(CSRC, n) for n in ("common.h", "fused_step.cuh", "grad_stats.cuh", "staged.cuh",
+HEADERS = [os.path.join(CSRC, n) for n in ("bulk.cuh", "common.h", "fused_step.cuh", "grad_stats.cuh", "staged.cuh",
                                                         "staged_launch.h", "step_launch.h")] + [os.path.join(INCLUDE, "zero.h")]
 
 NVCC_FLAGS = [
