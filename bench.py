@@ -254,8 +254,7 @@ def cpu_baseline(w: workloads.Workload, sample_elems: int, min_seconds: float = 
 
 
 def run_cpu_configs(args):
-    """The oracle timed on every workload the way the survey's measurement
-    plan asks: the full arrays of the tiny and the dynamic-loss-scale
+    """The oracle timed on every workload: the full arrays of the tiny and the dynamic-loss-scale
     workloads, 64M-element slices of the GPT-2 1.5B bucket, of one 6.7B unit
     and of the sweep's flat buffers (N = 1, 8, 16 and 64), each on every host
     core and on one thread.  One JSON line; no GPU is used."""
