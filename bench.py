@@ -92,15 +92,19 @@ PASSES = {"banks": "single fused pass", "inplace": "statistics pass (2N B/elem) 
 # ----------------------------------------------------------------- helpers
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+    """nvidia-smi clocks / throttle reasons sampled during the timed region.
+    With keep_samples, stop() also returns every sample as (unix time, SM MHz,
+    reasons), for attributing clocks to sub-intervals."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,timestamp")
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, keep_samples: bool = False):
         self.dev = device_index
         self.proc = None
         self.path = None
+        self.keep = keep_samples
+        self.samples = []
 
     def start(self):
         try:
@@ -123,28 +127,45 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.fh.close()
-        sm, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
             lines = f.readlines()
-        for line in lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = max(mx, float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
         os.unlink(self.path)
-        if not sm:
-            return None
-        under_load = [x for x in sm if x >= 0.5 * max(sm)] or sm
-        return {"sm_mhz": statistics.median(under_load), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        summary, samples = parse_clock_csv(lines)
+        if self.keep:
+            self.samples = samples
+        return summary
+
+
+def parse_clock_csv(lines):
+    """nvidia-smi lines of ClockSampler.Q -> (summary, samples): the median SM
+    clock under load, the largest max clock, the throttle reasons seen; and
+    every sample as (unix time, SM MHz, reasons) when it has a timestamp."""
+    import datetime
+    sm, mx, reasons, samples = [], 0.0, set(), []
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for line in lines:
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            clk = float(parts[1])
+            mx = max(mx, float(parts[2]))
+        except ValueError:
+            continue
+        sm.append(clk)
+        here = [n for n, v in zip(names, parts[5:9]) if v.lower() == "active"]
+        reasons.update(here)
+        if len(parts) >= 10:
+            try:
+                ts = datetime.datetime.strptime(parts[9], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                samples.append((ts, clk, here))
+            except ValueError:
+                pass
+    if not sm:
+        return None, samples
+    under_load = [x for x in sm if x >= 0.5 * max(sm)] or sm
+    return ({"sm_mhz": statistics.median(under_load), "sm_max_mhz": mx, "reasons": sorted(reasons),
+             "samples": len(sm)}, samples)
 
 
 def source_digest(files=("fused_step.cuh",)) -> str:
@@ -586,6 +607,13 @@ def run_sweep(args):
                                                "cudaMemcpy): this box's copy rate, median of 20"}), flush=True)
     names = {Z.STEP_KERNEL_REGISTER: "register", Z.STEP_KERNEL_PIPE: "pipeline", Z.STEP_KERNEL_QUAD: "quad",
              Z.STEP_KERNEL_OCT: "oct"}
+    # SM clocks beside every point: one sampler for the whole sweep (many
+    # points time less than one sampling interval), each point given the
+    # samples taken during its timed calls or, failing that, the nearest one
+    clocks = ClockSampler(0, keep_samples=True)
+    clocks.start()
+    time.sleep(0.3)
+    windows = []
     free_gb = torch.cuda.mem_get_info()[0] / 1e9
     flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
     dtypes = [args.grad_dtype] if args.sweep_dtype_only else ["f16", "bf16"]
@@ -621,6 +649,7 @@ def run_sweep(args):
             times = []
             # median of >= 20 timed calls, >= 5 when a call moves more than 20 GB
             reps = args.steps if psi * bpe > 20e9 else max(20, args.steps)
+            w0 = time.time()
             for _ in range(reps):
                 opt.flag.zero_()
                 if small:
@@ -635,6 +664,7 @@ def run_sweep(args):
                 e1.record()
                 torch.cuda.synchronize()
                 times.append(e0.elapsed_time(e1))
+            windows.append(((psi, N, dt), w0, time.time()))
             assert int(opt.flag.item()) == 0
             ms = statistics.median(times)
             gbs = psi * bpe / (ms * 1e-3) / 1e9
@@ -649,6 +679,19 @@ def run_sweep(args):
                               else "footprint > 4x L2"}), flush=True)
             del opt
             torch.cuda.empty_cache()
+    summary = clocks.stop()
+    per_point = {}
+    for (psi, N, dt), w0, w1 in windows:
+        inside = [x for x in clocks.samples if w0 <= x[0] <= w1]
+        if not inside and clocks.samples:
+            inside = [min(clocks.samples, key=lambda x: min(abs(x[0] - w0), abs(x[0] - w1)))]
+        if inside:
+            per_point[f"{dt}/{psi}/{N}"] = {"sm_mhz": statistics.median(x[1] for x in inside),
+                                            "reasons": sorted({r for x in inside for r in x[2]}),
+                                            "samples": len(inside)}
+    print(json.dumps({"sweep": True, "clocks": summary, "clocks_by_point": per_point,
+                      "note": "SM clock per point: the samples taken during its timed calls, else the nearest"}),
+          flush=True)
     return 0
 
 

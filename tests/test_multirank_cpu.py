@@ -175,3 +175,24 @@ def test_p2p_byte_model_matches_the_pages_volumes():
     m = bench.p2p_bytes_per_rank([10], 3, 4, 2, "banks")
     assert (m["pull_bytes"], m["gather_bytes"]) == (80, 40)
     assert bench.p2p_bytes_per_rank([10], 1, 2, 2, "staged")["elements_moved"] == 0
+
+
+def test_clock_csv_parsing():
+    """bench.parse_clock_csv: median SM clock under load, max clock, the
+    throttle reasons seen, timestamps kept per sample; idle samples below half
+    the top clock left out of the median; malformed lines skipped."""
+    import bench
+    lines = [
+        "0, 1965, 1965, 900.1, 0x0, Not Active, Not Active, Not Active, Not Active, 2026/12/03 10:00:00.000\n",
+        "0, 1650, 1965, 1000.0, 0x4, Not Active, Not Active, Not Active, Active, 2026/12/03 10:00:00.100\n",
+        "0, 1700, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active, 2026/12/03 10:00:00.200\n",
+        "0, 345, 1965, 120.0, 0x0, Not Active, Not Active, Not Active, Not Active, 2026/12/03 10:00:00.300\n",
+        "garbage line\n",
+        "0, [N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active, 2026/12/03 10:00:00.400\n",
+    ]
+    summary, samples = bench.parse_clock_csv(lines)
+    assert summary == {"sm_mhz": 1700.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 4}
+    assert [s[1] for s in samples] == [1965.0, 1650.0, 1700.0, 345.0]
+    assert samples[1][2] == ["sw_power_cap"] and samples[0][2] == []
+    assert abs((samples[3][0] - samples[0][0]) - 0.3) < 1e-6
+    assert bench.parse_clock_csv([]) == (None, [])
