@@ -26,6 +26,7 @@ Other modes (each prints JSON lines of its own):
   --mode {inplace,staged}, --max-grad-norm X   the one-bank step routes, clipping
   --flat PSI --world N                         a flat workload instead of GPT-2
   --sweep                                      the flat bandwidth sweep (kernel calls alone)
+  --kernel-ab PSI --world N                    one flat point with each step kernel forced in turn
   --allgather P --world N                      the all-gather of N slices of P elements
   --stage3                                     the layer-wise ZeRO-3 step, 6.7B shape
   --distributed {banks,staged} [--stage3]      one process per GPU under torchrun (real ranks)
@@ -570,6 +571,95 @@ def run_gpu(args):
     return 0
 
 
+def run_kernel_ab(args):
+    """The fused step at one flat point (--kernel-ab PSI --world N) with each
+    step kernel forced in turn through zero_test_force_step_kernel: automatic
+    choice, register, pipeline, quad, oct.  Each call timed alone as in the
+    sweep (median of >= 20 calls, >= 5 above 20 GB, banks alternating, a
+    sleep kernel before each, L2 written over between calls below 4x L2);
+    the kernel that ran is named by zero_runner_bucket_kernel (a forced
+    kernel that cannot run the call leaves the automatic choice); each
+    kernel's outputs of one call from the same inputs are compared with the
+    automatic choice's on a strided sample.  One JSON line."""
+    import torch
+    import zero_sharded_optimizer_reduce_b200 as Z
+    torch.cuda.set_device(0)
+    peak, peak_kind = peaks()
+    psi, N = args.kernel_ab, args.world
+    if psi % N:
+        raise SystemExit("--kernel-ab needs PSI to be a multiple of --world")
+    gdt = torch.bfloat16 if args.grad_dtype == "bf16" else torch.float16
+    w = workloads.Workload(f"flat_{psi}_n{N}_{args.grad_dtype}", (psi,), N, 65536.0, 1,
+                           workloads.AdamConfig(weight_decay=0.01), seed=5)
+    opt = Z.ZeroAdam(w.numels, N, 0, lr=w.adam.lr, weight_decay=0.01, loss_scale=65536.0, grad_dtype=gdt,
+                     param_dtype=gdt)
+    fill_workload(opt, w, w.seed)
+    bpe = bytes_per_elem(N)
+    small = psi * bpe < 4 * 126e6
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda") if small else None
+    banks = [[opt.master[0][i], opt.m[0][i], opt.v[0][i]] for i in (0, 1)]
+    names = {Z.STEP_KERNEL_AUTO: "auto", Z.STEP_KERNEL_REGISTER: "register", Z.STEP_KERNEL_PIPE: "pipeline",
+             Z.STEP_KERNEL_QUAD: "quad", Z.STEP_KERNEL_OCT: "oct"}
+
+    def call(i, hp_t):
+        hp = Z.hparams(w.adam.lr, w.adam.beta1, w.adam.beta2, w.adam.eps, w.adam.weight_decay, hp_t)
+        Z.zero_reduce_scatter_adam_step(opt.grads[0], psi, Z.ZERO_ALL_PARTITIONS, *banks[i % 2], *banks[(i + 1) % 2],
+                                        opt.params_bank[0][(i + 1) % 2], hp, 65536.0, opt.flag)
+
+    def sample(x):
+        # every 997th element and the last 65,536: a cheap comparison of two
+        # kernels' outputs (the parity tests compare every element)
+        return torch.cat([x[::997].contiguous().view(torch.uint8), x[-65536:].contiguous().view(torch.uint8)])
+
+    results, ran, same = {}, {}, {}
+    reps = args.steps if psi * bpe > 20e9 else max(20, args.steps)
+    try:
+        # first one call per kernel from the same inputs (bank 0, untouched
+        # until the timing below), outputs sampled and compared with the
+        # automatic choice's
+        ref = None
+        for kind, name in names.items():
+            Z.zero_test_force_step_kernel(kind)
+            ran[name] = names[opt.bucket_kernels()[0]]
+            opt.flag.zero_()
+            call(0, 1)
+            out = [sample(x) for x in banks[1] + [opt.params_bank[0][1]]]
+            if ref is None:
+                ref = out
+            else:
+                same[name] = all(torch.equal(a, b) for a, b in zip(out, ref))
+            assert int(opt.flag.item()) == 0
+        for kind, name in names.items():
+            Z.zero_test_force_step_kernel(kind)
+            for i in range(3):
+                call(i, i + 1)
+            times = []
+            for i in range(reps):
+                opt.flag.zero_()
+                if small:
+                    flush.fill_(1)
+                torch.cuda._sleep(200_000)
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                call(i, i + 1)
+                e1.record()
+                torch.cuda.synchronize()
+                times.append(e0.elapsed_time(e1))
+            assert int(opt.flag.item()) == 0
+            ms = statistics.median(times)
+            gbs = psi * bpe / (ms * 1e-3) / 1e9
+            results[name] = {"kernel_ran": ran[name], "ms_median": ms, "gbs": gbs, "frac_measured": gbs / peak,
+                             "sample_bit_identical_to_auto": same.get(name)}
+    finally:
+        Z.zero_test_force_step_kernel(Z.STEP_KERNEL_AUTO)
+    print(json.dumps({"kernel_ab": True, "psi": psi, "world": N, "grad_dtype": args.grad_dtype,
+                      "bytes_per_elem": bpe, "reps": reps, "peak": peak, "peak_kind": peak_kind,
+                      "l2": "L2-influenced (512 MB written between calls)" if small else "footprint > 4x L2",
+                      "results": results}), flush=True)
+    return 0
+
+
 def run_sweep(args):
     """Flat bandwidth sweep: psi in {1M, 16M, 256M, 1B, 2B} x N in {1..64}
     (N x 2 x psi <= 96 GB), fp16 and bf16; one JSON line per point.  Each
@@ -1057,6 +1147,9 @@ def main(argv=None):
     ap.add_argument("--sweep-dtype-only", action="store_true", help="sweep only --grad-dtype")
     ap.add_argument("--cpu-configs", action="store_true",
                     help="time the CPU oracle on every workload (full arrays or 64M slices), one JSON line")
+    ap.add_argument("--kernel-ab", type=int, default=0,
+                    help="time the fused step on a flat bucket of this many elements (--world N) with each "
+                         "step kernel forced in turn, one JSON line")
     ap.add_argument("--allgather", type=int, default=0,
                     help="time the all-gather of --world slices of this many elements, one JSON line")
     ap.add_argument("--distributed", choices=["banks", "staged"], default=None,
@@ -1073,6 +1166,8 @@ def main(argv=None):
         return run_cpu_configs(args)
     if args.sweep:
         return run_sweep(args)
+    if args.kernel_ab:
+        return run_kernel_ab(args)
     if args.allgather:
         return run_allgather(args)
     if args.distributed is not None:

@@ -476,11 +476,12 @@ int zero_test_wait_timeout(int32_t* status, int64_t limit_ns, zero_stream_t stre
  * The paper has no counterpart: a test hook of this library.  Every fused
  * step call (zero_reduce_scatter_adam_step, its gated and no-alloc variants,
  * the runner) normally picks one of four kernels that compute the same bits:
- * the shared-memory pipeline kernel for large calls with N >= 5, the
- * oct-streaming kernel (32-byte state stores) for N <= 4, mid-size calls and
+ * the shared-memory pipeline kernel for large calls with N >= 6, the
+ * oct-streaming kernel (32-byte state stores) for N <= 2, mid-size calls and
  * peer memory when the fp32 outputs are 32-byte aligned where the vector
  * region starts, the quad-streaming kernel for those calls otherwise, the
- * register kernel for N > 20 or arrays off a common 16-byte phase.  This call
+ * register kernel for large calls with 3 <= N <= 5, N > 20 or arrays off a
+ * common 16-byte phase.  This call
  * makes the process's later calls take `kind` instead wherever that kernel
  * can run the call (the pipeline kernel needs a common phase, N <= 20, one
  * whole tile and gradients in this GPU's memory; the quad kernel a common

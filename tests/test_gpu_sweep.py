@@ -140,3 +140,34 @@ def test_every_sweep_point(dtype):
         assert int(flag.item()) == 1, f"psi={psi} N={N}: +inf at replica {k}, element {pos} not flagged"
         checked += 1
     assert checked == len(fits)
+
+
+@pytest.mark.parametrize("psi,world", [(1 << 20, 4), (8 * 1_000_003, 8), (24 * 43_691, 24)])
+def test_bench_kernel_ab_mode(psi, world):
+    """bench.py --kernel-ab: one JSON line with every kernel's timing; the
+    forced kernels that can run the call report themselves (the others the
+    automatic choice), and every kernel's sampled outputs equal the automatic
+    choice's."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "bench.py", "--kernel-ab", str(psi), "--world", str(world), "--steps", "3"],
+                       cwd=root, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    res = d["results"]
+    assert set(res) == {"auto", "register", "pipeline", "quad", "oct"}
+    assert res["register"]["kernel_ran"] == "register"
+    if world <= 16:
+        assert res["quad"]["kernel_ran"] == "quad" and res["oct"]["kernel_ran"] == "oct"
+        assert res["pipeline"]["kernel_ran"] == "pipeline"
+    else:
+        assert res["quad"]["kernel_ran"] == res["oct"]["kernel_ran"] == res["auto"]["kernel_ran"]
+    for name, v in res.items():
+        assert v["gbs"] > 0
+        if name != "auto":
+            assert v["sample_bit_identical_to_auto"] is True, name

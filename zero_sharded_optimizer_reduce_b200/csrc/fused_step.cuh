@@ -490,13 +490,14 @@ __global__ void __launch_bounds__(NT, MINB) fused_step_oct_kernel(const __grid_c
     finish_block<NT>(p, bad, sq);
 }
 
-// Shapes of the oct kernel by replica count: NT threads per block and the
-// blocks per SM its registers are sized for (no spills).
+// Shapes of the oct kernel by replica count: NT threads per block, the
+// blocks per SM its registers are sized for (no spills) and the blocks per
+// SM of the grid (several waves).
 template <int B> struct OctShape;
-template <> struct OctShape<2> { static constexpr int NT = 512, MINB = 2; };
-template <> struct OctShape<4> { static constexpr int NT = 256, MINB = 3; };
-template <> struct OctShape<8> { static constexpr int NT = 256, MINB = 2; };
-template <> struct OctShape<16> { static constexpr int NT = 256, MINB = 2; };
+template <> struct OctShape<2> { static constexpr int NT = 512, MINB = 2, BPS = 16; };
+template <> struct OctShape<4> { static constexpr int NT = 256, MINB = 3, BPS = 16; };
+template <> struct OctShape<8> { static constexpr int NT = 256, MINB = 2, BPS = 16; };
+template <> struct OctShape<16> { static constexpr int NT = 256, MINB = 2, BPS = 16; };
 
 // Shapes of the quad kernel by replica count: B replicas' loads and U quads
 // in flight per thread, NT threads per block (two or three blocks per SM at

@@ -17,7 +17,7 @@ constexpr uint32_t kPipeMinTile = 1536;             // elements: 3/4 of 4 x cons
 constexpr uint32_t kPipeSmemMax = 220u * 1024u;     // dynamic shared memory cap
 constexpr int kPipeMaxWorld = 20;                   // largest N measured to gain from the pipeline
 constexpr int64_t kPipeMinTilesPerSm = 128;         // calls with fewer tiles per SM take the oct / quad kernel
-constexpr int kOctMaxWorldAtAnySize = 4;            // N up to this takes the oct kernel at every size
+constexpr int kRegMaxWorldLarge = 5;                // large calls with 3 <= N <= this take the register kernel
 constexpr int64_t kStatsPipeMinTilesPerSm = 128;    // the same for the staged reduce-scatter
 constexpr int kStatsPipeMaxWorldWrite = 8;          // largest N whose reduce-scatter takes that pipeline
 
@@ -95,13 +95,14 @@ inline KernelFn pick_oct_b(zero_dtype_t g, zero_dtype_t pd) {
     return fused_step_oct_kernel<__nv_bfloat16, __nv_bfloat16, B, NT, M>;
 }
 
-// The oct-kernel instance for N replicas (N <= kQuadMaxWorld) and its threads
-// per block.
-inline KernelFn pick_oct_kernel(zero_dtype_t g, zero_dtype_t pd, int world, int* nt) {
-    if (world <= 2) { *nt = OctShape<2>::NT; return pick_oct_b<2>(g, pd); }
-    if (world <= 4) { *nt = OctShape<4>::NT; return pick_oct_b<4>(g, pd); }
-    if (world <= 8) { *nt = OctShape<8>::NT; return pick_oct_b<8>(g, pd); }
+// The oct-kernel instance for N replicas (N <= kQuadMaxWorld), its threads
+// per block and the blocks per SM of its grid.
+inline KernelFn pick_oct_kernel(zero_dtype_t g, zero_dtype_t pd, int world, int* nt, int* bps) {
+    if (world <= 2) { *nt = OctShape<2>::NT; *bps = OctShape<2>::BPS; return pick_oct_b<2>(g, pd); }
+    if (world <= 4) { *nt = OctShape<4>::NT; *bps = OctShape<4>::BPS; return pick_oct_b<4>(g, pd); }
+    if (world <= 8) { *nt = OctShape<8>::NT; *bps = OctShape<8>::BPS; return pick_oct_b<8>(g, pd); }
     *nt = OctShape<16>::NT;
+    *bps = OctShape<16>::BPS;
     return pick_oct_b<16>(g, pd);
 }
 
@@ -389,22 +390,27 @@ inline int prepare_step(const char* fn, const void* const* grad_bufs, int32_t wo
     }
 
     // Kernel choice (measured on B200 against a measured copy rate of
-    // 6.43 TB/s, L2 cold):
+    // 6.43 TB/s, L2 cold, each call alone, each kernel forced in turn):
     //  - arrays whose 16-byte phases never coincide, or N > kPipeMaxWorld: the
     //    register kernel (its scalar path when unaligned; at N = 64 it runs at
     //    the copy rate);
-    //  - N <= 16 streams: the oct kernel when the fp32 outputs are 32-byte
-    //    aligned at the vector region (its 32-byte stores: N = 1 / 2 at 256M
-    //    and 1B elements 1.00-1.02 against 0.98-0.99 for the quad kernel;
-    //    N = 4 at 256M 1.01 against 0.99 for the pipeline), else the quad
-    //    kernel; they take N <= kOctMaxWorldAtAnySize (2 for the quad kernel)
-    //    at every size, calls below kPipeMinTilesPerSm tiles per SM (no
-    //    pipeline to fill and drain: 16M elements at N = 1..16, 0.97-1.04
-    //    against 0.82-1.04) and gradients in another GPU's memory;
+    //  - 3 <= N <= kRegMaxWorldLarge with at least kPipeMinTilesPerSm tiles
+    //    per SM: the register kernel (256M-1B elements, N = 3 / 4 / 5:
+    //    1.01-1.02 / 1.03 / 1.02 against 1.00-1.01 for the oct kernel and
+    //    0.96-1.02 for the pipeline; the cause was not isolated: the oct
+    //    kernel with the register kernel's grid, store width, load form or
+    //    load order measured the same);
+    //  - N <= 16 streams otherwise: the oct kernel when the fp32 outputs are
+    //    32-byte aligned at the vector region (its 32-byte stores: N = 1 / 2 at
+    //    256M and 1B elements 1.00-1.02 against 0.98-0.99 for the quad kernel
+    //    and 0.96-0.99 for the register kernel), else the quad kernel; they
+    //    take N <= 2 at every size, calls below kPipeMinTilesPerSm tiles per
+    //    SM (no pipeline to fill and drain: 16M elements at N = 1..16,
+    //    0.96-1.04 against 0.82-1.04) and gradients in another GPU's memory;
     //  - otherwise, with every gradient buffer in this GPU's memory, the
     //    pipeline kernel (its bulk copies never read another GPU's memory;
-    //    N = 8 / 16 at 256M: 1.05 / 1.09-1.10 against 1.04 / 1.08 for the oct
-    //    kernel);
+    //    N = 8 / 16 at 256M-1B: 1.04-1.08 / 1.09-1.10 against 1.03-1.04 /
+    //    1.08 for the oct kernel);
     //  - 17 <= N <= 20 calls below the pipeline threshold: the pipeline kernel
     //    when the gradients are local and every SM gets two tiles, else the
     //    register kernel.
@@ -426,8 +432,9 @@ inline int prepare_step(const char* fn, const void* const* grad_bufs, int32_t wo
         const bool quad_ok = world <= kQuadMaxWorld;
         const bool big = ntiles >= kPipeMinTilesPerSm * static_cast<int64_t>(sms);
         const int stream_kind = prm.st32 ? kKindOct : kKindQuad;
-        const bool small_n = world <= (prm.st32 ? kOctMaxWorldAtAnySize : 2);
-        if (quad_ok && (small_n || !big)) {
+        if (big && world >= 3 && world <= kRegMaxWorldLarge) {
+            kind = kKindRegister;
+        } else if (quad_ok && (world <= 2 || !big)) {
             kind = stream_kind;
         } else if (all_local_device_memory(grad_bufs, world)) {   // queried only where it decides
             if (big || ntiles >= 2 * static_cast<int64_t>(sms)) kind = kKindPipe;
@@ -441,10 +448,10 @@ inline int prepare_step(const char* fn, const void* const* grad_bufs, int32_t wo
     if (force == kKindOct && h >= 0 && world <= kQuadMaxWorld && prm.st32) kind = kKindOct;
     if (kind == kKindOct) {
         prm.kind = kKindOct;
-        int nt = 0;
-        (void)pick_oct_kernel(grad_dtype, param_dtype, world, &nt);
+        int nt = 0, bps = 0;
+        (void)pick_oct_kernel(grad_dtype, param_dtype, world, &nt, &bps);
         blocks = (prm.nvec + nt - 1) / nt;
-        int64_t cap = static_cast<int64_t>(sms) * kQuadBlocksPerSm;
+        int64_t cap = static_cast<int64_t>(sms) * bps;
         if (cap > kMaxBlocks) cap = kMaxBlocks;   // one norm partial per block in the workspace
         if (blocks > cap) blocks = cap;
         if (blocks < 1) blocks = 1;
@@ -712,8 +719,8 @@ inline int launch_step(const char* fn, const StepParams& prm, int64_t blocks, ze
         KernelFn k = pick_quad_kernel(grad_dtype, param_dtype, prm.world, &nt, &u);
         k<<<static_cast<unsigned int>(blocks), nt, 0, s>>>(prm);
     } else if (prm.kind == kKindOct) {
-        int nt = 0;
-        KernelFn k = pick_oct_kernel(grad_dtype, param_dtype, prm.world, &nt);
+        int nt = 0, bps = 0;
+        KernelFn k = pick_oct_kernel(grad_dtype, param_dtype, prm.world, &nt, &bps);
         k<<<static_cast<unsigned int>(blocks), nt, 0, s>>>(prm);
     } else {
         pick_kernel(grad_dtype, param_dtype)<<<static_cast<unsigned int>(blocks), kThreads, 0, s>>>(prm);
