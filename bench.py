@@ -26,7 +26,8 @@ Other modes (each prints JSON lines of its own):
   --mode {inplace,staged}, --max-grad-norm X   the one-bank step routes, clipping
   --flat PSI --world N                         a flat workload instead of GPT-2
   --sweep                                      the flat bandwidth sweep (kernel calls alone)
-  --kernel-ab PSI --world N                    one flat point with each step kernel forced in turn
+  --kernel-ab PSI --world N [--mode staged]    one flat point with each step kernel forced in turn
+                                               (--mode staged: the one-bank routes' passes)
   --allgather P --world N                      the all-gather of N slices of P elements
   --stage3                                     the layer-wise ZeRO-3 step, 6.7B shape
   --distributed {banks,staged} [--stage3]      one process per GPU under torchrun (real ranks)
@@ -568,6 +569,106 @@ def run_gpu(args):
     if world_gpus > 1:
         dist.barrier()
         dist.destroy_process_group()
+    return 0
+
+
+def run_kernel_ab_passes(args):
+    """--kernel-ab PSI --world N with --mode staged or inplace: the passes of
+    the one-bank routes with each kernel forced in turn -- the staged
+    reduce-scatter (gradients in, fp32 reduced gradients out, 2N + 4 B/elem),
+    the statistics pass (gradients in, flag and norm out, 2N) and the staged
+    update (reduced gradients and states in, states and parameters out, 30).
+    Each call timed alone as in --kernel-ab; each kernel's reduced gradients,
+    flag and norm compared with the automatic choice's (the norm within two
+    fp64 summation orders).  One JSON line."""
+    import torch
+    import zero_sharded_optimizer_reduce_b200 as Z
+    torch.cuda.set_device(0)
+    peak, peak_kind = peaks()
+    psi, N = args.kernel_ab, args.world
+    if psi % N:
+        raise SystemExit("--kernel-ab needs PSI to be a multiple of --world")
+    gdt = torch.bfloat16 if args.grad_dtype == "bf16" else torch.float16
+    gen = torch.Generator(device="cuda")
+    grads = []
+    for k in range(N):
+        gen.manual_seed(workloads.seed_for(5, 1, k))
+        g = torch.empty(psi, dtype=gdt, device="cuda")
+        for o in range(0, psi, 1 << 27):
+            e = min(psi, o + (1 << 27))
+            g[o:e].copy_(torch.randn(e - o, generator=gen, device="cuda").mul_(1e-3 * 65536.0))
+        grads.append(g)
+    red = torch.empty(psi, device="cuda")
+    st = [torch.randn(psi, device="cuda", generator=gen).mul_(0.02), torch.zeros(psi, device="cuda"),
+          torch.zeros(psi, device="cuda")]
+    par = torch.empty(psi, dtype=gdt, device="cuda")
+    flags = torch.zeros(2, dtype=torch.int32, device="cuda")
+    sq = torch.zeros(1, dtype=torch.float64, device="cuda")
+    ws = torch.zeros(Z.zero_step_workspace_bytes(), dtype=torch.uint8, device="cuda")
+    hp = Z.hparams(1e-3, 0.9, 0.999, 1e-8, 0.01, 1)
+    small = psi * (2 * N + 4) < 4 * 126e6
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda") if small else None
+    names = {Z.STEP_KERNEL_AUTO: "auto", Z.STEP_KERNEL_REGISTER: "register", Z.STEP_KERNEL_PIPE: "pipeline",
+             Z.STEP_KERNEL_QUAD: "quad", Z.STEP_KERNEL_OCT: "oct"}
+    passes = {
+        "reduce_scatter": (2 * N + 4, lambda: Z.zero_reduce_scatter_grads(grads, psi, -1, 65536.0, red, flags[0:1],
+                                                                          sq, ws)),
+        "statistics": (2 * N, lambda: Z.zero_grad_stats(grads, psi, -1, 65536.0, flags[0:1], sq, ws)),
+        "update": (30, lambda: Z.zero_adam_step_reduced(red, psi, *st, *st, par, hp, flags[1:2])),
+    }
+    reps = args.steps if psi * (2 * N + 4) > 20e9 else max(20, args.steps)
+    out = {}
+    try:
+        # agreement: the reduced gradients, flag and norm of each kernel's
+        # reduce-scatter against the automatic choice's
+        ref = None
+        agree = {}
+        for kind, name in names.items():
+            Z.zero_test_force_step_kernel(kind)
+            flags.zero_()
+            sq.zero_()
+            passes["reduce_scatter"][1]()
+            torch.cuda.synchronize()
+            got = (red[::997].clone(), red[-65536:].clone(), int(flags[0].item()), float(sq.item()))
+            if ref is None:
+                ref = got
+            else:
+                agree[name] = (torch.equal(got[0].view(torch.int32), ref[0].view(torch.int32)) and
+                               torch.equal(got[1].view(torch.int32), ref[1].view(torch.int32)) and
+                               got[2] == ref[2] and abs(got[3] - ref[3]) <= 2.0 * psi * 2.0 ** -53 * ref[3])
+        for pname, (bpe, fn) in passes.items():
+            res = {}
+            for kind, name in names.items():
+                Z.zero_test_force_step_kernel(kind)
+                for _ in range(3):
+                    fn()
+                times = []
+                for _ in range(reps):
+                    flags.zero_()
+                    if small:
+                        flush.fill_(1)
+                    torch.cuda._sleep(200_000)
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    fn()
+                    e1.record()
+                    torch.cuda.synchronize()
+                    times.append(e0.elapsed_time(e1))
+                assert int(flags[0].item()) == 0 and int(flags[1].item()) == 0
+                ms = statistics.median(times)
+                gbs = psi * bpe / (ms * 1e-3) / 1e9
+                res[name] = {"ms_median": ms, "gbs": gbs, "frac_measured": gbs / peak}
+            out[pname] = {"bytes_per_elem": bpe, "results": res}
+    finally:
+        Z.zero_test_force_step_kernel(Z.STEP_KERNEL_AUTO)
+    print(json.dumps({"kernel_ab": True, "passes": True, "psi": psi, "world": N, "grad_dtype": args.grad_dtype,
+                      "reps": reps, "peak": peak, "peak_kind": peak_kind,
+                      "reduce_scatter_agrees_with_auto": agree,
+                      "note": "a forced kernel that cannot run a call leaves that call's automatic choice; the "
+                              "staged update has register and pipeline versions only",
+                      "l2": "L2-influenced (512 MB written between calls)" if small else "footprint > 4x L2",
+                      "passes_timed": out}), flush=True)
     return 0
 
 
@@ -1167,7 +1268,7 @@ def main(argv=None):
     if args.sweep:
         return run_sweep(args)
     if args.kernel_ab:
-        return run_kernel_ab(args)
+        return run_kernel_ab_passes(args) if args.mode != "banks" else run_kernel_ab(args)
     if args.allgather:
         return run_allgather(args)
     if args.distributed is not None:

@@ -171,3 +171,27 @@ def test_bench_kernel_ab_mode(psi, world):
         assert v["gbs"] > 0
         if name != "auto":
             assert v["sample_bit_identical_to_auto"] is True, name
+
+
+@pytest.mark.parametrize("world", [2, 8])
+def test_bench_kernel_ab_passes_mode(world):
+    """bench.py --kernel-ab --mode staged: the reduce-scatter, statistics and
+    update passes timed under every kernel; every kernel's reduce-scatter
+    output, flag and norm agree with the automatic choice's."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "bench.py", "--kernel-ab", str(world * 131_072), "--world", str(world),
+                        "--mode", "staged", "--steps", "3"], cwd=root, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert set(d["passes_timed"]) == {"reduce_scatter", "statistics", "update"}
+    for p in d["passes_timed"].values():
+        assert set(p["results"]) == {"auto", "register", "pipeline", "quad", "oct"}
+        assert all(v["gbs"] > 0 for v in p["results"].values())
+    assert set(d["reduce_scatter_agrees_with_auto"]) == {"register", "pipeline", "quad", "oct"}
+    assert all(d["reduce_scatter_agrees_with_auto"].values())
