@@ -18,6 +18,9 @@ benchmark times (every rank's partition in one launch per bucket).
 - Flat bandwidth-sweep points: windows.
 - The staged route on a bucket past 2^31 elements (64-bit indexing) and on a
   bf16 N = 16 point: windows of the reduced gradients, states, parameters.
+- The native runner with buckets that take different step kernels in one
+  step (pipeline or register beside oct): windows over two steps, then a
+  skipped step that leaves every bank bit-identical.
 """
 import numpy as np
 import pytest
@@ -314,3 +317,60 @@ def test_staged_windows_beyond_int32(psi, world, dtype):
         assert assert_f32_close(host_f32(st["m"][lo:hi]), ref.m, "m") == 0
         assert assert_f32_close(host_f32(st["v"][lo:hi]), ref.v, "v") == 0
         assert assert_u16_close(_u16(params[lo:hi]), ref.params, "params") == 0
+
+
+@pytest.mark.skipif(not torch.cuda.is_available() or _free_gb() < 12, reason="needs ~6 GB of HBM")
+@pytest.mark.parametrize("numels,world,kinds", [
+    ([64 << 20, 1 << 20, 240_007], 8, [Z.STEP_KERNEL_PIPE, Z.STEP_KERNEL_OCT]),
+    ([88 << 20, 1 << 20], 4, [Z.STEP_KERNEL_REGISTER, Z.STEP_KERNEL_OCT]),
+])
+def test_runner_step_with_mixed_kernels(numels, world, kinds):
+    """One native-runner step whose buckets take different kernels (the
+    pipeline or the register kernel on a large bucket, the oct kernel on a
+    small one), sharing one overflow flag: windows against the oracle over two
+    steps; then an inf in the small bucket skips the whole step, every bank
+    bit-identical."""
+    adam = workloads.AdamConfig(weight_decay=0.01)
+    opt = Z.ZeroAdam(numels, world, 64 << 20 if world == 8 else 88 << 20, lr=adam.lr, weight_decay=adam.weight_decay,
+                     loss_scale=65536.0)
+    L = opt.layout
+    assert opt.bucket_kernels() == kinds
+    wins, refs = [], []
+    for b in range(L.n_buckets):
+        _device_master(opt.master[b][0], 900 + b)
+        opt.master[b][0][L.bucket_numel[b]:].zero_()
+        opt.params_bank[b][0].copy_(opt.master[b][0])
+        opt.master[b][1].copy_(opt.master[b][0])
+        opt.params_bank[b][1].copy_(opt.params_bank[b][0])
+        wb = _windows(L.bucket_padded[b], world, n_random=8, seed=50 + b)
+        wins.append(wb)
+        refs.append([oracle.FlatState(host_f32(opt.master[b][0][lo:hi]).copy(), np.zeros(hi - lo, np.float32),
+                                      np.zeros(hi - lo, np.float32), _u16(opt.params_bank[b][0][lo:hi]).copy())
+                     for lo, hi in wb])
+    for step in (1, 2):
+        win_grads = []
+        for b in range(L.n_buckets):
+            for k in range(world):
+                _device_grads(opt.grads[b][k], 7000 + 100 * step + 10 * b + k, 1e-3, 65536.0)
+                opt.grads[b][k][L.bucket_numel[b]:].zero_()
+            win_grads.append([[_u16(opt.grads[b][k][lo:hi]) for k in range(world)] for lo, hi in wins[b]])
+        assert opt.step()
+        for b in range(L.n_buckets):
+            for G, st in zip(win_grads[b], refs[b]):
+                assert oracle.flat_step(G, st, adam, step, 65536.0, float(world))[0] == 0
+    for b in range(L.n_buckets):
+        master, m, v, p = opt.state(b)
+        for (lo, hi), st in zip(wins[b], refs[b]):
+            assert assert_f32_close(host_f32(master[lo:hi]), st.master, "master") == 0
+            assert assert_f32_close(host_f32(m[lo:hi]), st.m, "m") == 0
+            assert assert_f32_close(host_f32(v[lo:hi]), st.v, "v") == 0
+            assert assert_u16_close(_u16(p[lo:hi]), st.params, "params") == 0
+    # an inf in the last bucket's last replica: nothing in any bucket changes
+    before = [[x.clone() for x in opt.state(b)] for b in range(L.n_buckets)]
+    small = L.n_buckets - 1
+    opt.grads[small][world - 1][12345] = float("inf")
+    assert not opt.step()
+    assert opt.t == 2 and opt.scale == 32768.0
+    for b in range(L.n_buckets):
+        for x, y in zip(opt.state(b), before[b]):
+            assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
